@@ -1,0 +1,364 @@
+/*
+ * lightning_oracle.c -- plain, slow, fp64 CPU oracle for Lightning Attention
+ * (blocked causal linear attention).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link,
+ * load or call this file: only the test suite, the smoke check of the entry
+ * module and the CPU-baseline leg of the benchmark use it.  It shares no code,
+ * header, table or helper with the CUDA library; both sides only receive the
+ * same seeded input bits.
+ *
+ * Every input value is a bf16 bit pattern (uint16) and is widened exactly to
+ * double; all arithmetic is fp64 with plain loops in the order the definitions
+ * state.  OpenMP splits the independent (sequence, head) pairs across threads;
+ * nothing inside one pair is blocked, fused or reordered beyond the definition.
+ *
+ * Sources (web pages on the MiniMax-01 report):
+ *   [P2] "MiniMax-01技术报告解读（一）模型架构" (blog.csdn.net), §2.2 线性注意力:
+ *        the right-product kernel trick with a recursively updated KV product;
+ *        intra-block left product, inter-block right product; Q/K/V split into
+ *        row blocks.
+ *   [P5] "MiniMax-01技术报告解读" (qingkelab.github.io), §2.2 (same text as P2),
+ *        §3.2 item 3 (LASP+: local prefix KV_t, AllGather, global prefix KV_G),
+ *        §3.2 item 1 (data packing: samples joined end to end),
+ *        §3.3 items 1-2 (decode: length-1 tokens, KV update fused with the
+ *        prefix-KV cache).
+ *   The pages print no formula; the formula used is the plainest reading of
+ *   that prose: O = (Q K^T ⊙ M) V with the inclusive causal mask
+ *   M[t][s] = 1 iff s <= t, no scale, feature map, normalisation or decay
+ *   inside the operation, and state S[i][j] = sum_s k_s[i] v_s[j]
+ *   (d_k rows x d_v columns).
+ *
+ * Layouts (all row-major, token-major packing as in [P5] §3.2 item 1):
+ *   q, k, v     : uint16 bf16 bits [T][H][d]; sequence i owns tokens
+ *                 [cu_seqlens[i], cu_seqlens[i+1]).
+ *   heads       : the nh head indices to compute (NULL = all H, in order).
+ *   state_in    : double [nseq][nh][d][d] or NULL (= zero state).
+ *   out         : double [T][nh][d].
+ *   state_out   : double [nseq][nh][d][d] or NULL.
+ * Every function returns 0 on success and -1 on an invalid argument.
+ *
+ * Parity status: every function here is pinned by the CPU test suite against
+ * closed forms, exact-integer library routines and brute force (see the
+ * test files); none is "parity unpinned".
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 is the upper half of an IEEE binary32; the widening is exact. */
+static double widen_bf16(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int check_common(const int32_t *cu, int nseq, int H, int d,
+                        const int32_t *heads, int nh)
+{
+    if (!cu || nseq < 0 || H <= 0 || d <= 0 || nh <= 0) return -1;
+    if (cu[0] != 0) return -1;
+    for (int i = 0; i < nseq; ++i)
+        if (cu[i + 1] < cu[i]) return -1;
+    if (heads)
+        for (int j = 0; j < nh; ++j)
+            if (heads[j] < 0 || heads[j] >= H) return -1;
+    if (!heads && nh != H) return -1;
+    return 0;
+}
+
+static void set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+int lao_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Pointer to the d-vector of token t, head h in a [T][H][d] array. */
+#define ROW(x, t, h) ((x) + ((size_t)(t) * (size_t)H + (size_t)(h)) * (size_t)d)
+
+/*
+ * Recurrent form ([P2]/[P5] §2.2: "the KV product is updated recursively"):
+ *   S_0 = S_in,  S_t = S_{t-1} + k_t^T v_t,  o_t = q_t S_t.
+ * The state after token t includes token t, so o_t sees s <= t (inclusive).
+ */
+int lao_recurrent(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  const int32_t *cu_seqlens, int nseq, int H, int d,
+                  const int32_t *heads, int nh, const double *state_in,
+                  double *out, double *state_out, int nthreads)
+{
+    if (!q || !k || !v || !out) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        double *S = (double *)calloc((size_t)d * d, sizeof(double));
+        double *kt = (double *)malloc((size_t)d * sizeof(double));
+        double *vt = (double *)malloc((size_t)d * sizeof(double));
+        double *qt = (double *)malloc((size_t)d * sizeof(double));
+        if (!S || !kt || !vt || !qt) {
+            bad = 1;
+            free(S); free(kt); free(vt); free(qt);
+            continue;
+        }
+        if (state_in)
+            memcpy(S, state_in + (size_t)p * d * d, (size_t)d * d * sizeof(double));
+        for (int t = cu_seqlens[i]; t < cu_seqlens[i + 1]; ++t) {
+            for (int a = 0; a < d; ++a) {
+                qt[a] = widen_bf16(ROW(q, t, h)[a]);
+                kt[a] = widen_bf16(ROW(k, t, h)[a]);
+                vt[a] = widen_bf16(ROW(v, t, h)[a]);
+            }
+            /* S_t = S_{t-1} + k_t^T v_t */
+            for (int a = 0; a < d; ++a)
+                for (int b = 0; b < d; ++b)
+                    S[(size_t)a * d + b] += kt[a] * vt[b];
+            /* o_t = q_t S_t */
+            double *o = out + ((size_t)t * nh + j) * d;
+            for (int b = 0; b < d; ++b) o[b] = 0.0;
+            for (int a = 0; a < d; ++a)
+                for (int b = 0; b < d; ++b)
+                    o[b] += qt[a] * S[(size_t)a * d + b];
+        }
+        if (state_out)
+            memcpy(state_out + (size_t)p * d * d, S, (size_t)d * d * sizeof(double));
+        free(S); free(kt); free(vt); free(qt);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Quadratic (masked, left-product) form, spec definition
+ * O = (Q K^T ⊙ M) V with M[t][s] = 1 iff s <= t; a carried-in state adds
+ * q_t S_in to every row.
+ *   o_t = sum_{s <= t} (q_t . k_s) v_s + q_t S_in
+ */
+int lao_quadratic(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  const int32_t *cu_seqlens, int nseq, int H, int d,
+                  const int32_t *heads, int nh, const double *state_in,
+                  double *out, double *state_out, int nthreads)
+{
+    if (!q || !k || !v || !out) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        const int t0 = cu_seqlens[i], t1 = cu_seqlens[i + 1];
+        const double *Sin = state_in ? state_in + (size_t)p * d * d : NULL;
+        for (int t = t0; t < t1; ++t) {
+            double *o = out + ((size_t)t * nh + j) * d;
+            for (int b = 0; b < d; ++b) o[b] = 0.0;
+            for (int s = t0; s <= t; ++s) {
+                double score = 0.0;                  /* (Q K^T)[t][s] */
+                for (int a = 0; a < d; ++a)
+                    score += widen_bf16(ROW(q, t, h)[a]) * widen_bf16(ROW(k, s, h)[a]);
+                for (int b = 0; b < d; ++b)
+                    o[b] += score * widen_bf16(ROW(v, s, h)[b]);
+            }
+            if (Sin)
+                for (int a = 0; a < d; ++a) {
+                    const double qa = widen_bf16(ROW(q, t, h)[a]);
+                    for (int b = 0; b < d; ++b) o[b] += qa * Sin[(size_t)a * d + b];
+                }
+        }
+        if (state_out) {
+            /* final state: S_in + K^T V over the whole sequence */
+            double *S = state_out + (size_t)p * d * d;
+            for (size_t e = 0; e < (size_t)d * d; ++e) S[e] = Sin ? Sin[e] : 0.0;
+            for (int s = t0; s < t1; ++s)
+                for (int a = 0; a < d; ++a) {
+                    const double ka = widen_bf16(ROW(k, s, h)[a]);
+                    for (int b = 0; b < d; ++b)
+                        S[(size_t)a * d + b] += ka * widen_bf16(ROW(v, s, h)[b]);
+                }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Blocked form ([P2]/[P5] §2.2): Q, K, V are split along the sequence into row
+ * blocks of `block` tokens (the last block of a sequence may be shorter).
+ * Within block b the left product is used, across blocks the right product:
+ *   O_b     = (Q_b K_b^T ⊙ M_b) V_b + Q_b S_{<b}
+ *   S_{<=b} = S_{<b} + K_b^T V_b,          S_{<0} = S_in.
+ */
+static void blocked_one(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        int H, int d, int h, int j, int nh, int t0, int t1,
+                        int block, double *S, double *out)
+{
+    for (int b0 = t0; b0 < t1; b0 += block) {
+        const int b1 = (b0 + block < t1) ? b0 + block : t1;
+        for (int t = b0; t < b1; ++t) {
+            double *o = out + ((size_t)t * nh + j) * d;
+            for (int b = 0; b < d; ++b) o[b] = 0.0;
+            /* intra-block left product (Q_b K_b^T ⊙ M_b) V_b */
+            for (int s = b0; s <= t; ++s) {
+                double score = 0.0;
+                for (int a = 0; a < d; ++a)
+                    score += widen_bf16(ROW(q, t, h)[a]) * widen_bf16(ROW(k, s, h)[a]);
+                for (int b = 0; b < d; ++b)
+                    o[b] += score * widen_bf16(ROW(v, s, h)[b]);
+            }
+            /* inter-block right product Q_b S_{<b} */
+            for (int a = 0; a < d; ++a) {
+                const double qa = widen_bf16(ROW(q, t, h)[a]);
+                for (int b = 0; b < d; ++b) o[b] += qa * S[(size_t)a * d + b];
+            }
+        }
+        /* S_{<=b} = S_{<b} + K_b^T V_b */
+        for (int s = b0; s < b1; ++s)
+            for (int a = 0; a < d; ++a) {
+                const double ka = widen_bf16(ROW(k, s, h)[a]);
+                for (int b = 0; b < d; ++b)
+                    S[(size_t)a * d + b] += ka * widen_bf16(ROW(v, s, h)[b]);
+            }
+    }
+}
+
+int lao_blocked(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                const int32_t *cu_seqlens, int nseq, int H, int d,
+                const int32_t *heads, int nh, int block, const double *state_in,
+                double *out, double *state_out, int nthreads)
+{
+    if (!q || !k || !v || !out || block <= 0) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        double *S = (double *)calloc((size_t)d * d, sizeof(double));
+        if (!S) { bad = 1; continue; }
+        if (state_in)
+            memcpy(S, state_in + (size_t)p * d * d, (size_t)d * d * sizeof(double));
+        blocked_one(q, k, v, H, d, h, j, nh, cu_seqlens[i], cu_seqlens[i + 1],
+                    block, S, out);
+        if (state_out)
+            memcpy(state_out + (size_t)p * d * d, S, (size_t)d * d * sizeof(double));
+        free(S);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Segmented form, the LASP+ recipe of [P5] §3.2 item 3 applied to the
+ * segments of one sequence instead of to ranks:
+ *   1. every segment r (seg_len tokens, the last one shorter) computes its
+ *      local KV sum KV_r = sum_{s in r} k_s^T v_s;
+ *   2. the local sums are gathered;
+ *   3. segment r forms its global prefix KV_G(r) = S_in + sum_{r' < r} KV_r'
+ *      and runs the blocked form over its own tokens starting from it.
+ * The final state is KV_G(last) + KV_last.
+ */
+int lao_segmented(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                  const int32_t *cu_seqlens, int nseq, int H, int d,
+                  const int32_t *heads, int nh, int seg_len, int block,
+                  const double *state_in, double *out, double *state_out,
+                  int nthreads)
+{
+    if (!q || !k || !v || !out || block <= 0 || seg_len <= 0) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        const int t0 = cu_seqlens[i], t1 = cu_seqlens[i + 1];
+        const int nseg = (t1 - t0 + seg_len - 1) / seg_len;
+        const size_t dd = (size_t)d * d;
+        /* step 1: local sums, one per segment (the "gathered" array of step 2) */
+        double *local = (double *)calloc((size_t)(nseg > 0 ? nseg : 1) * dd, sizeof(double));
+        double *G = (double *)malloc(dd * sizeof(double));
+        if (!local || !G) { bad = 1; free(local); free(G); continue; }
+        for (int r = 0; r < nseg; ++r) {
+            const int s0 = t0 + r * seg_len;
+            const int s1 = (s0 + seg_len < t1) ? s0 + seg_len : t1;
+            double *L = local + (size_t)r * dd;
+            for (int s = s0; s < s1; ++s)
+                for (int a = 0; a < d; ++a) {
+                    const double ka = widen_bf16(ROW(k, s, h)[a]);
+                    for (int b = 0; b < d; ++b)
+                        L[(size_t)a * d + b] += ka * widen_bf16(ROW(v, s, h)[b]);
+                }
+        }
+        /* step 3: each segment's global prefix, then its blocked scan */
+        for (int r = 0; r < nseg; ++r) {
+            for (size_t e = 0; e < dd; ++e)
+                G[e] = state_in ? state_in[(size_t)p * dd + e] : 0.0;
+            for (int r2 = 0; r2 < r; ++r2)
+                for (size_t e = 0; e < dd; ++e) G[e] += local[(size_t)r2 * dd + e];
+            const int s0 = t0 + r * seg_len;
+            const int s1 = (s0 + seg_len < t1) ? s0 + seg_len : t1;
+            blocked_one(q, k, v, H, d, h, j, nh, s0, s1, block, G, out);
+        }
+        if (state_out) {
+            double *So = state_out + (size_t)p * dd;
+            for (size_t e = 0; e < dd; ++e)
+                So[e] = state_in ? state_in[(size_t)p * dd + e] : 0.0;
+            for (int r = 0; r < nseg; ++r)
+                for (size_t e = 0; e < dd; ++e) So[e] += local[(size_t)r * dd + e];
+        }
+        free(local); free(G);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * One decode step on a persistent state ([P5] §3.3 items 1-2: length-1 tokens
+ * go to their own kernel, whose KV computation is fused with the update of
+ * the prefix-KV cache).  For every (b, h):
+ *   S <- S + k^T v,   o = q S          (inclusive: the new token sees itself)
+ * q, k, v: bf16 bits [B][H][d]; state: double [B][H][d][d] updated in place;
+ * out: double [B][H][d].
+ */
+int lao_decode_step(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                    int B, int H, int d, double *state, double *out, int nthreads)
+{
+    if (!q || !k || !v || !state || !out || B < 0 || H <= 0 || d <= 0) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)B * H;
+#pragma omp parallel for schedule(static)
+    for (long p = 0; p < npairs; ++p) {
+        double *S = state + (size_t)p * d * d;
+        const uint16_t *qp = q + (size_t)p * d, *kp = k + (size_t)p * d, *vp = v + (size_t)p * d;
+        for (int a = 0; a < d; ++a) {
+            const double ka = widen_bf16(kp[a]);
+            for (int b = 0; b < d; ++b) S[(size_t)a * d + b] += ka * widen_bf16(vp[b]);
+        }
+        double *o = out + (size_t)p * d;
+        for (int b = 0; b < d; ++b) o[b] = 0.0;
+        for (int a = 0; a < d; ++a) {
+            const double qa = widen_bf16(qp[a]);
+            for (int b = 0; b < d; ++b) o[b] += qa * S[(size_t)a * d + b];
+        }
+    }
+    return 0;
+}
