@@ -1,0 +1,178 @@
+/*
+ * lightning_attn.h -- C ABI of the B200 (sm_100a) Lightning Attention library.
+ *
+ * Lightning Attention is blocked causal linear attention.  Per sequence and
+ * head, with q_t, k_t, v_t row vectors of length d:
+ *
+ *     o_t = sum_{s <= t} (q_t . k_s) v_s + q_t S_in          O = (Q K^T ⊙ M) V
+ *     S   = S_in + sum_s k_s^T v_s        S[i][j] = S_in[i][j] + sum_s k_s[i] v_s[j]
+ *
+ * computed blockwise: inside a block of rows the left product (Q_b K_b^T ⊙ M) V_b,
+ * across blocks the right product Q_b S_{<b}, with the running d x d state
+ * updated by S += K_b^T V_b ("MiniMax-01技术报告解读", §2.2 线性注意力: the
+ * right-product kernel trick, the recursively updated KV product, intra-block
+ * left product and inter-block right product over row blocks of Q/K/V).
+ * No scale, feature map, normalisation or decay is applied inside the
+ * operation: callers pass q/k/v already scaled.
+ *
+ * Conventions shared by every entry point
+ *   - Ownership: the caller allocates and owns every buffer (inputs, outputs,
+ *     states, workspace).  Only the functions that say so read host memory.
+ *   - Asynchrony: device work is enqueued on `stream` and the call returns
+ *     without waiting.  Nothing synchronises except la_get_device_status.
+ *   - Errors: argument, shape and size errors are returned synchronously with
+ *     nothing launched.  A failed launch returns LA_ERR_CUDA.  Problems found
+ *     on the device (an invalid cu_seqlens array, a bounded wait that ran out)
+ *     are recorded in a sticky per-device word that la_get_device_status
+ *     returns; the kernels never trap and every device-side wait is bounded.
+ *   - Shapes: only head dimension d = 128 is built (other d: LA_ERR_UNSUPPORTED).
+ *     Every device pointer must be 16-byte aligned, the workspace 256-byte aligned.
+ *   - Dtypes: q, k, v are bf16; accumulation is fp32 on the tensor cores; the
+ *     output is bf16 or fp32 (la_dtype); states are fp32.
+ */
+#ifndef LIGHTNING_ATTN_H
+#define LIGHTNING_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARGUMENT = 1, /* bad pointer, shape, alignment or dtype        */
+    LA_ERR_UNSUPPORTED = 2,      /* valid but not built (d != 128, block != 128)  */
+    LA_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed          */
+    LA_ERR_TIMEOUT = 4,          /* a bounded device-side wait ran out            */
+    LA_ERR_WORKSPACE = 5         /* workspace missing or smaller than required    */
+} la_status;
+
+typedef enum { LA_BF16 = 0, LA_FP32 = 1 } la_dtype;
+
+/* Row-block length the kernels use when `block` is 0.  Row blocks are the
+ * units of the blocked algorithm; the result does not depend on the block
+ * length except through rounding. */
+#define LA_DEFAULT_BLOCK 128
+
+/* ---------------------------------------------------------------------------
+ * Prefill of B equal-length sequences.
+ *
+ *   q, k, v    device, bf16, [B, N, H, d] contiguous (token-major, heads inner).
+ *   block      row-block length: 0 (= LA_DEFAULT_BLOCK) or 128.
+ *   state_in   device fp32 [B, H, d, d] (row i = key feature, column j = value
+ *              feature) carried-in state, or NULL for a zero state.
+ *   out        device, [B, N, H, d], dtype out_dtype.
+ *   state_out  device fp32 [B, H, d, d] final state, or NULL.  May be the same
+ *              pointer as state_in (updated in place); any other overlap with
+ *              an input or output is an error.
+ *   workspace  device scratch of at least la_prefill_workspace_size(...)
+ *              bytes, owned by the caller; its contents on entry do not matter
+ *              and it must not be used by another call that overlaps on the GPU.
+ *
+ * Splits every (sequence, head) scan into segments that run on different SMs,
+ * combining them with the local-prefix / gather / global-prefix recipe of
+ * LASP+ ("MiniMax-01技术报告解读", §3.2 item 3) applied to SMs instead of ranks.
+ * ------------------------------------------------------------------------- */
+LA_API size_t la_prefill_workspace_size(int B, int N, int H, int d, int block);
+
+LA_API la_status la_prefill(const void *q, const void *k, const void *v,
+                     int B, int N, int H, int d, int block,
+                     const float *state_in, void *out, la_dtype out_dtype,
+                     float *state_out, void *workspace, size_t ws_bytes,
+                     cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Prefill of nseq packed sequences of different lengths (data packing:
+ * "MiniMax-01技术报告解读", §3.2 item 1 -- samples joined end to end along the
+ * sequence; §3.2 item 4 pads each to a block of 256 in memory, which is not
+ * done here: a short last block is masked in the kernel instead).
+ *
+ *   q, k, v      device, bf16, [total_tokens, H, d] packed.
+ *   cu_seqlens   DEVICE int32 [nseq + 1]: cu_seqlens[0] = 0, non-decreasing,
+ *                cu_seqlens[nseq] = total_tokens; sequence i owns tokens
+ *                [cu_seqlens[i], cu_seqlens[i+1]).  Zero-length sequences are
+ *                allowed.  It is checked on the device; a bad array computes
+ *                nothing and records LA_ERR_INVALID_ARGUMENT in the sticky word.
+ *   max_seqlen   an upper bound on every length (checked on the device too).
+ *   state_in     device fp32 [nseq, H, d, d] or NULL;  state_out likewise.
+ *   out          device [total_tokens, H, d], dtype out_dtype.
+ *   Other arguments as for la_prefill.
+ * ------------------------------------------------------------------------- */
+LA_API size_t la_prefill_varlen_workspace_size(int nseq, int total_tokens, int max_seqlen,
+                                        int H, int d, int block);
+
+LA_API la_status la_prefill_varlen(const void *q, const void *k, const void *v,
+                            const int *cu_seqlens, int nseq, int total_tokens,
+                            int max_seqlen, int H, int d, int block,
+                            const float *state_in, void *out, la_dtype out_dtype,
+                            float *state_out, void *workspace, size_t ws_bytes,
+                            cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * One fused decode step on a persistent fp32 state ("MiniMax-01技术报告解读",
+ * §3.3 items 1-2: length-1 tokens run in their own kernel, whose KV
+ * computation is fused with the update of the prefix-KV cache).
+ * For every (b, h):   S <- S + k^T v,   o = q S   (the new token sees itself).
+ *
+ *   q, k, v   device bf16 [B, H, d].
+ *   state     device fp32 [B, H, d, d], read and updated in place.
+ *   out       device [B, H, d], dtype out_dtype.
+ * ------------------------------------------------------------------------- */
+LA_API la_status la_decode_step(const void *q, const void *k, const void *v, float *state,
+                         void *out, la_dtype out_dtype, int B, int H, int d,
+                         cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Status.
+ * la_get_device_status synchronises `stream`, then returns and clears the
+ * sticky device word of the current device (LA_ERR_TIMEOUT,
+ * LA_ERR_INVALID_ARGUMENT from a device-side check), or LA_ERR_CUDA when the
+ * synchronisation itself reports an error.  LA_OK when nothing was recorded.
+ * ------------------------------------------------------------------------- */
+LA_API la_status la_get_device_status(cudaStream_t stream);
+
+/* Static English text for a status code (never NULL). */
+LA_API const char *la_status_string(la_status status);
+
+/* ---------------------------------------------------------------------------
+ * Controls and diagnostics (process-wide, host side; not thread-safe against
+ * concurrent launches).
+ *
+ * la_set_wait_limit_ns: upper bound for every device-side wait (mbarrier
+ *   phases, the cross-SM segment hand-off).  Default 2e9 ns.  A wait that runs
+ *   out records LA_ERR_TIMEOUT and the kernel finishes without hanging.
+ *   0 restores the default.
+ * la_set_segment_len: tokens per segment of the cross-SM scan; 0 = automatic,
+ *   otherwise a positive multiple of 128.  Changes only speed and rounding.
+ * la_debug_inject: fault injection made on the host side, for tests.
+ *   LA_INJECT_NONE (0): normal operation.
+ *   LA_INJECT_SKIP_PUBLISH (1): segments never publish their prefix, so every
+ *   segment with a predecessor waits until the limit runs out; outputs are
+ *   then meaningless and la_get_device_status returns LA_ERR_TIMEOUT.
+ * la_last_segment_len: the segment length the last prefill launch used.
+ * la_kernel_launches: cumulative number of kernels this library has
+ *   launched in this process (all entry points), for launch accounting.
+ * ------------------------------------------------------------------------- */
+#define LA_INJECT_NONE 0
+#define LA_INJECT_SKIP_PUBLISH 1
+
+LA_API la_status la_set_wait_limit_ns(unsigned long long ns);
+LA_API la_status la_set_segment_len(int tokens);
+LA_API la_status la_debug_inject(int mode);
+LA_API int la_last_segment_len(void);
+LA_API unsigned long long la_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LIGHTNING_ATTN_H */

@@ -1,0 +1,18 @@
+"""Lightning Attention (blocked causal linear attention) for NVIDIA B200.
+
+The computation runs in the in-tree CUDA library (sm_100a, tcgen05/TMEM
+tensor-core MMAs, TMA-staged tiles); this package is the Python face of its C
+ABI (include/lightning_attn.h).  Entry points:
+
+  prefill(q, k, v, ...)                      la_prefill          [B, N, H, 128]
+  prefill_varlen(q, k, v, cu_seqlens, ...)   la_prefill_varlen   [T, H, 128] packed
+  decode_step(q, k, v, state, ...)           la_decode_step      [B, H, 128]
+  get_device_status()                        la_get_device_status
+"""
+from ._binding import (D, DEFAULT_BLOCK, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
+                       LA_ERR_INVALID_ARGUMENT, LA_ERR_TIMEOUT, LA_ERR_UNSUPPORTED,
+                       LA_ERR_WORKSPACE, LA_FP32, LA_INJECT_NONE, LA_INJECT_SKIP_PUBLISH, LA_OK,
+                       LAError, debug_inject, decode_step, get_device_status, kernel_launches,
+                       last_segment_len, lib, library_path, prefill, prefill_varlen,
+                       set_segment_len, set_wait_limit_ns, status_string, varlen_workspace_size,
+                       workspace_size)

@@ -1,0 +1,235 @@
+"""ctypes binding of the C ABI in include/lightning_attn.h.
+
+Argument marshalling only: shapes, dtypes and pointers are checked and handed
+to the CUDA library, which does every step of the computation on the GPU.
+PyTorch provides device memory (outputs, workspace) and the current stream.
+There is no CPU fallback: if the library or a GPU is missing, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import _build
+
+LA_OK, LA_ERR_INVALID_ARGUMENT, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT, LA_ERR_WORKSPACE = range(6)
+LA_BF16, LA_FP32 = 0, 1
+LA_INJECT_NONE, LA_INJECT_SKIP_PUBLISH = 0, 1
+D = 128
+DEFAULT_BLOCK = 128
+
+EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size",
+            "la_prefill_varlen", "la_decode_step", "la_get_device_status", "la_status_string",
+            "la_set_wait_limit_ns", "la_set_segment_len", "la_debug_inject",
+            "la_last_segment_len", "la_kernel_launches")
+
+
+class LAError(RuntimeError):
+    """A non-OK status from the library."""
+
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def lib():
+    """Load the in-tree shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        path = _build.LIB_PATH
+        if not os.path.exists(path):
+            raise ImportError(f"CUDA library not built: {path} is missing "
+                              "(run linear_attention_blocked_b200._build.build())")
+        L = ctypes.CDLL(path)
+        vp, c_int, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.la_prefill_workspace_size.argtypes = [c_int] * 5
+        L.la_prefill_workspace_size.restype = sz
+        L.la_prefill.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp, sz, vp]
+        L.la_prefill.restype = c_int
+        L.la_prefill_varlen_workspace_size.argtypes = [c_int] * 6
+        L.la_prefill_varlen_workspace_size.restype = sz
+        L.la_prefill_varlen.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                        vp, vp, c_int, vp, vp, sz, vp]
+        L.la_prefill_varlen.restype = c_int
+        L.la_decode_step.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
+        L.la_decode_step.restype = c_int
+        L.la_get_device_status.argtypes = [vp]
+        L.la_get_device_status.restype = c_int
+        L.la_status_string.argtypes = [c_int]
+        L.la_status_string.restype = ctypes.c_char_p
+        L.la_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.la_set_wait_limit_ns.restype = c_int
+        L.la_set_segment_len.argtypes = [c_int]
+        L.la_set_segment_len.restype = c_int
+        L.la_debug_inject.argtypes = [c_int]
+        L.la_debug_inject.restype = c_int
+        L.la_last_segment_len.argtypes = []
+        L.la_last_segment_len.restype = c_int
+        L.la_kernel_launches.argtypes = []
+        L.la_kernel_launches.restype = ctypes.c_ulonglong
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().la_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != LA_OK:
+        raise LAError(status, where)
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _out_code(dtype):
+    if dtype == torch.bfloat16:
+        return LA_BF16
+    if dtype == torch.float32:
+        return LA_FP32
+    raise TypeError("out dtype must be torch.bfloat16 or torch.float32")
+
+
+def _need(t, name, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def workspace_size(B: int, N: int, H: int, d: int = D, block: int = 0) -> int:
+    return int(lib().la_prefill_workspace_size(B, N, H, d, block))
+
+
+def varlen_workspace_size(nseq: int, total_tokens: int, max_seqlen: int, H: int, d: int = D,
+                          block: int = 0) -> int:
+    return int(lib().la_prefill_varlen_workspace_size(nseq, total_tokens, max_seqlen, H, d, block))
+
+
+def _alloc_workspace(nbytes, device):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def prefill(q, k, v, block: int = 0, state_in=None, out=None, out_dtype=torch.bfloat16,
+            state_out=None, want_state: bool = True, workspace=None, stream=None):
+    """la_prefill on [B, N, H, d] bf16 tensors. Returns (out, state_out or None)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, N, H, d]")
+    B, N, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (B, N, H, d))
+    if out is None:
+        out = torch.empty((B, N, H, d), dtype=out_dtype, device=q.device)
+    _need(out, "out", out.dtype, (B, N, H, d))
+    if state_in is not None:
+        _need(state_in, "state_in", torch.float32, (B, H, d, d))
+    if state_out is None and want_state:
+        state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _need(state_out, "state_out", torch.float32, (B, H, d, d))
+    ws_bytes = workspace_size(B, N, H, d, block)
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, q.device)
+    st = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), B, N, H, d, block, _ptr(state_in), _ptr(out),
+                          _out_code(out.dtype), _ptr(state_out), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "la_prefill")
+    return out, state_out
+
+
+def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, block: int = 0, state_in=None, out=None,
+                   out_dtype=torch.bfloat16, state_out=None, want_state: bool = True, workspace=None,
+                   stream=None):
+    """la_prefill_varlen on packed [T, H, d] tensors with device int32 cu_seqlens."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, d]")
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (T, H, d))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    nseq = cu_seqlens.numel() - 1
+    if nseq < 0:
+        raise ValueError("cu_seqlens must hold nseq + 1 entries")
+    if out is None:
+        out = torch.empty((T, H, d), dtype=out_dtype, device=q.device)
+    _need(out, "out", out.dtype, (T, H, d))
+    if state_in is not None:
+        _need(state_in, "state_in", torch.float32, (nseq, H, d, d))
+    if state_out is None and want_state:
+        state_out = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device)
+    if state_out is not None:
+        _need(state_out, "state_out", torch.float32, (nseq, H, d, d))
+    ws_bytes = varlen_workspace_size(nseq, T, max_seqlen, H, d, block)
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, q.device)
+    st = lib().la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, int(max_seqlen),
+                                 H, d, block, _ptr(state_in), _ptr(out), _out_code(out.dtype),
+                                 _ptr(state_out), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "la_prefill_varlen")
+    return out, state_out
+
+
+def decode_step(q, k, v, state, out=None, out_dtype=torch.bfloat16, stream=None):
+    """la_decode_step on [B, H, d] bf16 tensors; `state` [B, H, d, d] fp32 is updated in place."""
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, d]")
+    B, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (B, H, d))
+    _need(state, "state", torch.float32, (B, H, d, d))
+    if out is None:
+        out = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
+    _need(out, "out", out.dtype, (B, H, d))
+    st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), _out_code(out.dtype),
+                              B, H, d, _stream_handle(stream))
+    _check(st, "la_decode_step")
+    return out
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the sticky device status."""
+    return int(lib().la_get_device_status(_stream_handle(stream)))
+
+
+def set_wait_limit_ns(ns: int):
+    _check(lib().la_set_wait_limit_ns(int(ns)), "la_set_wait_limit_ns")
+
+
+def set_segment_len(tokens: int):
+    _check(lib().la_set_segment_len(int(tokens)), "la_set_segment_len")
+
+
+def debug_inject(mode: int):
+    _check(lib().la_debug_inject(int(mode)), "la_debug_inject")
+
+
+def last_segment_len() -> int:
+    return int(lib().la_last_segment_len())
+
+
+def kernel_launches() -> int:
+    return int(lib().la_kernel_launches())

@@ -1,0 +1,330 @@
+// la_lib.cu -- C ABI of the Lightning Attention library (declared in
+// include/lightning_attn.h): argument checks, workspace partitioning, TMA
+// tensor-map encoding and kernel launches.  Everything is one translation unit
+// so that the sticky device status word is a plain __device__ variable.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "lightning_attn.h"
+#include "la_decode.cuh"
+#include "la_prefill.cuh"
+
+namespace {
+
+__device__ int g_la_status;  // sticky per-device status word (0 = OK)
+
+std::atomic<unsigned long long> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_seg_len_override{0};
+std::atomic<int> g_inject{0};
+std::atomic<int> g_last_seg_len{0};
+std::atomic<unsigned long long> g_launches{0};
+
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+
+// ---------------------------------------------------------------------------
+// driver entry point for cuTensorMapEncodeTiled (no link-time libcuda dependency)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// [T, H, 128] bf16 viewed as a 3-D tensor {128, H, T}; box {64, 1, 128},
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_qkv_map(CUtensorMap *map, const void *base, int T, int H) {
+    EncodeTiledFn fn = get_encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)la::D, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)la::D * 2, (cuuint64_t)H * la::D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)la::BLK};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return 148;
+    return sms;
+}
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Segment length of the cross-SM scan.  Depends on the problem only (not on
+// the device) so that the workspace size is a pure function of the shape.
+int choose_seg_len(int nseq, long long T, int H) {
+    const int ov = g_seg_len_override.load();
+    if (ov > 0) return ov;
+    int L = (H <= 16) ? 2048 : 1024;
+    const long long target = 2 * 148;  // want at least ~2 items per SM of a B200
+    while (L > la::BLK) {
+        const long long segs = (T + L - 1) / L + 0;  // lower bound of segments over all sequences
+        if (segs * (long long)H >= target) break;
+        L /= 2;
+    }
+    (void)nseq;
+    return L;
+}
+
+struct WsLayout {
+    size_t hdr, segs, flags, incl, total;
+    long long gmax;
+};
+
+WsLayout ws_layout(long long gmax, int H) {
+    WsLayout w;
+    w.gmax = gmax;
+    w.hdr = 0;
+    w.segs = la::HDR_BYTES;
+    w.flags = w.segs + round_up((size_t)gmax * sizeof(int4), 256);
+    w.incl = w.flags + round_up((size_t)gmax * H * sizeof(int), 256);
+    w.total = w.incl + (size_t)gmax * H * la::D * la::D * sizeof(float);
+    return w;
+}
+
+long long gmax_for(int nseq, long long T, int L) { return (T + L - 1) / L + nseq; }
+
+bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+la_status check_common(int H, int d, int block, la_dtype out_dtype) {
+    if (H <= 0 || d <= 0 || block < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (out_dtype != LA_BF16 && out_dtype != LA_FP32) return LA_ERR_INVALID_ARGUMENT;
+    if (d != la::D) return LA_ERR_UNSUPPORTED;
+    if (block != 0 && block != la::BLK) return LA_ERR_UNSUPPORTED;
+    return LA_OK;
+}
+
+// Shared body of la_prefill / la_prefill_varlen.
+la_status prefill_impl(const void *q, const void *k, const void *v, const int *cu, int fixed_len,
+                       int nseq, long long T, int max_seqlen, int H, int d, int block,
+                       const float *state_in, void *out, la_dtype out_dtype, float *state_out,
+                       void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    la_status st = check_common(H, d, block, out_dtype);
+    if (st != LA_OK) return st;
+    if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (T > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    if (nseq == 0) return T == 0 ? LA_OK : LA_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[6] = {q, k, v, out, state_in, state_out};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
+    const size_t n_in = (size_t)T * H * la::D * 2, n_out = (size_t)T * H * la::D * esz;
+    const size_t n_state = (size_t)nseq * H * la::D * la::D * 4;
+    if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+    const void *ins[3] = {q, k, v};
+    for (const void *p : ins) {
+        if (ranges_overlap(out, n_out, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(state_out, n_state, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (ranges_overlap(out, n_out, state_out, n_state) || ranges_overlap(out, n_out, state_in, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+
+    const int L = choose_seg_len(nseq, T, H);
+    if (L <= 0 || L % la::BLK) return LA_ERR_INVALID_ARGUMENT;
+    const long long gmax = gmax_for(nseq, T, L);
+    const WsLayout w = ws_layout(gmax, H);
+    if (!workspace || ws_bytes < w.total) return LA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return LA_ERR_INVALID_ARGUMENT;
+    if (gmax * (long long)H > 0x7fffffffLL) return LA_ERR_UNSUPPORTED;
+    if (ranges_overlap(workspace, w.total, out, n_out)) return LA_ERR_INVALID_ARGUMENT;
+    g_last_seg_len = L;
+
+    int *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_la_status) != cudaSuccess)
+        return LA_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+
+    la::ScheduleParams sp;
+    sp.cu = cu;
+    sp.fixed_len = fixed_len;
+    sp.nseq = nseq;
+    sp.T = (int)T;
+    sp.max_seqlen = max_seqlen;
+    sp.H = H;
+    sp.seg_len = L;
+    sp.Gmax = (int)gmax;
+    sp.hdr = reinterpret_cast<int *>(ws + w.hdr);
+    sp.segs = reinterpret_cast<int4 *>(ws + w.segs);
+    sp.flags = reinterpret_cast<int *>(ws + w.flags);
+    sp.state_in = state_in;
+    sp.state_out = state_out;
+    sp.status = status;
+    la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    if (T == 0) return LA_OK;
+
+    CUtensorMap mq, mk, mv;
+    if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
+        !encode_qkv_map(&mv, v, (int)T, H))
+        return LA_ERR_CUDA;
+
+    la::PrefillParams pp;
+    pp.state_in = state_in;
+    pp.state_out = state_out;
+    pp.out = out;
+    pp.out_fp32 = out_dtype == LA_FP32;
+    pp.H = H;
+    pp.hdr = sp.hdr;
+    pp.segs = sp.segs;
+    pp.flags = sp.flags;
+    pp.incl = reinterpret_cast<float *>(ws + w.incl);
+    pp.wait_limit_ns = g_wait_limit_ns.load();
+    pp.inject = g_inject.load();
+    pp.status = status;
+
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(la::la_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        la::PREFILL_SMEM);
+    });
+    if (attr_err != cudaSuccess) return LA_ERR_CUDA;
+    const long long items = gmax * (long long)H;
+    const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
+    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_prefill_workspace_size(int B, int N, int H, int d, int block) {
+    (void)d;
+    (void)block;
+    if (B <= 0 || N < 0 || H <= 0) return la::HDR_BYTES;
+    const long long T = (long long)B * N;
+    const int L = choose_seg_len(B, T, H);
+    return ws_layout(gmax_for(B, T, L), H).total;
+}
+
+size_t la_prefill_varlen_workspace_size(int nseq, int total_tokens, int max_seqlen, int H, int d,
+                                        int block) {
+    (void)d;
+    (void)block;
+    (void)max_seqlen;
+    if (nseq <= 0 || total_tokens < 0 || H <= 0) return la::HDR_BYTES;
+    const int L = choose_seg_len(nseq, total_tokens, H);
+    return ws_layout(gmax_for(nseq, total_tokens, L), H).total;
+}
+
+la_status la_prefill(const void *q, const void *k, const void *v, int B, int N, int H, int d, int block,
+                     const float *state_in, void *out, la_dtype out_dtype, float *state_out,
+                     void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (B < 0 || N < 0) return LA_ERR_INVALID_ARGUMENT;
+    const long long T = (long long)B * N;
+    return prefill_impl(q, k, v, nullptr, N, B, T, N, H, d, block, state_in, out, out_dtype, state_out,
+                        workspace, ws_bytes, stream);
+}
+
+la_status la_prefill_varlen(const void *q, const void *k, const void *v, const int *cu_seqlens,
+                            int nseq, int total_tokens, int max_seqlen, int H, int d, int block,
+                            const float *state_in, void *out, la_dtype out_dtype, float *state_out,
+                            void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!cu_seqlens || nseq < 0 || total_tokens < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARGUMENT;
+    return prefill_impl(q, k, v, cu_seqlens, 0, nseq, total_tokens, max_seqlen, H, d, block, state_in,
+                        out, out_dtype, state_out, workspace, ws_bytes, stream);
+}
+
+la_status la_decode_step(const void *q, const void *k, const void *v, float *state, void *out,
+                         la_dtype out_dtype, int B, int H, int d, cudaStream_t stream) {
+    la_status st = check_common(H, d, 0, out_dtype);
+    if (st != LA_OK) return st;
+    if (B < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (B == 0) return LA_OK;
+    if (!q || !k || !v || !state || !out) return LA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[5] = {q, k, v, state, out};
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+    const long long npairs = (long long)B * H;
+    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
+    if (ranges_overlap(out, npairs * la::D * esz, state, npairs * la::D * la::D * 4))
+        return LA_ERR_INVALID_ARGUMENT;
+    const long long grid = npairs < (1LL << 30) ? npairs : (1LL << 30);
+    la::la_decode_kernel<<<(unsigned)grid, la::DEC_THREADS, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), state, out, out_dtype == LA_FP32, npairs);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
+
+la_status la_get_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return LA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_la_status, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_la_status, &zero, sizeof(int)) != cudaSuccess) return LA_ERR_CUDA;
+    }
+    return static_cast<la_status>(v);
+}
+
+const char *la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "ok";
+        case LA_ERR_INVALID_ARGUMENT: return "invalid argument";
+        case LA_ERR_UNSUPPORTED: return "unsupported (only d = 128 and block 0/128 are built)";
+        case LA_ERR_CUDA: return "CUDA error";
+        case LA_ERR_TIMEOUT: return "a bounded device-side wait ran out";
+        case LA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+la_status la_set_wait_limit_ns(unsigned long long ns) {
+    g_wait_limit_ns = ns ? ns : kDefaultWaitNs;
+    return LA_OK;
+}
+
+la_status la_set_segment_len(int tokens) {
+    if (tokens < 0 || (tokens > 0 && tokens % la::BLK)) return LA_ERR_INVALID_ARGUMENT;
+    g_seg_len_override = tokens;
+    return LA_OK;
+}
+
+la_status la_debug_inject(int mode) {
+    if (mode != LA_INJECT_NONE && mode != LA_INJECT_SKIP_PUBLISH) return LA_ERR_INVALID_ARGUMENT;
+    g_inject = mode;
+    return LA_OK;
+}
+
+int la_last_segment_len(void) { return g_last_seg_len.load(); }
+
+unsigned long long la_kernel_launches(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,132 @@
+"""C-ABI library checks that need no GPU: it builds for sm_100a, loads, exports
+every entry point the header declares, and rejects bad arguments synchronously
+before touching the device.  (Only argument combinations that fail
+validation are passed here, so nothing is ever launched.)"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_blocked_b200 as la
+from linear_attention_blocked_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lightning_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return la.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LA_API\s+[\w\s\*]*?\b(la_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("la_prefill", "la_prefill_varlen", "la_decode_step", "la_get_device_status",
+                     "la_status_string", "la_prefill_workspace_size",
+                     "la_prefill_varlen_workspace_size"):
+        assert required in names
+    assert set(names) == set(la.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_no_link_time_driver_dependency():
+    # the library reaches the driver at run time; it must load without a GPU
+    out = os.popen(f"ldd {_build.LIB_PATH}").read()
+    assert "libcuda.so" not in out
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert la.status_string(code)
+    assert la.status_string(99) == "unknown status"
+
+
+V = ctypes.c_void_p
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _prefill(L, B=1, N=128, H=1, d=128, block=0, q=FAKE, out=FAKE, state_in=None, state_out=None,
+             ws=FAKE, ws_bytes=0, dtype=0):
+    return L.la_prefill(V(q), V(FAKE), V(FAKE), B, N, H, d, block, V(state_in) if state_in else None,
+                        V(out), dtype, V(state_out) if state_out else None, V(ws), ws_bytes, None)
+
+
+def test_prefill_argument_errors(L):
+    assert _prefill(L, d=64) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(L, block=64) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(L, block=256) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(L, block=-1) == la.LA_ERR_INVALID_ARGUMENT
+    assert _prefill(L, H=0) == la.LA_ERR_INVALID_ARGUMENT
+    assert _prefill(L, B=-1) == la.LA_ERR_INVALID_ARGUMENT
+    assert _prefill(L, dtype=7) == la.LA_ERR_INVALID_ARGUMENT
+    assert _prefill(L, q=0) == la.LA_ERR_INVALID_ARGUMENT             # null input
+    assert _prefill(L, q=FAKE + 8) == la.LA_ERR_INVALID_ARGUMENT      # misaligned
+    assert _prefill(L, out=FAKE) == la.LA_ERR_INVALID_ARGUMENT        # out overlaps q
+    far = 1 << 40
+    assert _prefill(L, out=far, ws=0) == la.LA_ERR_WORKSPACE          # no workspace
+    need = L.la_prefill_workspace_size(1, 128, 1, 128, 0)
+    assert _prefill(L, out=far, ws=2 * far, ws_bytes=need - 1) == la.LA_ERR_WORKSPACE
+    assert _prefill(L, out=far, ws=2 * far + 16, ws_bytes=need) == la.LA_ERR_INVALID_ARGUMENT  # ws alignment
+    # state_out partially overlapping state_in
+    assert _prefill(L, out=far, state_in=3 * far, state_out=3 * far + 64) == la.LA_ERR_INVALID_ARGUMENT
+
+
+def test_varlen_and_decode_argument_errors(L):
+    assert L.la_prefill_varlen(V(FAKE), V(FAKE), V(FAKE), None, 1, 10, 10, 1, 128, 0, None, V(FAKE), 0,
+                               None, V(FAKE), 0, None) == la.LA_ERR_INVALID_ARGUMENT  # null cu_seqlens
+    assert L.la_prefill_varlen(V(FAKE), V(FAKE), V(FAKE), V(FAKE), -1, 10, 10, 1, 128, 0, None, V(FAKE),
+                               0, None, V(FAKE), 0, None) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_prefill_varlen(V(FAKE), V(FAKE), V(FAKE), V(FAKE), 2, 10, 10, 1, 96, 0, None, V(FAKE),
+                               0, None, V(FAKE), 0, None) == la.LA_ERR_UNSUPPORTED
+    assert L.la_decode_step(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 1, 1, 64, None) == \
+        la.LA_ERR_UNSUPPORTED
+    assert L.la_decode_step(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, -1, 1, 128, None) == \
+        la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_decode_step(None, V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 1, 1, 128, None) == \
+        la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_decode_step(V(FAKE + 4), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 1, 1, 128, None) == \
+        la.LA_ERR_INVALID_ARGUMENT
+    # output overlapping the state
+    assert L.la_decode_step(V(FAKE), V(FAKE), V(FAKE), V(1 << 40), V((1 << 40) + 256), 0, 1, 1, 128,
+                            None) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_decode_step(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 0, 1, 128, None) == la.LA_OK
+
+
+def test_workspace_sizes(L):
+    small = L.la_prefill_workspace_size(1, 1024, 2, 128, 0)
+    big = L.la_prefill_workspace_size(1, 32768, 64, 128, 0)
+    assert 0 < small < big
+    assert L.la_prefill_varlen_workspace_size(8, 1 << 18, 65536, 64, 128, 0) > big
+    assert L.la_prefill_workspace_size(0, 10, 1, 128, 0) == 256
+
+
+def test_segment_len_control(L):
+    assert L.la_set_segment_len(100) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_set_segment_len(-128) == la.LA_ERR_INVALID_ARGUMENT
+    before = L.la_prefill_workspace_size(1, 65536, 64, 128, 0)
+    assert L.la_set_segment_len(128) == la.LA_OK
+    assert L.la_prefill_workspace_size(1, 65536, 64, 128, 0) > before
+    assert L.la_set_segment_len(0) == la.LA_OK
+    assert L.la_prefill_workspace_size(1, 65536, 64, 128, 0) == before
+    assert L.la_debug_inject(5) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_debug_inject(0) == la.LA_OK
+    assert L.la_set_wait_limit_ns(0) == la.LA_OK
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 128, 1, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        la.prefill(q, q, q)
