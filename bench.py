@@ -1,0 +1,426 @@
+"""Benchmark of the Lightning Attention hot path on B200.
+
+One step = one la_prefill of the 32K-token workload shaped like the
+MiniMax-01 attention layer: B=1, H=64, N=32768, d=128, bf16 q/k/v drawn
+iid N(0,1)*128^-0.5, fp32 accumulation, bf16 output plus the final fp32
+128x128 state of every head.  The step runs every prefill row of the hot path
+(segment table + TMA staging + the four tcgen05 contractions + masking +
+cross-SM segment hand-off + epilogue).  In the same run the fused batched
+decode step is timed on its own workload (256 sequences x 64 heads, fp32
+states initialised by a 4096-token prefill) and reported under "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W]      # CUDA path
+  python bench.py --impl reference ...                     # fp64 CPU oracle arm
+
+Under torchrun (N > 1) every rank runs its own independent batch (no
+collective on the data path; weak scaling); timing is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import la_inputs  # noqa: E402
+
+METRIC = "lightning-attn prefill tok/s + TFLOP/s; decode tok/s; % of roofline"
+B, N, H, D = 1, 32768, 64, 128
+BLOCK = 128
+DEC_SEQS, DEC_PREFILL = 256, 4096
+SEED = 20250101
+
+
+# --------------------------------------------------------------------------- helpers
+def prefill_bytes(tok_heads: int, heads: int, seqs: int) -> int:
+    """Algorithmic HBM bytes of one prefill: read q, k, v (bf16), write out
+    (bf16), write the final fp32 state of every (sequence, head)."""
+    return tok_heads * D * 2 * 4 + seqs * heads * D * D * 4
+
+
+def prefill_flops(tok_heads: int, block: int, frac_phase_a: float):
+    """(algorithmic, executed) FLOPs, 2 FLOP per multiply-add.
+    algorithmic per token-head: 2*(Bk+1)*d for the causal triangle of the
+    block including its diagonal (scores and P V) + 4*d^2 (inter term Q S and
+    state update K^T V).
+    executed per token-head, what the tensor pipe runs in this kernel:
+    Q K^T and P V over full 128x128 blocks (4*Bk*d), Q S_hi + Q S_lo (4*d^2),
+    K^T V in the scan (2*d^2) and again in the segment-sum pass for the
+    fraction of tokens whose segment has a successor (2*d^2*frac_phase_a)."""
+    alg = 2 * (block + 1) * D + 4 * D * D
+    exe = 4 * block * D + 6 * D * D + 2 * D * D * frac_phase_a
+    return tok_heads * alg, tok_heads * exe
+
+
+def decode_bytes(pairs: int) -> int:
+    """Read + write the fp32 state, read q, k, v and write o (bf16)."""
+    return pairs * (2 * D * D * 4 + 4 * D * 2)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("la_prefill.cuh", "la_ptx.cuh", "la_lib.cu"):
+        with open(os.path.join(ROOT, "linear_attention_blocked_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        e = rec[kernel][workload]
+        if e.get("source_hash") == kernel_source_hash():
+            return float(e["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) tagged with host time."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.samples = []
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1]
+        if not rows:  # very short region: take the samples nearest to it
+            rows = [s for (t, s) in self.samples if t0 - 0.5 <= t <= t1 + 0.5]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 6 + i and r[6 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle arms
+def oracle_sample_rate(budget_s: float, seed: int):
+    """Time the fp64 oracle (recurrent form) on heads of the 32K workload until
+    `budget_s` seconds of CPU work are spent.  Returns (tok/s scaled to all 64
+    heads, threads used, description)."""
+    import oracle
+    oracle.build()
+    q, k, v = la_inputs.qkv((N, H, D), seed)
+    Q, K, V = la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v)
+    cu = np.array([0, N], np.int32)
+    threads = oracle.max_threads()
+    heads_done, elapsed = 0, 0.0
+    step = max(1, min(H, threads))
+    while heads_done < H and elapsed < budget_s:
+        hs = list(range(heads_done, min(H, heads_done + step)))
+        t = time.perf_counter()
+        oracle.recurrent(Q, K, V, cu, heads=hs)
+        elapsed += time.perf_counter() - t
+        heads_done += len(hs)
+    rate = N * heads_done / H / elapsed
+    desc = (f"fp64 recurrent oracle, {heads_done} of {H} heads x {N} tokens in {elapsed:.1f} s; "
+            f"tok/s scaled by {heads_done}/{H}")
+    return rate, threads, desc
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    threads = oracle.max_threads()
+    q, k, v = la_inputs.qkv((N, H, D), SEED)
+    Q, K, V = la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v)
+    # each step: a bounded sample (tokens x 1 head) sized so the whole run takes ~60 s
+    per_step_s = max(0.02, 60.0 / max(1, args.steps + args.warmup))
+    probe_tok = 1024
+    t = time.perf_counter()
+    oracle.recurrent(Q[:probe_tok], K[:probe_tok], V[:probe_tok], np.array([0, probe_tok], np.int32), heads=[0],
+                     threads=1)
+    per_tok = (time.perf_counter() - t) / probe_tok
+    nh = max(1, min(H, threads))
+    ntok = int(max(64, min(N, per_step_s / per_tok * 0.8)))
+    cu = np.array([0, ntok], np.int32)
+    hs = list(range(nh))
+    for _ in range(args.warmup):
+        oracle.recurrent(Q[:ntok], K[:ntok], V[:ntok], cu, heads=hs)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.recurrent(Q[:ntok], K[:ntok], V[:ntok], cu, heads=hs)
+    dt = time.perf_counter() - t
+    value = ntok * nh / H * args.steps / dt       # tok/s of the 64-head workload
+    sample = f"each step: fp64 recurrent oracle on the first {ntok} tokens of {nh} of {H} heads; tok/s scaled by {nh}/{H}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(ngpu):
+    return {"workload": "lightning-attn causal prefill B=1 H=64 N=32768 d=128 bf16 in/out + fp32 final state",
+            "B": B, "N": N, "H": H, "d": D, "block": BLOCK, "global_batch": B * ngpu, "seq_len": N,
+            "parallelism": f"replicas x{ngpu} (independent batches, no collective)",
+            "l2": "inputs larger than L2 (805 MB of q/k/v read per step), no flush",
+            "seed": SEED}
+
+
+# --------------------------------------------------------------------------- CUDA arm
+def run_cuda(args, world, rank, local):
+    import linear_attention_blocked_b200 as la
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    hbm_peak, tc_peak, tc_sust, peak_src = load_peaks()
+
+    q, k, v = la_inputs.qkv((B, N, H, D), SEED + rank, device=dev)
+    out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=dev)
+    st = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(la.workspace_size(B, N, H, D, BLOCK), dtype=torch.uint8, device=dev)
+
+    def step():
+        la.prefill(q, k, v, block=BLOCK, out=out, state_out=st, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    if la.get_device_status() != la.LA_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    sampler = ClockSampler(local if world > 1 else 0) if rank == 0 else None
+    time.sleep(0.3 if sampler else 0)
+    launches0 = la.kernel_launches()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_host1 = time.time()
+    barrier(world)
+    launches = la.kernel_launches() - launches0
+    ms = ev0.elapsed_time(ev1) / args.steps
+    ms_max = max_over_ranks(ms, world)
+    status = la.get_device_status()
+    clocks = sampler.summary(t_host0, t_host1) if sampler else None
+    if sampler:
+        sampler.stop()
+
+    tok_heads = B * N * H
+    tokens_all = B * N * world
+    value = tokens_all / (ms_max * 1e-3)
+    byts = prefill_bytes(tok_heads, H, B)
+    L = la.last_segment_len()
+    nseg = -(-N // L)
+    f_alg, f_exe = prefill_flops(tok_heads, BLOCK, (nseg - 1) * L / N)
+    achieved_gbs = byts / (ms * 1e-3) / 1e9
+
+    # ---------------- end to end through the public API with host buffers
+    e2e_steps = max(3, min(args.steps, 20))
+    qh = q.cpu().pin_memory(); kh = k.cpu().pin_memory(); vh = v.cpu().pin_memory()
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    sh = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+        la.prefill(qd, kd, vd, block=BLOCK, out=out, state_out=st, workspace=ws)
+        oh.copy_(out, non_blocking=True); sh.copy_(st, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    del qd, kd, vd
+
+    # ---------------- fused batched decode on its own workload
+    dec = None
+    if rank == 0 or world > 1:
+        dec = bench_decode(la, dev, stream, args, hbm_peak, world)
+
+    status2 = la.get_device_status()
+    if rank != 0:
+        return 0
+    traffic = recorded_traffic("la_prefill_kernel", "prefill_B1_H64_N32768")
+    cpu = None
+    if world == 1 and args.cpu_seconds > 0:
+        rate, cores, desc = oracle_sample_rate(args.cpu_seconds, SEED)
+        cpu = {"value": rate, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(world),
+        "segment_len": L,
+        "tflops_alg": f_alg / (ms * 1e-3) / 1e12, "tflops_exec": f_exe / (ms * 1e-3) / 1e12,
+        "tensor_frac_exec": f_exe / (ms * 1e-3) / 1e12 / tc_peak,
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                     "kernel": "la_prefill_kernel", "bytes_per_launch": byts,
+                     "duration": "CUDA events around each la_prefill call (scheduler + prefill kernel)",
+                     "peak_source": f"{peak_src} hbm_gbs"},
+        "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tok/s", "ms_per_step": e2e_ms,
+                "steps": e2e_steps,
+                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                "d2h_bytes_per_step": out.numel() * out.element_size() + st.numel() * st.element_size()},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+        "decode": dec,
+        "cpu_baseline": cpu,
+        "device_status": [int(status), int(status2)],
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_decode(la, dev, stream, args, hbm_peak, world):
+    """Decode workload: 256 sequences x 64 heads, states from a 4096-token
+    prefill (run in chunks of sequences), then timed decode steps."""
+    state = torch.empty((DEC_SEQS, H, D, D), dtype=torch.float32, device=dev)
+    chunk = 16
+    for s0 in range(0, DEC_SEQS, chunk):
+        qp, kp, vp = la_inputs.qkv((chunk, DEC_PREFILL, H, D), SEED + 7 + s0, device=dev)
+        la.prefill(qp, kp, vp, block=BLOCK, state_out=state[s0:s0 + chunk])
+        del qp, kp, vp
+    steps = max(16, min(args.steps, 1024))
+    qs = [la_inputs.qkv((DEC_SEQS, H, D), la_inputs.decode_seed(SEED, s), device=dev) for s in range(8)]
+    o = torch.empty((DEC_SEQS, H, D), dtype=torch.bfloat16, device=dev)
+    for i in range(3):
+        la.decode_step(*qs[i % 8], state, out=o)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        la.decode_step(*qs[i % 8], state, out=o)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    pairs = DEC_SEQS * H
+    gbs = decode_bytes(pairs) / (ms * 1e-3) / 1e9
+    del state
+    return {"workload": "decode 256 seqs x H=64 x d=128, fp32 state (1 GiB) from a 4096-token prefill",
+            "tok_s": DEC_SEQS * world / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "kernel": "la_decode_kernel",
+                         "bytes_per_launch": decode_bytes(pairs)}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="CPU time budget of the oracle baseline sample (rank 0, N=1)")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        # the oracle runs on the host cores of rank 0 only; no process group needed
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+    world, rank, local = dist_setup()
+    try:
+        rc = run_cuda(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())
