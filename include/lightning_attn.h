@@ -132,6 +132,33 @@ LA_API la_status la_decode_step(const void *q, const void *k, const void *v, flo
                          cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * la_prefill without a workspace argument, for callers that cannot allocate
+ * device memory when they call: e.g. a plugin inside a host framework that
+ * owns the allocator and offers no allocation hook, or a serving process that
+ * reserved all device memory up front and forbids cudaMalloc (a slow call
+ * that may synchronise the device) on its request path.  This entry point has
+ * no counterpart on the pages; it is a convenience of this library.
+ *
+ * Arguments, layouts and results are those of la_prefill minus the workspace.
+ * Scratch is a fixed 32 MiB array inside the library, reserved on every GPU
+ * the process uses from library load until exit; the call allocates and frees
+ * nothing.  To fit, it may use longer cross-SM segments than la_prefill
+ * (changing only speed and rounding).  A problem whose scratch needs exceed
+ * 32 MiB even with one segment per sequence -- more than about 500
+ * (sequence, head) pairs -- is rejected with LA_ERR_WORKSPACE before any
+ * launch.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  Every call uses the same array and the kernels reset
+ * the parts that must start at zero, so leftover contents do not matter, but
+ * calls that overlap on the GPU (other streams, other host threads) race on
+ * it: serialise them.
+ * ------------------------------------------------------------------------- */
+LA_API la_status la_prefill_noalloc(const void *q, const void *k, const void *v,
+                                    int B, int N, int H, int d, int block,
+                                    const float *state_in, void *out, la_dtype out_dtype,
+                                    float *state_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status.
  * la_get_device_status synchronises `stream`, then returns and clears the
  * sticky device word of the current device (LA_ERR_TIMEOUT,

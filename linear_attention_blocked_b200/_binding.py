@@ -23,7 +23,7 @@ DEFAULT_BLOCK = 128
 EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size",
             "la_prefill_varlen", "la_decode_step", "la_get_device_status", "la_status_string",
             "la_set_wait_limit_ns", "la_set_segment_len", "la_debug_inject",
-            "la_last_segment_len", "la_kernel_launches")
+            "la_last_segment_len", "la_kernel_launches", "la_prefill_noalloc")
 
 
 class LAError(RuntimeError):
@@ -60,6 +60,8 @@ def lib():
         L.la_prefill_varlen.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
                                         vp, vp, c_int, vp, vp, sz, vp]
         L.la_prefill_varlen.restype = c_int
+        L.la_prefill_noalloc.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp]
+        L.la_prefill_noalloc.restype = c_int
         L.la_decode_step.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
         L.la_decode_step.restype = c_int
         L.la_get_device_status.argtypes = [vp]

@@ -328,3 +328,146 @@ int la_last_segment_len(void) { return g_last_seg_len.load(); }
 unsigned long long la_kernel_launches(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ===========================================================================
+// la_prefill_noalloc -- la_prefill for callers that cannot allocate.
+//
+// Some callers have no way to hand us a workspace: a plugin loaded into a host
+// framework that owns the device allocator and offers no allocation hook, or a
+// serving process that reserves all device memory up front (for its caches)
+// and forbids further cudaMalloc calls on its request path, where cudaMalloc
+// would also be a slow, device-synchronising call.  For them this entry point
+// takes no workspace: its scratch is the fixed-size device array below,
+// reserved once in every process that loads the library, on every GPU it
+// touches, until the process exits.
+//
+// Its scratch needs grow with the number of (segment, head) work items, so
+// this variant lengthens the segments (which changes only speed and
+// rounding) until the scratch fits; if even one segment per sequence does not
+// fit, the call is rejected with LA_ERR_WORKSPACE before anything is launched.
+// The scheduler kernel re-initialises every word of scratch that must start
+// at zero (ticket counter, hand-off flags) at the start of each call, so the
+// contents left by the previous call do not matter.  All calls share the one
+// array: calls that can overlap on the GPU (different streams, or different
+// host threads) race on it and must be serialised by the caller.
+// ===========================================================================
+#define LA_NOALLOC_SCRATCH_BYTES (32u << 20)  // 32 MiB per GPU
+static __device__ __align__(256) unsigned char g_la_noalloc_scratch[LA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  The host-side
+// symbol is only a stand-in; the real address comes from cudaGetSymbolAddress,
+// looked up once per device on the first call made with that device current.
+la_status noalloc_scratch_address(void **addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return LA_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return LA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_la_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) return LA_ERR_CUDA;
+        g_noalloc_addr[dev] = p;
+    }
+    *addr = g_noalloc_addr[dev];
+    return LA_OK;
+}
+
+}  // namespace
+
+extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void *v, int B, int N, int H,
+                                        int d, int block, const float *state_in, void *out,
+                                        la_dtype out_dtype, float *state_out, cudaStream_t stream) {
+    la_status st = check_common(H, d, block, out_dtype);
+    if (st != LA_OK) return st;
+    if (B < 0 || N < 0) return LA_ERR_INVALID_ARGUMENT;
+    const long long T = (long long)B * N;
+    if (T > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    if (B == 0) return LA_OK;
+    if (T > 0 && (!q || !k || !v || !out)) return LA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[6] = {q, k, v, out, state_in, state_out};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
+    const size_t n_in = (size_t)T * H * la::D * 2, n_out = (size_t)T * H * la::D * esz;
+    const size_t n_state = (size_t)B * H * la::D * la::D * 4;
+    if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+    const void *ins[3] = {q, k, v};
+    for (const void *p : ins) {
+        if (ranges_overlap(out, n_out, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(state_out, n_state, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (ranges_overlap(out, n_out, state_out, n_state) || ranges_overlap(out, n_out, state_in, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+
+    // longest useful segment: one per sequence
+    const int max_len = (int)(((long long)(N > 0 ? N : 1) + la::BLK - 1) / la::BLK * la::BLK);
+    int L = choose_seg_len(B, T, H);
+    while (ws_layout(gmax_for(B, T, L), H).total > LA_NOALLOC_SCRATCH_BYTES && L < max_len)
+        L = (2 * L < max_len) ? 2 * L : max_len;
+    const long long gmax = gmax_for(B, T, L);
+    const WsLayout w = ws_layout(gmax, H);
+    if (w.total > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;  // beyond the built-in scratch
+
+    void *scratch = nullptr;
+    st = noalloc_scratch_address(&scratch);
+    if (st != LA_OK) return st;
+    int *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_la_status) != cudaSuccess)
+        return LA_ERR_CUDA;
+    uint8_t *ws = static_cast<uint8_t *>(scratch);
+    g_last_seg_len = L;
+
+    la::ScheduleParams sp;
+    sp.cu = nullptr;
+    sp.fixed_len = N;
+    sp.nseq = B;
+    sp.T = (int)T;
+    sp.max_seqlen = N;
+    sp.H = H;
+    sp.seg_len = L;
+    sp.Gmax = (int)gmax;
+    sp.hdr = reinterpret_cast<int *>(ws + w.hdr);
+    sp.segs = reinterpret_cast<int4 *>(ws + w.segs);
+    sp.flags = reinterpret_cast<int *>(ws + w.flags);
+    sp.state_in = state_in;
+    sp.state_out = state_out;
+    sp.status = status;
+    la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    if (T == 0) return LA_OK;
+
+    CUtensorMap mq, mk, mv;
+    if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
+        !encode_qkv_map(&mv, v, (int)T, H))
+        return LA_ERR_CUDA;
+    la::PrefillParams pp;
+    pp.state_in = state_in;
+    pp.state_out = state_out;
+    pp.out = out;
+    pp.out_fp32 = out_dtype == LA_FP32;
+    pp.H = H;
+    pp.hdr = sp.hdr;
+    pp.segs = sp.segs;
+    pp.flags = sp.flags;
+    pp.incl = reinterpret_cast<float *>(ws + w.incl);
+    pp.wait_limit_ns = g_wait_limit_ns.load();
+    pp.inject = g_inject.load();
+    pp.status = status;
+    if (cudaFuncSetAttribute(la::la_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             la::PREFILL_SMEM) != cudaSuccess)
+        return LA_ERR_CUDA;
+    const long long items = gmax * (long long)H;
+    const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
+    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
