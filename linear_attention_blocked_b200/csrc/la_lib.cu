@@ -201,6 +201,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.incl = reinterpret_cast<float *>(ws + w.incl);
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
+    pp.seg_len = L;
     pp.status = status;
 
     static std::once_flag attr_once;
@@ -460,6 +461,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.incl = reinterpret_cast<float *>(ws + w.incl);
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
+    pp.seg_len = L;
     pp.status = status;
     if (cudaFuncSetAttribute(la::la_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              la::PREFILL_SMEM) != cudaSuccess)

@@ -14,23 +14,27 @@
 //   phase O (blocked scan over the segment's row blocks, starting from E_j):
 //       Sc  = Q_b K_b^T                    a2   (SS MMA, M=N=128, K=d)
 //       P   = bf16(Sc ⊙ M), inclusive mask a3   (TMEM -> regs -> TMEM)
-//       O   = Q_b S_hi + Q_b S_lo          a5   (S split in two bf16 terms)
+//       O   = Q_b S_hi + Q_b S_lo          a5   (S split in two bf16 terms, two
+//                                               64-column halves)
 //       S  += K_b^T V_b                    a6   (SS MMA, both MN-major)
 //       O  += P V_b                        a4   (TS MMA, P read from TMEM)
 //       out = O (bf16 or fp32)             a7
 //   and, for the last segment, the final state S goes to state_out.
 //
-// Warp roles (192 threads): warp 0 = TMA producer + ticket fetch, warp 1 =
-// TMEM allocator + MMA issuer (lane 0 issues), warps 2-5 = TMEM-lane owners
-// doing masking, state snapshots, look-back and output stores.
+// Warp roles (320 threads): warp 0 = TMA producer + ticket fetch, warp 1 =
+// TMEM allocator + MMA issuer (lane 0 issues), warps 2-5 = causal mask (a3)
+// and output store (a7), warps 6-9 = segment hand-off (phase L), state
+// snapshots for a5 and the final state.  A warp may only touch the 32 TMEM
+// lanes of its quarter (warp % 4), so each group of four covers all 128 rows.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzle everywhere):
-//   K ring 2 x 32 KiB | V ring 2 x 32 KiB | Q 32 KiB | S_hi 32 KiB | S_lo 32 KiB
-//   | barriers + item queue.
+//   K ring 2 x 32 KiB | V ring 2 x 32 KiB | Q ring 2 x 32 KiB | S_hi half 16 KiB |
+//   S_lo half 16 KiB | barriers + item queue.
 // A [128 x 128] bf16 tile is two 16 KiB halves (columns 0-63, 64-127), each
 // 128 rows of 128 bytes as TMA writes them with a {64, 1, 128} box.
-// TMEM (512 columns x 128 lanes x 32 bit): Sc [0,128) | P [128,192) |
-//   O [256,384) | S [384,512).
+// TMEM (512 columns x 128 lanes x 32 bit): Sc [0,128) (P overwrites its first
+//   64 columns in place) | O0 [128,256) | O1 [256,384) (double-buffered output)
+//   | S [384,512).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,18 +48,32 @@ constexpr int BLK = 128;                    // rows per block (= MMA M)
 constexpr int HALF_BYTES = BLK * 128;       // [128 rows x 64 bf16]
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // [128 x 128] bf16
 constexpr int KV_STAGES = 2;
-constexpr int PREFILL_THREADS = 192;
+constexpr int PREFILL_THREADS = 320;
+// L2 prefetch distances, in row blocks, ahead of the shared-memory loads.
+// Shared memory holds about one block ahead; in phase O the only DRAM reads
+// are the Q tiles (K and V come back from L2), so Q is prefetched further
+// ahead to keep enough DRAM reads in flight per SM.  Phase A already keeps
+// two 64 KiB K/V stages in flight and gets no K/V prefetch by default.
+#ifndef LA_PREFETCH_Q
+#define LA_PREFETCH_Q 0
+#endif
+#ifndef LA_PREFETCH_KV
+#define LA_PREFETCH_KV 0
+#endif
+constexpr int PF_Q = LA_PREFETCH_Q;
+constexpr int PF_KV = LA_PREFETCH_KV;
 
 constexpr int SM_K = 0;
 constexpr int SM_V = SM_K + KV_STAGES * TILE_BYTES;
+constexpr int Q_STAGES = 2;
 constexpr int SM_Q = SM_V + KV_STAGES * TILE_BYTES;
-constexpr int SM_SHI = SM_Q + TILE_BYTES;
-constexpr int SM_SLO = SM_SHI + TILE_BYTES;
-constexpr int SM_CTRL = SM_SLO + TILE_BYTES;  // 229376
+constexpr int SM_SHI = SM_Q + Q_STAGES * TILE_BYTES;  // one 64-column half of S as bf16 hi
+constexpr int SM_SLO = SM_SHI + HALF_BYTES;           // ... and its bf16 lo residual
+constexpr int SM_CTRL = SM_SLO + HALF_BYTES;          // 229376
 constexpr int SM_CTRL_BYTES = 1024;
 constexpr int PREFILL_SMEM = SM_CTRL + SM_CTRL_BYTES + 1024;  // + alignment slack
 
-constexpr uint32_t TM_SC = 0, TM_P = 128, TM_O = 256, TM_S = 384, TM_COLS = 512;
+constexpr uint32_t TM_SC = 0, TM_O0 = 128, TM_S = 384, TM_COLS = 512;  // O1 = TM_O0 + 128
 
 // device status codes (match la_status)
 constexpr int ST_INVALID = 1;
@@ -79,6 +97,7 @@ struct PrefillParams {
     const int4 *segs;       // [G] {seq, tok0, tok1, jinfo}
     int *flags;             // [G*H] 0 = empty, 2 = inclusive prefix published
     float *incl;            // [G*H][D*D] inclusive prefixes, column-quad interleaved
+    int seg_len;            // tokens per segment (the last one of a sequence may be shorter)
     unsigned long long wait_limit_ns;
     int inject;
     int *status;            // sticky device status word
@@ -86,8 +105,8 @@ struct PrefillParams {
 
 struct CtrlBlock {
     uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
-    uint64_t q_full, q_empty;
-    uint64_t sc_full, p_full, o_full, o_empty;
+    uint64_t q_full[Q_STAGES], q_empty[Q_STAGES];
+    uint64_t sc_full, p_full, o_full[2], o_empty[2];
     uint64_t s_done, snap_full, snap_empty, agg_full;
     uint64_t item_full[2], item_empty[2];
     uint64_t fin, pub;
@@ -98,7 +117,20 @@ struct CtrlBlock {
 static_assert(sizeof(CtrlBlock) <= SM_CTRL_BYTES, "control block too large");
 
 // item fields
-enum { IT_T = 0, IT_H, IT_TOK0, IT_TOK1, IT_J, IT_LAST, IT_SEQ, IT_VALID };
+enum { IT_T = 0, IT_H, IT_TOK0, IT_TOK1, IT_J, IT_FLAGS, IT_SEQ, IT_VALID };
+constexpr int ITF_LAST = 1;  // last segment of its sequence (no successor, no phase A)
+constexpr int ITF_LO = 2;    // inter-block product uses S = S_hi + S_lo
+
+// Precision of the inter-block product Q_b S_{<b}.  S is rounded to bf16 for
+// the tensor cores (relative error 2^-9).  S grows like sqrt(position) for the
+// unit-scaled inputs this operation sees, so up to LA_LO_SPLIT_FROM tokens into
+// a sequence a single bf16 term keeps the output error far inside the error
+// budget (max abs ~1e-2 at 64K tokens).  Segments that reach past it use
+// S = S_hi + S_lo, two bf16 terms with ~2^-16 relative error, at twice the
+// tensor-core and shared-memory cost of that product.
+#ifndef LA_LO_SPLIT_FROM
+#define LA_LO_SPLIT_FROM 65536
+#endif
 
 __device__ __forceinline__ void record_status(int *status, int code) {
     atomicCAS(status, 0, code);
@@ -150,6 +182,74 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&b);
 }
 
+// fp32 pair (bit patterns) -> packed bf16 pair (first value in the low half),
+// rounding the magnitude to nearest with ties away from zero: adding half an
+// ulp of bf16 to the sign-magnitude bits and keeping the upper 16.  Error
+// <= half an ulp like round-to-nearest-even (they differ only on exact ties);
+// integer-pipe work only, for finite inputs.
+__device__ __forceinline__ uint32_t bf16x2_round(uint32_t u0, uint32_t u1) {
+    return __byte_perm(u0 + 0x8000u, u1 + 0x8000u, 0x7632);
+}
+
+// Split two fp32 values (bit patterns u0, u1) into a bf16 pair `hi` (rounded
+// as in bf16x2_round) and a bf16 pair `lo` holding the exact fp32 residual
+// x - hi truncated to bf16, so that x = hi + lo to within 2^-16 |x|.
+// Integer and fp32-add work only (finite inputs).
+__device__ __forceinline__ void split_hi_lo(uint32_t u0, uint32_t u1, uint32_t &hi, uint32_t &lo) {
+    const uint32_t r0 = u0 + 0x8000u;
+    const uint32_t r1 = u1 + 0x8000u;
+    hi = __byte_perm(r0, r1, 0x7632);
+    const float l0 = __uint_as_float(u0) - __uint_as_float(r0 & 0xffff0000u);
+    const float l1 = __uint_as_float(u1) - __uint_as_float(r1 & 0xffff0000u);
+    lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
+}
+
+// Read S from TMEM and hand it to a5 through the snapshot buffer: either the
+// whole state as bf16 (one arrival), or, when `lo`, as bf16 hi + lo one
+// 64-column half at a time (two arrivals).  The first arrival on snap_full
+// also tells the MMA warp that S has been read, so a6 may overwrite it.
+__device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint8_t *slo, int r, int lane, bool lo,
+                                               uint32_t &snap_n, const PrefillParams &p, CtrlBlock *cb) {
+    uint32_t x[D];
+    tmem_ld_cols<D>(trow + TM_S, x);
+    if (!lo) {
+        if (!warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) return false;
+#pragma unroll
+        for (int q = 0; q < D / 8; ++q) {  // 16-byte chunks of 8 columns, two 64-column halves
+            const uint32_t off = (uint32_t)((q >> 3) * HALF_BYTES + r * 128 + (((q & 7) ^ (r & 7)) << 4));
+            *reinterpret_cast<uint4 *>(shi + off) =
+                make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
+                           bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7]));
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cb->snap_full);
+        ++snap_n;
+        return true;
+    }
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        if (!warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) return false;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // 16-byte chunks of 8 columns
+            uint32_t hv[4], lv[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                split_hi_lo(x[hf * 64 + 8 * q + 2 * w], x[hf * 64 + 8 * q + 2 * w + 1], hv[w], lv[w]);
+            const uint32_t off = (uint32_t)(r * 128 + ((q ^ (r & 7)) << 4));
+            *reinterpret_cast<uint4 *>(shi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+            *reinterpret_cast<uint4 *>(slo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&cb->snap_full);
+        ++snap_n;
+    }
+    return true;
+}
+
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
@@ -165,20 +265,22 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             mbar_init(&cb->kv_full[s], 1);
             mbar_init(&cb->kv_empty[s], 1);
         }
-        mbar_init(&cb->q_full, 1);
-        mbar_init(&cb->q_empty, 1);
+        for (int s = 0; s < Q_STAGES; ++s) {
+            mbar_init(&cb->q_full[s], 1);
+            mbar_init(&cb->q_empty[s], 1);
+        }
         mbar_init(&cb->sc_full, 1);
         mbar_init(&cb->p_full, 4);
-        mbar_init(&cb->o_full, 1);
-        mbar_init(&cb->o_empty, 4);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&cb->o_full[s], 1);
+            mbar_init(&cb->o_empty[s], 4);
+            mbar_init(&cb->item_full[s], 1);
+            mbar_init(&cb->item_empty[s], 9);
+        }
         mbar_init(&cb->s_done, 1);
         mbar_init(&cb->snap_full, 4);
         mbar_init(&cb->snap_empty, 1);
         mbar_init(&cb->agg_full, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&cb->item_full[s], 1);
-            mbar_init(&cb->item_empty[s], 5);
-        }
         mbar_init(&cb->fin, 1);
         mbar_init(&cb->pub, 4);
         cb->abort = 0;
@@ -202,9 +304,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         if (lane == 0) {
             const uint64_t pol_first = policy_evict_first();
             const uint64_t pol_last = policy_evict_last();
+            const uint64_t pol_norm = policy_evict_normal();
             uint32_t it = 0, kv_n = 0, q_n = 0;
             int kv_last_fill[KV_STAGES] = {-1, -1};
-            int q_last_fill = -1;
+            int q_last_fill[Q_STAGES] = {-1, -1};
             const int total = *reinterpret_cast<volatile int *>(&p.hdr[HDR_TOTAL]);
             bool ok = true;
             for (;;) {
@@ -224,7 +327,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     item[IT_TOK0] = seg.y;
                     item[IT_TOK1] = seg.z;
                     item[IT_J] = seg.w & (SEG_LAST - 1);
-                    item[IT_LAST] = (seg.w & SEG_LAST) ? 1 : 0;
+                    const int jj = seg.w & (SEG_LAST - 1);
+                    const long long seg_end = (long long)jj * p.seg_len + (seg.z - seg.y);
+                    item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) | (seg_end > LA_LO_SPLIT_FROM ? ITF_LO : 0);
                 }
                 mbar_arrive(&cb->item_full[islot]);
                 ++it;
@@ -232,11 +337,29 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 const int tok0 = seg.y, tok1 = seg.z;
                 const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
                 const bool last = (seg.w & SEG_LAST) != 0;
+                // L2 prefetch of whole [128 x 128] tiles (two 64-column boxes each)
+                auto prefetch_tile = [&](const CUtensorMap *m, int b, uint64_t pol) {
+                    if (b < nblk) {
+                        tma_prefetch_3d(m, 0, h, tok0 + b * BLK, pol);
+                        tma_prefetch_3d(m, 64, h, tok0 + b * BLK, pol);
+                    }
+                };
+                for (int b = 0; b < PF_KV; ++b) {
+                    prefetch_tile(&tmk, b, pol_last);
+                    prefetch_tile(&tmv, b, pol_last);
+                }
+                if (last)  // no phase A: the scan starts at once
+                    for (int b = 0; b < PF_Q; ++b) prefetch_tile(&tmq, b, pol_last);
                 if (!last) {  // phase A: K and V only; kept in L2 for phase O
                     for (int b = 0; b < nblk && ok; ++b) {
                         if (cb->abort) { ok = false; break; }
                         const int s = kv_n % KV_STAGES;
                         if (!wait_or_abort(&cb->kv_empty[s], ((kv_n / KV_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
+                        if (PF_KV > 0) {
+                            prefetch_tile(&tmk, b + PF_KV, pol_last);
+                            prefetch_tile(&tmv, b + PF_KV, pol_last);
+                        }
+                        if (b >= nblk - PF_Q) prefetch_tile(&tmq, b - (nblk - PF_Q), pol_last);  // phase O's first Q tiles
                         mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
                         const int row = tok0 + b * BLK;
                         uint8_t *kt = smem + SM_K + s * TILE_BYTES;
@@ -252,13 +375,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 for (int b = 0; b < nblk && ok; ++b) {  // phase O: Q, K, V
                     if (cb->abort) { ok = false; break; }
                     const int row = tok0 + b * BLK;
-                    if (!wait_or_abort(&cb->q_empty, (q_n & 1) ^ 1, p, cb)) { ok = false; break; }
-                    mbar_expect_tx(&cb->q_full, TILE_BYTES);
-                    uint8_t *qt = smem + SM_Q;
-                    tma_load_3d(qt, &tmq, &cb->q_full, 0, h, row, pol_first);
-                    tma_load_3d(qt + HALF_BYTES, &tmq, &cb->q_full, 64, h, row, pol_first);
-                    q_last_fill = q_n;
-                    ++q_n;
+                    if (PF_Q > 0) prefetch_tile(&tmq, b + PF_Q, pol_last);
                     const int s = kv_n % KV_STAGES;
                     if (!wait_or_abort(&cb->kv_empty[s], ((kv_n / KV_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
                     mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
@@ -270,6 +387,14 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     tma_load_3d(vt + HALF_BYTES, &tmv, &cb->kv_full[s], 64, h, row, pol_first);
                     kv_last_fill[s] = kv_n / KV_STAGES;
                     ++kv_n;
+                    const int qs = q_n % Q_STAGES;
+                    if (!wait_or_abort(&cb->q_empty[qs], ((q_n / Q_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
+                    mbar_expect_tx(&cb->q_full[qs], TILE_BYTES);
+                    uint8_t *qt = smem + SM_Q + qs * TILE_BYTES;
+                    tma_load_3d(qt, &tmq, &cb->q_full[qs], 0, h, row, pol_first);
+                    tma_load_3d(qt + HALF_BYTES, &tmq, &cb->q_full[qs], 64, h, row, pol_first);
+                    q_last_fill[qs] = q_n / Q_STAGES;
+                    ++q_n;
                 }
                 if (!ok) break;
             }
@@ -280,22 +405,28 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     int dummy = 0;
                     la_wait(&cb->kv_full[s], kv_last_fill[s] & 1, dl, &dummy);
                 }
-            if (q_last_fill >= 0) {
-                const uint64_t dl = globaltimer_ns() + p.wait_limit_ns;
-                int dummy = 0;
-                la_wait(&cb->q_full, q_last_fill & 1, dl, &dummy);
-            }
-            if (!ok) {
-                // unblock the consumers waiting for an item: hand them a stop item
-                cb->abort = 1;
-            }
+            for (int s = 0; s < Q_STAGES; ++s)
+                if (q_last_fill[s] >= 0) {
+                    const uint64_t dl = globaltimer_ns() + p.wait_limit_ns;
+                    int dummy = 0;
+                    la_wait(&cb->q_full[s], q_last_fill[s] & 1, dl, &dummy);
+                }
+            if (!ok) cb->abort = 1;
         }
     } else if (warp == 1) {
         // ===================== MMA issuer =====================
-        constexpr uint32_t ID_QK = idesc_bf16_f32(BLK, BLK, 0, 0);  // Q (K-major) x K (K-major)
-        constexpr uint32_t ID_QS = idesc_bf16_f32(BLK, D, 0, 1);    // Q (K-major) x S (MN-major)
-        constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1);      // K^T (MN) x V (MN)
-        constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1);    // P (TMEM) x V (MN)
+        // Phase O runs two dependency chains per block b:
+        //   intra chain:  a2(b) -> [mask] -> a4(b)            (needs Q, K, V tiles)
+        //   state chain:  a5 half 0 (S_{<b}) -> a6(b) -> a5 half 1
+        // a4(b) initialises the block's O buffer, the a5 halves accumulate onto it.
+        // Instead of a fixed program order, the issuing lane polls the barriers
+        // and issues whatever is ready, so the intra chain can run up to two
+        // blocks (the two O buffers) ahead of the state chain.
+        constexpr uint32_t ID_QK = idesc_bf16_f32(BLK, BLK, 0, 0);    // Q (K-major) x K (K-major)
+        constexpr uint32_t ID_QS = idesc_bf16_f32(BLK, D / 2, 0, 1);  // Q (K-major) x S half (MN-major)
+        constexpr uint32_t ID_QF = idesc_bf16_f32(BLK, D, 0, 1);      // Q (K-major) x S (MN-major)
+        constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1);        // K^T (MN) x V (MN)
+        constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1);      // P (TMEM) x V (MN)
         uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0;
         bool ok = true;
         while (ok) {
@@ -310,11 +441,14 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             if (!item[IT_VALID]) break;
             const int tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
-            const bool last = item[IT_LAST] != 0;
-            if (!last) {  // phase A: A_j = sum_b K_b^T V_b, accumulated in the O columns
-                // (S may still be read by the previous item's final-state store; O is
-                // free once the previous block's output has been read out)
-                if (!warp_wait(&cb->o_empty, (blk_n & 1) ^ 1, p, cb)) break;
+            const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
+            const bool lo = (item[IT_FLAGS] & ITF_LO) != 0;
+            if (!last) {
+                // phase A: A_j = sum_b K_b^T V_b, accumulated in the O buffer that
+                // the item's first block will use
+                const uint32_t ob0 = blk_n & 1;
+                if (!warp_wait(&cb->o_empty[ob0], ((blk_n >> 1) & 1) ^ 1, p, cb)) break;
+                tc_fence_after();
                 for (int b = 0; b < nblk; ++b) {
                     if (cb->abort) { ok = false; break; }
                     const int s = kv_n % KV_STAGES;
@@ -325,7 +459,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < BLK / 16; ++kk)
-                            mma_ss(tmem + TM_O, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
+                            mma_ss(tmem + TM_O0 + ob0 * 128, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
                                    (b > 0 || kk > 0) ? 1u : 0u);
                         tc_commit(&cb->kv_empty[s]);
                     }
@@ -336,75 +470,148 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 if (lane == 0) tc_commit(&cb->agg_full);
                 __syncwarp();
             }
+            // ---------------- phase O: polled two-chain schedule ----------------
             const bool want_final = last && p.state_out != nullptr;
-            for (int b = 0; b < nblk; ++b) {  // phase O
-                const int valid = min(BLK, tok1 - (tok0 + b * BLK));
-                const bool update = (b < nblk - 1) || want_final;
-                const int s = kv_n % KV_STAGES;
-                if (cb->abort) { ok = false; break; }
-                if (!warp_wait(&cb->q_full, q_n & 1, p, cb)) { ok = false; break; }
-                if (!warp_wait(&cb->kv_full[s], (kv_n / KV_STAGES) & 1, p, cb)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t qt = sbase + SM_Q;
-                const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
-                const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
-                if (valid < BLK) {
-                    // rows past the end of the sequence must add nothing to S or O:
-                    // zero them in K and V (they may hold the next sequence's tokens)
-                    uint8_t *kp = smem + SM_K + s * TILE_BYTES;
-                    uint8_t *vp = smem + SM_V + s * TILE_BYTES;
-                    const int nbytes = (BLK - valid) * 128;
-                    for (int half = 0; half < 2; ++half)
-                        for (int o = lane * 16; o < nbytes; o += 32 * 16) {
-                            *reinterpret_cast<uint4 *>(kp + half * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4 *>(vp + half * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+            const uint32_t kv0 = kv_n, q0 = q_n, blk0 = blk_n;
+            int i2 = 0, i4 = 0, i5 = 0, half = 0;  // next block of a2 / a4 / a5; a5 half pending
+            uint32_t spins = 0;
+            uint64_t deadline = 0;
+            while (i5 < nblk) {
+                int prog = 0;
+                if (lane == 0) {
+                    // intra chain, a4(i4): P ready and the O buffer free
+                    if (i4 < i2) {
+                        const uint32_t bn = blk0 + i4, ob = bn & 1;
+                        // a4 of the first block overwrites the O buffer that holds A_j:
+                        // it must wait until phase L has read A_j (first E snapshot out)
+                        const bool a_read = last || i4 > 0 || mbar_test(&cb->snap_full, snap_n & 1);
+                        if (a_read && mbar_test(&cb->p_full, bn & 1) &&
+                            mbar_test(&cb->o_empty[ob], ((bn >> 1) & 1) ^ 1)) {
+                            tc_fence_after();
+                            const int s = (kv0 + i4) % KV_STAGES;
+                            const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
+#pragma unroll
+                            for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns
+                                mma_ts(tmem + TM_O0 + ob * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV,
+                                       kk > 0 ? 1u : 0u);
+                            ++i4;
+                            prog = 1;
                         }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                if (lane == 0) {  // a2: Sc = Q K^T
+                    }
+                    // intra chain, a2(i2): score columns free (previous a4 issued), tiles landed
+                    if (i2 < nblk && i2 == i4) {
+                        const int s = (kv0 + i2) % KV_STAGES;
+                        const uint32_t kn = (kv0 + i2) / KV_STAGES, qn = q0 + i2;
+                        if (mbar_test(&cb->kv_full[s], kn & 1) &&
+                            mbar_test(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1))
+                            prog = 2;  // a2 is issued below, after the warp zeroes ragged rows
+                    }
+                    // state chain: a5 (one full-width pass, or half 0 (+ a6) then half 1)
+                    if (prog != 2 && i5 < i4 && mbar_test(&cb->snap_full, snap_n & 1)) {
+                        tc_fence_after();
+                        const uint32_t bn = blk0 + i5, ob = bn & 1;
+                        const int s = (kv0 + i5) % KV_STAGES;
+                        const uint32_t qn = q0 + i5;
+                        const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
+                        const uint32_t sh = sbase + SM_SHI, sl = sbase + SM_SLO;
+                        const bool upd = (i5 < nblk - 1) || want_final;
+                        if (!lo) {  // O += Q S_hi, S_hi = the whole [128 x 128] snapshot buffer
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK, kk > 0 ? 1u : 0u);
-                    tc_commit(&cb->sc_full);
-                }
-                __syncwarp();
-                if (!warp_wait(&cb->snap_full, snap_n & 1, p, cb)) { ok = false; break; }
-                if (!warp_wait(&cb->o_empty, (blk_n & 1) ^ 1, p, cb)) { ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {  // a5: O = Q S_hi + Q S_lo
-                    const uint32_t sh = sbase + SM_SHI, sl = sbase + SM_SLO;
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_ss(tmem + TM_O0 + ob * 128, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, 1u);
+                            tc_commit(&cb->snap_empty);
+                            ++snap_n;
+                        } else {
+                            const uint32_t to = tmem + TM_O0 + ob * 128 + half * 64;
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + TM_O, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_ss(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, 1u);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ss(tmem + TM_O, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
-                    tc_commit(&cb->snap_empty);
-                    tc_commit(&cb->q_empty);
-                    if (update) {  // a6: S += K^T V
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_ss(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
+                            tc_commit(&cb->snap_empty);
+                            ++snap_n;
+                        }
+                        if (!lo || half == 0) {
+                            if (upd) {  // a6: S += K^T V (S_{<b} has been read out)
+                                const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
+                                const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < BLK / 16; ++kk)
-                            mma_ss(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
-                        tc_commit(&cb->s_done);
+                                for (int kk = 0; kk < BLK / 16; ++kk)
+                                    mma_ss(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                                tc_commit(&cb->s_done);
+                            }
+                            tc_commit(&cb->kv_empty[s]);  // a2, a4 and a6 of this block are issued
+                        }
+                        if (lo && half == 0) {
+                            half = 1;
+                        } else {
+                            tc_commit(&cb->q_empty[qn % Q_STAGES]);
+                            tc_commit(&cb->o_full[ob]);
+                            half = 0;
+                            ++i5;
+                        }
+                        prog = 1;
                     }
                 }
-                __syncwarp();
-                ++q_n;
-                ++snap_n;
-                if (!warp_wait(&cb->p_full, blk_n & 1, p, cb)) { ok = false; break; }
-                tc_fence_after();
-                if (lane == 0) {  // a4: O += P V
+                prog = __shfl_sync(0xffffffffu, prog, 0);
+                if (prog == 2) {
+                    const int s = (kv0 + i2) % KV_STAGES;
+                    const int valid = min(BLK, tok1 - (tok0 + i2 * BLK));
+                    if (valid < BLK) {
+                        // rows past the end of the sequence must add nothing to S or O:
+                        // zero them in K and V (they may hold the next sequence's tokens)
+                        uint8_t *kp = smem + SM_K + s * TILE_BYTES;
+                        uint8_t *vp = smem + SM_V + s * TILE_BYTES;
+                        const int nbytes = (BLK - valid) * 128;
+                        for (int hh = 0; hh < 2; ++hh)
+                            for (int o = lane * 16; o < nbytes; o += 32 * 16) {
+                                *reinterpret_cast<uint4 *>(kp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                                *reinterpret_cast<uint4 *>(vp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                            }
+                        fence_proxy_async_smem();
+                    }
+                    __syncwarp();
+                    if (lane == 0) {  // a2: Sc = Q K^T
+                        tc_fence_after();
+                        const uint32_t qn = q0 + i2;
+                        const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
+                        const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
 #pragma unroll
-                    for (int kk = 0; kk < BLK / 16; ++kk)
-                        mma_ts(tmem + TM_O, tmem + TM_P + kk * 8, desc_mnmajor(vt, kk), ID_PV, 1u);
-                    tc_commit(&cb->o_full);
-                    tc_commit(&cb->kv_empty[s]);
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            mma_ss(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK, kk > 0 ? 1u : 0u);
+                        tc_commit(&cb->sc_full);
+                    }
+                    ++i2;
                 }
-                __syncwarp();
-                ++kv_n;
-                ++blk_n;
+                i2 = __shfl_sync(0xffffffffu, i2, 0);
+                i4 = __shfl_sync(0xffffffffu, i4, 0);
+                i5 = __shfl_sync(0xffffffffu, i5, 0);
+                half = __shfl_sync(0xffffffffu, half, 0);
+                snap_n = __shfl_sync(0xffffffffu, snap_n, 0);
+                if (prog) {
+                    spins = 0;
+                    deadline = 0;
+                } else if (((++spins) & 255u) == 0u) {
+                    int stop = 0;
+                    if (lane == 0) {
+                        const uint64_t now = globaltimer_ns();
+                        if (deadline == 0) deadline = now + p.wait_limit_ns;
+                        if (now > deadline || cb->abort) {
+                            cb->abort = 1;
+                            record_status(p.status, ST_TIMEOUT);
+                            stop = 1;
+                        }
+                    }
+                    if (__shfl_sync(0xffffffffu, stop, 0)) {
+                        ok = false;
+                        break;
+                    }
+                }
             }
+            kv_n = kv0 + nblk;
+            q_n = q0 + nblk;
+            blk_n = blk0 + nblk;
         }
         // Tear-down: all MMAs issued by this thread must finish before TMEM is freed.
         if (lane == 0) {
@@ -414,10 +621,92 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             la_wait(&cb->fin, 0, dl, &dummy);
         }
         __syncwarp();
-    } else {
-        // ===================== TMEM-lane owners (warps 2-5) =====================
+    } else if (warp < 6) {
+        // ============ warps 2-5: causal mask (a3) and output store (a7) ============
         const int q4 = warp & 3;               // TMEM lane quarter this warp may access
         const int r = q4 * 32 + lane;          // tile row = TMEM lane
+        const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+        uint32_t it = 0, blk_n = 0;
+        bool ok = true;
+        // O of block b -> out; the O buffer is released as soon as it is in registers
+        auto store_block = [&](uint32_t bn, int row0, int valid, int h) -> bool {
+            const uint32_t ob = bn & 1;
+            if (!warp_wait(&cb->o_full[ob], (bn >> 1) & 1, p, cb)) return false;
+            tc_fence_after();
+            uint32_t x[D];
+            tmem_ld_cols<D>(trow + TM_O0 + ob * 128, x);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&cb->o_empty[ob]);
+            if (r < valid) {
+                const size_t orow = ((size_t)(row0 + r) * H + h) * D;
+                if (p.out_fp32) {
+                    float *o = reinterpret_cast<float *>(p.out) + orow;
+#pragma unroll
+                    for (int q = 0; q < D / 4; ++q)
+                        __stcs(reinterpret_cast<float4 *>(o + 4 * q),
+                               make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
+                                           __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3])));
+                } else {
+                    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out) + orow;
+#pragma unroll
+                    for (int q = 0; q < D / 8; ++q) {
+                        uint4 u;
+                        u.x = bf16x2_round(x[8 * q], x[8 * q + 1]);
+                        u.y = bf16x2_round(x[8 * q + 2], x[8 * q + 3]);
+                        u.z = bf16x2_round(x[8 * q + 4], x[8 * q + 5]);
+                        u.w = bf16x2_round(x[8 * q + 6], x[8 * q + 7]);
+                        __stcs(reinterpret_cast<uint4 *>(o + 8 * q), u);
+                    }
+                }
+            }
+            return true;
+        };
+        while (ok) {
+            const int islot = it & 1;
+            if (!warp_wait(&cb->item_full[islot], (it >> 1) & 1, p, cb)) break;
+            int item[8];
+#pragma unroll
+            for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&cb->item_empty[islot]);
+            ++it;
+            if (!item[IT_VALID]) break;
+            const int h = item[IT_H], tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
+            const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
+            for (int b = 0; b < nblk; ++b) {
+                // a3: P = bf16(Sc ⊙ M), inclusive mask; written over the first 64 score columns
+                if (!warp_wait(&cb->sc_full, (blk_n + b) & 1, p, cb)) { ok = false; break; }
+                tc_fence_after();
+                {
+                    uint32_t x[BLK];
+                    tmem_ld_cols<BLK>(trow + TM_SC, x);
+                    // packed in place: x[w] <- (x[2w], x[2w+1]) only overwrites words already read
+#pragma unroll
+                    for (int w = 0; w < BLK / 2; ++w)
+                        x[w] = bf16x2_round((2 * w <= r) ? x[2 * w] : 0u, (2 * w + 1 <= r) ? x[2 * w + 1] : 0u);
+#pragma unroll
+                    for (int c = 0; c < BLK / 32; ++c)
+                        tmem_st16(trow + TM_SC + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&x[c * 16]));
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cb->p_full);
+                // a7 for the previous block, while the MMA warp works on this one
+                if (b > 0 && !store_block(blk_n + b - 1, tok0 + (b - 1) * BLK, min(BLK, tok1 - tok0 - (b - 1) * BLK), h)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok && !store_block(blk_n + nblk - 1, tok0 + (nblk - 1) * BLK, tok1 - tok0 - (nblk - 1) * BLK, h))
+                ok = false;
+            blk_n += nblk;
+        }
+    } else {
+        // ===== warps 6-9: segment hand-off (phase L), state snapshots, final state =====
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         uint32_t it = 0, blk_n = 0, snap_n = 0, upd_n = 0, agg_n = 0, pub_n = 0;
         uint8_t *shi = smem + SM_SHI;
@@ -434,8 +723,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             if (!item[IT_VALID]) break;
             const int t = item[IT_T], h = item[IT_H], seq = item[IT_SEQ];
             const int tok0 = item[IT_TOK0], tok1 = item[IT_TOK1], j = item[IT_J];
-            const bool last = item[IT_LAST] != 0;
+            const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
+            const bool lo = (item[IT_FLAGS] & ITF_LO) != 0;
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
+            const uint32_t ob0 = blk_n & 1;
             bool ok = true;
 
             // ---------------- phase L: prefix of this segment ----------------
@@ -472,69 +763,50 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 ++agg_n;
                 tc_fence_after();
             }
-            // the snapshot buffer must be free (a5 of the previous block done)
-            if (!warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) ok = false;
             float *dst_incl = p.incl + (size_t)t * D * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float e[32];
+            for (int hf = 0; hf < 2; ++hf) {  // two halves of 64 columns
+                float e[64];
                 if (src_incl && ok) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 x = __ldcg(reinterpret_cast<const float4 *>(src_incl + incl_off(r, c * 8 + q)));
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 x = __ldcg(reinterpret_cast<const float4 *>(src_incl + incl_off(r, hf * 16 + q)));
                         e[4 * q] = x.x; e[4 * q + 1] = x.y; e[4 * q + 2] = x.z; e[4 * q + 3] = x.w;
                     }
                 } else if (src_state) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const float4 x = __ldg(reinterpret_cast<const float4 *>(src_state + (size_t)r * D + c * 32 + 4 * q));
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 x = __ldg(reinterpret_cast<const float4 *>(src_state + (size_t)r * D + hf * 64 + 4 * q));
                         e[4 * q] = x.x; e[4 * q + 1] = x.y; e[4 * q + 2] = x.z; e[4 * q + 3] = x.w;
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) e[q] = 0.f;
+                    for (int q = 0; q < 64; ++q) e[q] = 0.f;
                 }
-                if (!last) {  // INCL_j = E_j + A_j  (A_j sits in the O columns)
-                    uint32_t a[32];
-                    tmem_ld32(trow + TM_O + c * 32, a);
-                    tmem_wait_ld();
+                if (!last) {  // INCL_j = E_j + A_j  (A_j sits in an O buffer)
+                    uint32_t a[64];
+                    tmem_ld_cols<64>(trow + TM_O0 + ob0 * 128 + hf * 64, a);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
+                    for (int q = 0; q < 16; ++q) {
                         float4 x;
                         x.x = e[4 * q] + __uint_as_float(a[4 * q]);
                         x.y = e[4 * q + 1] + __uint_as_float(a[4 * q + 1]);
                         x.z = e[4 * q + 2] + __uint_as_float(a[4 * q + 2]);
                         x.w = e[4 * q + 3] + __uint_as_float(a[4 * q + 3]);
-                        __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, c * 8 + q)), x);
+                        __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, hf * 16 + q)), x);
                     }
                 }
-                // S (TMEM) = E_j for the scan, and its bf16 hi/lo split for a5
-                uint32_t eu[32];
-#pragma unroll
-                for (int q = 0; q < 32; ++q) eu[q] = __float_as_uint(e[q]);
-                tmem_st32(trow + TM_S + c * 32, eu);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {  // 4 chunks of 8 columns
-                    uint32_t hv[4], lv[4];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const float x0 = e[8 * q + 2 * w], x1 = e[8 * q + 2 * w + 1];
-                        const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-                        hv[w] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-                        lv[w] = pack_bf16x2(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-                    }
-                    const uint32_t off = sw_off(r, c * 4 + q);
-                    *reinterpret_cast<uint4 *>(shi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                    *reinterpret_cast<uint4 *>(slo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-                }
+                // S (TMEM) = E_j: the state the scan of this segment starts from
+                tmem_st32(trow + TM_S + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&e[0]));
+                tmem_st32(trow + TM_S + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&e[32]));
             }
-            fence_proxy_async_smem();
             tmem_wait_st();
-            tc_fence_before();
+            // hand E_j to a5 (this also releases A_j's O buffer and lets a6 start)
+            if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) ok = false;
             if (!last) {
-                // publish INCL_j: every warp fences its stores and arrives; the
+                // publish INCL_j: every warp orders its stores and arrives; the
                 // owner of row 0 waits (bounded) for all four, then releases the flag
-                __threadfence();
+                asm volatile("fence.acq_rel.gpu;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cb->pub);
                 if (r == 0) {
@@ -547,124 +819,31 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
                 ++pub_n;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&cb->snap_full);
-            ++snap_n;
             if (!__all_sync(0xffffffffu, ok && !cb->abort)) break;
 
-            // ---------------- phase O: blocked scan ----------------
+            // ------------- phase O: state snapshots and the final state -------------
             const bool want_final = last && p.state_out != nullptr;
             for (int b = 0; b < nblk; ++b) {
-                const int row0 = tok0 + b * BLK;
-                const int valid = min(BLK, tok1 - row0);
                 const bool update = (b < nblk - 1) || want_final;
-                // a3: P = bf16(Sc ⊙ M), inclusive causal mask inside the block
-                if (!warp_wait(&cb->sc_full, blk_n & 1, p, cb)) { ok = false; break; }
+                if (!update) continue;
+                if (!warp_wait(&cb->s_done, upd_n & 1, p, cb)) { ok = false; break; }
+                ++upd_n;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c = 0; c < BLK / 32; ++c) {
-                    uint32_t x[32];
-                    tmem_ld32(trow + TM_SC + c * 32, x);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
+                if (b < nblk - 1) {
+                    if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }  // S_{<b+1} for the next block
+                } else {
+                    // final state of the sequence -> state_out (row-major fp32)
+                    uint32_t x[D];
+                    tmem_ld_cols<D>(trow + TM_S, x);
+                    float *so = p.state_out + ((size_t)seq * H + h) * D * D + (size_t)r * D;
 #pragma unroll
-                    for (int w = 0; w < 16; ++w) {
-                        const int s0 = c * 32 + 2 * w;
-                        const float a0 = (s0 <= r) ? __uint_as_float(x[2 * w]) : 0.f;
-                        const float a1 = (s0 + 1 <= r) ? __uint_as_float(x[2 * w + 1]) : 0.f;
-                        pk[w] = pack_bf16x2(a0, a1);
-                    }
-                    tmem_st16(trow + TM_P + c * 16, pk);
+                    for (int q = 0; q < D / 4; ++q)
+                        *reinterpret_cast<float4 *>(so + 4 * q) =
+                            make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
+                                        __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3]));
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->p_full);
-                if (update) {
-                    if (!warp_wait(&cb->s_done, upd_n & 1, p, cb)) { ok = false; break; }
-                    ++upd_n;
-                    tc_fence_after();
-                    if (b < nblk - 1) {
-                        // snapshot S_{<b+1} as bf16 hi + lo for the next block's a5
-                        if (!warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) { ok = false; break; }
-#pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t x[32];
-                            tmem_ld32(trow + TM_S + c * 32, x);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint32_t hv[4], lv[4];
-#pragma unroll
-                                for (int w = 0; w < 4; ++w) {
-                                    const float x0 = __uint_as_float(x[8 * q + 2 * w]);
-                                    const float x1 = __uint_as_float(x[8 * q + 2 * w + 1]);
-                                    const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
-                                    hv[w] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-                                    lv[w] = pack_bf16x2(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
-                                }
-                                const uint32_t off = sw_off(r, c * 4 + q);
-                                *reinterpret_cast<uint4 *>(shi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-                                *reinterpret_cast<uint4 *>(slo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-                            }
-                        }
-                        fence_proxy_async_smem();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&cb->snap_full);
-                        ++snap_n;
-                    } else {
-                        // final state of the sequence -> state_out (row-major fp32)
-                        float *so = p.state_out + ((size_t)seq * H + h) * D * D + (size_t)r * D;
-#pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t x[32];
-                            tmem_ld32(trow + TM_S + c * 32, x);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                *reinterpret_cast<float4 *>(so + c * 32 + 4 * q) =
-                                    make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
-                                                __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3]));
-                        }
-                    }
-                }
-                // a7: O -> out
-                if (!warp_wait(&cb->o_full, blk_n & 1, p, cb)) { ok = false; break; }
-                tc_fence_after();
-                const size_t orow = ((size_t)(row0 + r) * H + h) * D;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t x[32];
-                    tmem_ld32(trow + TM_O + c * 32, x);
-                    tmem_wait_ld();
-                    if (r < valid) {
-                        if (p.out_fp32) {
-                            float *o = reinterpret_cast<float *>(p.out) + orow + c * 32;
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                __stcs(reinterpret_cast<float4 *>(o + 4 * q),
-                                       make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
-                                                   __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3])));
-                        } else {
-                            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out) + orow + c * 32;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                uint4 u;
-                                u.x = pack_bf16x2(__uint_as_float(x[8 * q]), __uint_as_float(x[8 * q + 1]));
-                                u.y = pack_bf16x2(__uint_as_float(x[8 * q + 2]), __uint_as_float(x[8 * q + 3]));
-                                u.z = pack_bf16x2(__uint_as_float(x[8 * q + 4]), __uint_as_float(x[8 * q + 5]));
-                                u.w = pack_bf16x2(__uint_as_float(x[8 * q + 6]), __uint_as_float(x[8 * q + 7]));
-                                __stcs(reinterpret_cast<uint4 *>(o + 8 * q), u);
-                            }
-                        }
-                    }
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->o_empty);
-                ++blk_n;
             }
+            blk_n += nblk;
             if (!ok) break;
         }
     }

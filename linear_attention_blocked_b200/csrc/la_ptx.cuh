@@ -56,6 +56,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete.
 // Returns false if `deadline` (globaltimer ns) passed or *abort became nonzero.
 __device__ __forceinline__ bool la_wait(uint64_t *bar, uint32_t parity, uint64_t deadline,
@@ -103,6 +114,14 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *tmap, uint64_
         " [%0], [%1, {%2, %3, %4}], [%5], %6;"
         ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2),
           "r"(smem_u32(bar)), "l"(cache_hint)
+        : "memory");
+}
+
+// 3-D tile prefetch global -> L2 (no shared memory, no completion tracking).
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int c0, int c1, int c2, uint64_t cache_hint) {
+    asm volatile(
+        "cp.async.bulk.prefetch.tensor.3d.L2.global.tile.L2::cache_hint [%0, {%1, %2, %3}], %4;"
+        ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "l"(cache_hint)
         : "memory");
 }
 
@@ -183,6 +202,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// After tmem_wait_ld(): tie every loaded register to a point after the wait
+// so that no use of it can be scheduled above the wait.
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// Load `N` (multiple of 32) consecutive columns of this warp's 32 lanes,
+// issued back to back, with a single wait at the end.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    static_assert(N % 32 == 0, "whole 32-column groups");
+#pragma unroll
+    for (int c = 0; c < N / 32; ++c)
+        tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&r[c * 32]));
+    tmem_wait_ld();
+    reg_fence(r);
 }
 
 // 32 lanes x 16 columns store

@@ -196,3 +196,18 @@ def test_kernel_launch_count_increases():
     la.prefill(q, k, v)
     torch.cuda.synchronize()
     assert la.kernel_launches() == before + 2    # scheduler + prefill
+
+
+def test_long_sequence_uses_split_state_and_stays_accurate(oracle_mod):
+    """128K tokens: segments past token 65536 switch the inter-block product to
+    the two-term (bf16 hi + lo) state; fp32 outputs stay within 2e-2 max abs
+    everywhere along the sequence."""
+    B, N, H = 1, 131072, 2
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=13, device="cuda")
+    out, st = la.prefill(q, k, v, out_dtype=torch.float32)
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = _oracle_prefill(oracle_mod, q[0], k[0], v[0], np.array([0, N], np.int32))
+    got = to_np(out[0])
+    for lo, hi in ((0, 65536), (65536, N)):   # both precision regimes
+        check_out(got[lo:hi], ref[lo:hi], bf16_out=False, what=f"tokens [{lo}, {hi})")
+    check_state(to_np(st[0]), rst[0])
