@@ -48,18 +48,21 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// [T, H, 128] bf16 viewed as a 3-D tensor {128, H, T}; box {64, 1, 128},
-// 128-byte swizzle, zero fill outside the tensor.
+// [T, H, 128] bf16 viewed as a 4-D tensor {64, H, T, 2}: dimension 0 = the
+// 64 features of one half, 1 = head (256-byte stride), 2 = token (H*256-byte
+// stride), 3 = which half (128-byte stride).  A box {64, 1, 128, 2} loads both
+// halves of 128 tokens as two [128 x 64] blocks with the 128-byte swizzle; zero
+// fill outside the tensor.
 bool encode_qkv_map(CUtensorMap *map, const void *base, int T, int H) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)la::D, (cuuint64_t)H, (cuuint64_t)T};
-    const cuuint64_t strides[2] = {(cuuint64_t)la::D * 2, (cuuint64_t)H * la::D * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)la::BLK};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const cuuint64_t dims[4] = {64, (cuuint64_t)H, (cuuint64_t)T, 2};
+    const cuuint64_t strides[3] = {(cuuint64_t)la::D * 2, (cuuint64_t)H * la::D * 2, 128};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)la::BLK, 2};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 int device_sm_count() {
@@ -184,10 +187,15 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     ++g_launches;
     if (T == 0) return LA_OK;
 
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
         !encode_qkv_map(&mv, v, (int)T, H))
         return LA_ERR_CUDA;
+    if (out_dtype == LA_BF16) {  // bf16 output tiles leave through TMA stores with the same geometry
+        if (!encode_qkv_map(&mo, out, (int)T, H)) return LA_ERR_CUDA;
+    } else {
+        mo = mq;  // unused: fp32 outputs are written with plain stores
+    }
 
     la::PrefillParams pp;
     pp.state_in = state_in;
@@ -213,7 +221,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     if (attr_err != cudaSuccess) return LA_ERR_CUDA;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, mo, pp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;
@@ -445,10 +453,15 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     ++g_launches;
     if (T == 0) return LA_OK;
 
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
         !encode_qkv_map(&mv, v, (int)T, H))
         return LA_ERR_CUDA;
+    if (out_dtype == LA_BF16) {  // bf16 output tiles leave through TMA stores with the same geometry
+        if (!encode_qkv_map(&mo, out, (int)T, H)) return LA_ERR_CUDA;
+    } else {
+        mo = mq;  // unused: fp32 outputs are written with plain stores
+    }
     la::PrefillParams pp;
     pp.state_in = state_in;
     pp.state_out = state_out;
@@ -468,7 +481,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
         return LA_ERR_CUDA;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, mo, pp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;

@@ -31,10 +31,12 @@
 //   K ring 2 x 32 KiB | V ring 2 x 32 KiB | Q ring 2 x 32 KiB | S_hi half 16 KiB |
 //   S_lo half 16 KiB | barriers + item queue.
 // A [128 x 128] bf16 tile is two 16 KiB halves (columns 0-63, 64-127), each
-// 128 rows of 128 bytes as TMA writes them with a {64, 1, 128} box.
-// TMEM (512 columns x 128 lanes x 32 bit): Sc [0,128) (P overwrites its first
-//   64 columns in place) | O0 [128,256) | O1 [256,384) (double-buffered output)
-//   | S [384,512).
+// 128 rows of 128 bytes, written by one TMA box {64, 1, 128, 2} of the 4-D
+// view {64, H, T, 2} of the [T, H, 128] tensor (the halves are its outer
+// dimension).
+// TMEM (512 columns x 128 lanes x 32 bit): Sc0 [0,128) | Sc1 [128,256)
+//   (double-buffered scores; P overwrites the first 64 columns of its buffer in
+//   place) | O [256,384) | S [384,512).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -61,6 +63,9 @@ constexpr int PREFILL_THREADS = 320;
 #define LA_PREFETCH_KV 0
 #endif
 constexpr int PF_Q = LA_PREFETCH_Q;
+#ifndef LA_PHASE_A_Q_PREFETCH
+#define LA_PHASE_A_Q_PREFETCH 0
+#endif
 constexpr int PF_KV = LA_PREFETCH_KV;
 
 constexpr int SM_K = 0;
@@ -73,7 +78,7 @@ constexpr int SM_CTRL = SM_SLO + HALF_BYTES;          // 229376
 constexpr int SM_CTRL_BYTES = 1024;
 constexpr int PREFILL_SMEM = SM_CTRL + SM_CTRL_BYTES + 1024;  // + alignment slack
 
-constexpr uint32_t TM_SC = 0, TM_O0 = 128, TM_S = 384, TM_COLS = 512;  // O1 = TM_O0 + 128
+constexpr uint32_t TM_SC = 0, TM_O = 256, TM_S = 384, TM_COLS = 512;  // SC1 = TM_SC + 128
 
 // device status codes (match la_status)
 constexpr int ST_INVALID = 1;
@@ -106,10 +111,10 @@ struct PrefillParams {
 struct CtrlBlock {
     uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
     uint64_t q_full[Q_STAGES], q_empty[Q_STAGES];
-    uint64_t sc_full, p_full, o_full[2], o_empty[2];
+    uint64_t sc_full[2], p_full[2], o_full, o_empty;
     uint64_t s_done, snap_full, snap_empty, agg_full;
     uint64_t item_full[2], item_empty[2];
-    uint64_t fin, pub;
+    uint64_t fin, pub, ostage;
     int item[2][8];
     uint32_t tmem_base;
     volatile int abort;
@@ -252,7 +257,8 @@ __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint
 
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
+                  const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -269,11 +275,11 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             mbar_init(&cb->q_full[s], 1);
             mbar_init(&cb->q_empty[s], 1);
         }
-        mbar_init(&cb->sc_full, 1);
-        mbar_init(&cb->p_full, 4);
+        mbar_init(&cb->o_full, 1);
+        mbar_init(&cb->o_empty, 4);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&cb->o_full[s], 1);
-            mbar_init(&cb->o_empty[s], 4);
+            mbar_init(&cb->sc_full[s], 1);
+            mbar_init(&cb->p_full[s], 4);
             mbar_init(&cb->item_full[s], 1);
             mbar_init(&cb->item_empty[s], 9);
         }
@@ -283,11 +289,13 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         mbar_init(&cb->agg_full, 1);
         mbar_init(&cb->fin, 1);
         mbar_init(&cb->pub, 4);
+        mbar_init(&cb->ostage, 4);
         cb->abort = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
+        if (!p.out_fp32) tma_prefetch_desc(&tmo);
     }
     if (warp == 1) {
         tmem_alloc(&cb->tmem_base, TM_COLS);
@@ -339,10 +347,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 const bool last = (seg.w & SEG_LAST) != 0;
                 // L2 prefetch of whole [128 x 128] tiles (two 64-column boxes each)
                 auto prefetch_tile = [&](const CUtensorMap *m, int b, uint64_t pol) {
-                    if (b < nblk) {
-                        tma_prefetch_3d(m, 0, h, tok0 + b * BLK, pol);
-                        tma_prefetch_3d(m, 64, h, tok0 + b * BLK, pol);
-                    }
+                    if (b < nblk) tma_prefetch_4d(m, 0, h, tok0 + b * BLK, 0, pol);
                 };
                 for (int b = 0; b < PF_KV; ++b) {
                     prefetch_tile(&tmk, b, pol_last);
@@ -359,15 +364,17 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                             prefetch_tile(&tmk, b + PF_KV, pol_last);
                             prefetch_tile(&tmv, b + PF_KV, pol_last);
                         }
+#if LA_PHASE_A_Q_PREFETCH
+                        prefetch_tile(&tmq, b, pol_last);  // phase O then finds Q in L2 as well as K and V
+#else
                         if (b >= nblk - PF_Q) prefetch_tile(&tmq, b - (nblk - PF_Q), pol_last);  // phase O's first Q tiles
+#endif
                         mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
                         const int row = tok0 + b * BLK;
                         uint8_t *kt = smem + SM_K + s * TILE_BYTES;
                         uint8_t *vt = smem + SM_V + s * TILE_BYTES;
-                        tma_load_3d(kt, &tmk, &cb->kv_full[s], 0, h, row, pol_last);
-                        tma_load_3d(kt + HALF_BYTES, &tmk, &cb->kv_full[s], 64, h, row, pol_last);
-                        tma_load_3d(vt, &tmv, &cb->kv_full[s], 0, h, row, pol_last);
-                        tma_load_3d(vt + HALF_BYTES, &tmv, &cb->kv_full[s], 64, h, row, pol_last);
+                        tma_load_4d(kt, &tmk, &cb->kv_full[s], 0, h, row, 0, pol_last);
+                        tma_load_4d(vt, &tmv, &cb->kv_full[s], 0, h, row, 0, pol_last);
                         kv_last_fill[s] = kv_n / KV_STAGES;
                         ++kv_n;
                     }
@@ -381,18 +388,15 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
                     uint8_t *kt = smem + SM_K + s * TILE_BYTES;
                     uint8_t *vt = smem + SM_V + s * TILE_BYTES;
-                    tma_load_3d(kt, &tmk, &cb->kv_full[s], 0, h, row, pol_first);
-                    tma_load_3d(kt + HALF_BYTES, &tmk, &cb->kv_full[s], 64, h, row, pol_first);
-                    tma_load_3d(vt, &tmv, &cb->kv_full[s], 0, h, row, pol_first);
-                    tma_load_3d(vt + HALF_BYTES, &tmv, &cb->kv_full[s], 64, h, row, pol_first);
+                    tma_load_4d(kt, &tmk, &cb->kv_full[s], 0, h, row, 0, pol_first);
+                    tma_load_4d(vt, &tmv, &cb->kv_full[s], 0, h, row, 0, pol_first);
                     kv_last_fill[s] = kv_n / KV_STAGES;
                     ++kv_n;
                     const int qs = q_n % Q_STAGES;
                     if (!wait_or_abort(&cb->q_empty[qs], ((q_n / Q_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
                     mbar_expect_tx(&cb->q_full[qs], TILE_BYTES);
                     uint8_t *qt = smem + SM_Q + qs * TILE_BYTES;
-                    tma_load_3d(qt, &tmq, &cb->q_full[qs], 0, h, row, pol_first);
-                    tma_load_3d(qt + HALF_BYTES, &tmq, &cb->q_full[qs], 64, h, row, pol_first);
+                    tma_load_4d(qt, &tmq, &cb->q_full[qs], 0, h, row, 0, pol_first);
                     q_last_fill[qs] = q_n / Q_STAGES;
                     ++q_n;
                 }
@@ -444,10 +448,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
             const bool lo = (item[IT_FLAGS] & ITF_LO) != 0;
             if (!last) {
-                // phase A: A_j = sum_b K_b^T V_b, accumulated in the O buffer that
-                // the item's first block will use
-                const uint32_t ob0 = blk_n & 1;
-                if (!warp_wait(&cb->o_empty[ob0], ((blk_n >> 1) & 1) ^ 1, p, cb)) break;
+                // phase A: A_j = sum_b K_b^T V_b, accumulated in the O columns once
+                // the previous block's output has been read out
+                if (!warp_wait(&cb->o_empty, (blk_n & 1) ^ 1, p, cb)) break;
                 tc_fence_after();
                 for (int b = 0; b < nblk; ++b) {
                     if (cb->abort) { ok = false; break; }
@@ -459,7 +462,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < BLK / 16; ++kk)
-                            mma_ss(tmem + TM_O0 + ob0 * 128, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
+                            mma_ss(tmem + TM_O, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
                                    (b > 0 || kk > 0) ? 1u : 0u);
                         tc_commit(&cb->kv_empty[s]);
                     }
@@ -481,25 +484,26 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 if (lane == 0) {
                     // intra chain, a4(i4): P ready and the O buffer free
                     if (i4 < i2) {
-                        const uint32_t bn = blk0 + i4, ob = bn & 1;
-                        // a4 of the first block overwrites the O buffer that holds A_j:
+                        const uint32_t bn = blk0 + i4;
+                        // a4 of the first block overwrites the O columns that hold A_j:
                         // it must wait until phase L has read A_j (first E snapshot out)
                         const bool a_read = last || i4 > 0 || mbar_test(&cb->snap_full, snap_n & 1);
-                        if (a_read && mbar_test(&cb->p_full, bn & 1) &&
-                            mbar_test(&cb->o_empty[ob], ((bn >> 1) & 1) ^ 1)) {
+                        if (a_read && mbar_test(&cb->p_full[bn & 1], (bn >> 1) & 1) &&
+                            mbar_test(&cb->o_empty, (bn & 1) ^ 1)) {
                             tc_fence_after();
                             const int s = (kv0 + i4) % KV_STAGES;
                             const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                             for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns
-                                mma_ts(tmem + TM_O0 + ob * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV,
+                                mma_ts(tmem + TM_O, tmem + TM_SC + (bn & 1) * 128 + kk * 8, desc_mnmajor(vt, kk), ID_PV,
                                        kk > 0 ? 1u : 0u);
                             ++i4;
                             prog = 1;
                         }
                     }
-                    // intra chain, a2(i2): score columns free (previous a4 issued), tiles landed
-                    if (i2 < nblk && i2 == i4) {
+                    // intra chain, a2(i2): its score buffer free (a4 of block i2 - 2
+                    // issued), tiles landed
+                    if (i2 < nblk && i2 < i4 + 2) {
                         const int s = (kv0 + i2) % KV_STAGES;
                         const uint32_t kn = (kv0 + i2) / KV_STAGES, qn = q0 + i2;
                         if (mbar_test(&cb->kv_full[s], kn & 1) &&
@@ -509,7 +513,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     // state chain: a5 (one full-width pass, or half 0 (+ a6) then half 1)
                     if (prog != 2 && i5 < i4 && mbar_test(&cb->snap_full, snap_n & 1)) {
                         tc_fence_after();
-                        const uint32_t bn = blk0 + i5, ob = bn & 1;
+                        const uint32_t bn = blk0 + i5;
                         const int s = (kv0 + i5) % KV_STAGES;
                         const uint32_t qn = q0 + i5;
                         const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
@@ -518,11 +522,11 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         if (!lo) {  // O += Q S_hi, S_hi = the whole [128 x 128] snapshot buffer
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(tmem + TM_O0 + ob * 128, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, 1u);
+                                mma_ss(tmem + TM_O, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, 1u);
                             tc_commit(&cb->snap_empty);
                             ++snap_n;
                         } else {
-                            const uint32_t to = tmem + TM_O0 + ob * 128 + half * 64;
+                            const uint32_t to = tmem + TM_O + half * 64;
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
                                 mma_ss(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, 1u);
@@ -546,8 +550,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         if (lo && half == 0) {
                             half = 1;
                         } else {
-                            tc_commit(&cb->q_empty[qn % Q_STAGES]);
-                            tc_commit(&cb->o_full[ob]);
+                            tc_commit(&cb->o_full);  // also: Q of this block is no longer read
                             half = 0;
                             ++i5;
                         }
@@ -579,8 +582,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)
-                            mma_ss(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK, kk > 0 ? 1u : 0u);
-                        tc_commit(&cb->sc_full);
+                            mma_ss(tmem + TM_SC + ((blk0 + i2) & 1) * 128, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
+                                   kk > 0 ? 1u : 0u);
+                        tc_commit(&cb->sc_full[(blk0 + i2) & 1]);
                     }
                     ++i2;
                 }
@@ -628,16 +632,48 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         uint32_t it = 0, blk_n = 0;
         bool ok = true;
-        // O of block b -> out; the O buffer is released as soon as it is in registers
+        uint32_t ostage_n = 0;
+        // O of block b -> out.  The O buffer is released as soon as it is in
+        // registers.  A full bf16 block is staged in the shared-memory slot of
+        // its own Q tile (o_full means every MMA that read that Q is done) and
+        // written by one TMA bulk store (full 128-byte lines); the slot goes
+        // back to the producer once the store has read it.  A ragged block
+        // (it must not write past the sequence) and fp32 outputs use direct
+        // 16-byte stores instead.
         auto store_block = [&](uint32_t bn, int row0, int valid, int h) -> bool {
-            const uint32_t ob = bn & 1;
-            if (!warp_wait(&cb->o_full[ob], (bn >> 1) & 1, p, cb)) return false;
+            if (!warp_wait(&cb->o_full, bn & 1, p, cb)) return false;
             tc_fence_after();
             uint32_t x[D];
-            tmem_ld_cols<D>(trow + TM_O0 + ob * 128, x);
+            tmem_ld_cols<D>(trow + TM_O, x);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&cb->o_empty[ob]);
+            if (lane == 0) mbar_arrive(&cb->o_empty);
+            const int qslot = bn % Q_STAGES;
+            if (!p.out_fp32 && valid == BLK) {
+                uint8_t *stage = smem + SM_Q + qslot * TILE_BYTES;
+#pragma unroll
+                for (int q = 0; q < D / 8; ++q) {
+                    const uint32_t off = (uint32_t)((q >> 3) * HALF_BYTES + r * 128 + (((q & 7) ^ (r & 7)) << 4));
+                    *reinterpret_cast<uint4 *>(stage + off) =
+                        make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
+                                   bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cb->ostage);
+                bool ok2 = true;
+                if (r == 0) {
+                    ok2 = wait_or_abort(&cb->ostage, ostage_n & 1, p, cb);
+                    if (ok2) {
+                        tma_store_4d(&tmo, stage, 0, h, row0, 0);
+                        bulk_commit_group();
+                        bulk_wait_read_all();
+                        mbar_arrive(&cb->q_empty[qslot]);
+                    }
+                }
+                ++ostage_n;
+                return __all_sync(0xffffffffu, ok2) != 0;
+            }
             if (r < valid) {
                 const size_t orow = ((size_t)(row0 + r) * H + h) * D;
                 if (p.out_fp32) {
@@ -660,6 +696,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                 }
             }
+            if (r == 0) mbar_arrive(&cb->q_empty[qslot]);  // the Q slot was not used here
             return true;
         };
         while (ok) {
@@ -676,23 +713,24 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
             for (int b = 0; b < nblk; ++b) {
                 // a3: P = bf16(Sc ⊙ M), inclusive mask; written over the first 64 score columns
-                if (!warp_wait(&cb->sc_full, (blk_n + b) & 1, p, cb)) { ok = false; break; }
+                const uint32_t bn = blk_n + b, scb = (bn & 1) * 128;
+                if (!warp_wait(&cb->sc_full[bn & 1], (bn >> 1) & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
                 {
                     uint32_t x[BLK];
-                    tmem_ld_cols<BLK>(trow + TM_SC, x);
+                    tmem_ld_cols<BLK>(trow + TM_SC + scb, x);
                     // packed in place: x[w] <- (x[2w], x[2w+1]) only overwrites words already read
 #pragma unroll
                     for (int w = 0; w < BLK / 2; ++w)
                         x[w] = bf16x2_round((2 * w <= r) ? x[2 * w] : 0u, (2 * w + 1 <= r) ? x[2 * w + 1] : 0u);
 #pragma unroll
                     for (int c = 0; c < BLK / 32; ++c)
-                        tmem_st16(trow + TM_SC + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&x[c * 16]));
+                        tmem_st16(trow + TM_SC + scb + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&x[c * 16]));
                     tmem_wait_st();
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->p_full);
+                if (lane == 0) mbar_arrive(&cb->p_full[bn & 1]);
                 // a7 for the previous block, while the MMA warp works on this one
                 if (b > 0 && !store_block(blk_n + b - 1, tok0 + (b - 1) * BLK, min(BLK, tok1 - tok0 - (b - 1) * BLK), h)) {
                     ok = false;
@@ -703,6 +741,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 ok = false;
             blk_n += nblk;
         }
+        if (r == 0) bulk_wait_all();  // output tiles in flight complete before exit
     } else {
         // ===== warps 6-9: segment hand-off (phase L), state snapshots, final state =====
         const int q4 = warp & 3;
@@ -726,7 +765,6 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
             const bool lo = (item[IT_FLAGS] & ITF_LO) != 0;
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
-            const uint32_t ob0 = blk_n & 1;
             bool ok = true;
 
             // ---------------- phase L: prefix of this segment ----------------
@@ -785,7 +823,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
                 if (!last) {  // INCL_j = E_j + A_j  (A_j sits in an O buffer)
                     uint32_t a[64];
-                    tmem_ld_cols<64>(trow + TM_O0 + ob0 * 128 + hf * 64, a);
+                    tmem_ld_cols<64>(trow + TM_O + hf * 64, a);
 #pragma unroll
                     for (int q = 0; q < 16; ++q) {
                         float4 x;
