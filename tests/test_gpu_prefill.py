@@ -211,3 +211,21 @@ def test_long_sequence_uses_split_state_and_stays_accurate(oracle_mod):
     for lo, hi in ((0, 65536), (65536, N)):   # both precision regimes
         check_out(got[lo:hi], ref[lo:hi], bf16_out=False, what=f"tokens [{lo}, {hi})")
     check_state(to_np(st[0]), rst[0])
+
+
+def test_empty_problems():
+    """B = 0 and N = 0 launch nothing or only carry the state; an all-empty
+    packed batch returns every carried-in state unchanged."""
+    z = torch.empty((0, 16, 2, D), dtype=torch.bfloat16, device="cuda")
+    out, st = la.prefill(z, z, z, want_state=False)
+    assert out.shape == (0, 16, 2, D)
+    z2 = torch.empty((3, 0, 2, D), dtype=torch.bfloat16, device="cuda")
+    sin = torch.randn((3, 2, D, D), device="cuda")
+    out, st = la.prefill(z2, z2, z2, state_in=sin)
+    assert torch.equal(st, sin)
+    zt = torch.empty((0, 2, D), dtype=torch.bfloat16, device="cuda")
+    cu = torch.zeros(4, dtype=torch.int32, device="cuda")
+    sin3 = torch.randn((3, 2, D, D), device="cuda")
+    out, st = la.prefill_varlen(zt, zt, zt, cu, 0, state_in=sin3)
+    assert torch.equal(st, sin3)
+    assert la.get_device_status() == la.LA_OK
