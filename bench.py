@@ -173,10 +173,8 @@ def barrier(world):
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from linear_attention_blocked_b200.replicas import max_over_ranks as _max
+    return _max(x)
 
 
 # --------------------------------------------------------------------------- oracle arms
@@ -212,8 +210,8 @@ def run_reference(args, world, rank):
     threads = oracle.max_threads()
     q, k, v = la_inputs.qkv((N, H, D), SEED)
     Q, K, V = la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v)
-    # each step: a bounded sample (tokens x 1 head) sized so the whole run takes ~60 s
-    per_step_s = max(0.02, 60.0 / max(1, args.steps + args.warmup))
+    # each step: a bounded sample (tokens x heads) sized so the whole run takes ~--ref-seconds
+    per_step_s = max(0.005, args.ref_seconds / max(1, args.steps + args.warmup))
     probe_tok = 1024
     t = time.perf_counter()
     oracle.recurrent(Q[:probe_tok], K[:probe_tok], V[:probe_tok], np.array([0, probe_tok], np.int32), heads=[0],
@@ -247,7 +245,7 @@ def workload_config(ngpu):
     return {"workload": "lightning-attn causal prefill B=1 H=64 N=32768 d=128 bf16 in/out + fp32 final state",
             "B": B, "N": N, "H": H, "d": D, "block": BLOCK, "global_batch": B * ngpu, "seq_len": N,
             "parallelism": f"replicas x{ngpu} (independent batches, no collective)",
-            "l2": "inputs larger than L2 (805 MB of q/k/v read per step), no flush",
+            "l2": "inputs larger than L2 (1.61 GB of q/k/v read per step), no flush",
             "seed": SEED}
 
 
@@ -408,6 +406,8 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="CPU time budget of the oracle baseline sample (rank 0, N=1)")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="approximate total CPU time of the --impl reference run")
     args = ap.parse_args()
     if args.impl == "reference":
         # the oracle runs on the host cores of rank 0 only; no process group needed
