@@ -78,9 +78,15 @@ def load_peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "la_prefill_kernel": ("la_prefill.cuh", "la_ptx.cuh", "la_lib.cu"),
+    "la_decode_kernel": ("la_decode.cuh", "la_lib.cu"),
+}
+
+
+def kernel_source_hash(kernel: str = "la_prefill_kernel") -> str:
     h = hashlib.sha256()
-    for name in ("la_prefill.cuh", "la_ptx.cuh", "la_lib.cu"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "linear_attention_blocked_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -94,7 +100,7 @@ def recorded_traffic(kernel: str, workload: str):
         with open(path) as f:
             rec = json.load(f)
         e = rec[kernel][workload]
-        if e.get("source_hash") == kernel_source_hash():
+        if e.get("source_hash") == kernel_source_hash(kernel):
             return float(e["bytes_per_launch"])
     except Exception:
         pass
@@ -395,6 +401,7 @@ def bench_decode(la, dev, stream, args, hbm_peak, world):
             "tok_s": DEC_SEQS * world / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": gbs / hbm_peak, "kernel": "la_decode_kernel",
+                         "traffic": recorded_traffic("la_decode_kernel", "decode_S256_H64"),
                          "bytes_per_launch": decode_bytes(pairs)}}
 
 
