@@ -187,15 +187,10 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     ++g_launches;
     if (T == 0) return LA_OK;
 
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv;
     if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
         !encode_qkv_map(&mv, v, (int)T, H))
         return LA_ERR_CUDA;
-    if (out_dtype == LA_BF16) {  // bf16 output tiles leave through TMA stores with the same geometry
-        if (!encode_qkv_map(&mo, out, (int)T, H)) return LA_ERR_CUDA;
-    } else {
-        mo = mq;  // unused: fp32 outputs are written with plain stores
-    }
 
     la::PrefillParams pp;
     pp.state_in = state_in;
@@ -221,7 +216,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     if (attr_err != cudaSuccess) return LA_ERR_CUDA;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, mo, pp);
+    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;
@@ -453,15 +448,10 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     ++g_launches;
     if (T == 0) return LA_OK;
 
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv;
     if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
         !encode_qkv_map(&mv, v, (int)T, H))
         return LA_ERR_CUDA;
-    if (out_dtype == LA_BF16) {  // bf16 output tiles leave through TMA stores with the same geometry
-        if (!encode_qkv_map(&mo, out, (int)T, H)) return LA_ERR_CUDA;
-    } else {
-        mo = mq;  // unused: fp32 outputs are written with plain stores
-    }
     la::PrefillParams pp;
     pp.state_in = state_in;
     pp.state_out = state_out;
@@ -481,7 +471,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
         return LA_ERR_CUDA;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, mo, pp);
+    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;

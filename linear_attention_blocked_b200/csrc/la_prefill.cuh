@@ -14,22 +14,28 @@
 //   phase O (blocked scan over the segment's row blocks, starting from E_j):
 //       Sc  = Q_b K_b^T                    a2   (SS MMA, M=N=128, K=d)
 //       P   = bf16(Sc ⊙ M), inclusive mask a3   (TMEM -> regs -> TMEM)
-//       O   = Q_b S_hi + Q_b S_lo          a5   (S split in two bf16 terms, two
-//                                               64-column halves)
-//       S  += K_b^T V_b                    a6   (SS MMA, both MN-major)
+//       O   = Q_b S_{<b}                   a5   (S as one bf16 term, or as
+//                                               bf16 hi + lo for long sequences)
 //       O  += P V_b                        a4   (TS MMA, P read from TMEM)
+//       S  += K_b^T V_b                    a6   (SS MMA, both MN-major)
 //       out = O (bf16 or fp32)             a7
 //   and, for the last segment, the final state S goes to state_out.
 //
-// Warp roles (320 threads): warp 0 = TMA producer + ticket fetch, warp 1 =
-// TMEM allocator + MMA issuer (lane 0 issues), warps 2-5 = causal mask (a3)
-// and output store (a7), warps 6-9 = segment hand-off (phase L), state
-// snapshots for a5 and the final state.  A warp may only touch the 32 TMEM
-// lanes of its quarter (warp % 4), so each group of four covers all 128 rows.
+// Warp roles (448 threads):
+//   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
+//               loads Q
+//   warp 1      TMEM allocator + MMA issuer (lane 0 issues)
+//   warps 2-5   causal mask (a3)
+//   warps 6-9   output store (a7) and publication of inclusive prefixes
+//   warps 10-13 segment hand-off (phase L), state snapshots for a5, final state
+// A warp may only touch the 32 TMEM lanes of its quarter (warp % 4), so each
+// group of four covers all 128 rows.  Every group has its own chain of TMEM
+// loads and barrier arrivals, so the mask of block b+1, the output of block b
+// and the state snapshot for block b+1 proceed independently.
 //
 // Shared memory (1024-byte aligned, 128-byte swizzle everywhere):
-//   K ring 2 x 32 KiB | V ring 2 x 32 KiB | Q ring 2 x 32 KiB | S_hi half 16 KiB |
-//   S_lo half 16 KiB | barriers + item queue.
+//   K ring 2 x 32 KiB | V ring 2 x 32 KiB | Q ring 2 x 32 KiB | S snapshot
+//   2 x 16 KiB | barriers + item queue.
 // A [128 x 128] bf16 tile is two 16 KiB halves (columns 0-63, 64-127), each
 // 128 rows of 128 bytes, written by one TMA box {64, 1, 128, 2} of the 4-D
 // view {64, H, T, 2} of the [T, H, 128] tensor (the halves are its outer
@@ -50,30 +56,25 @@ constexpr int BLK = 128;                    // rows per block (= MMA M)
 constexpr int HALF_BYTES = BLK * 128;       // [128 rows x 64 bf16]
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // [128 x 128] bf16
 constexpr int KV_STAGES = 2;
-constexpr int PREFILL_THREADS = 320;
-// L2 prefetch distances, in row blocks, ahead of the shared-memory loads.
-// Shared memory holds about one block ahead; in phase O the only DRAM reads
-// are the Q tiles (K and V come back from L2), so Q is prefetched further
-// ahead to keep enough DRAM reads in flight per SM.  Phase A already keeps
-// two 64 KiB K/V stages in flight and gets no K/V prefetch by default.
+constexpr int Q_STAGES = 2;
+constexpr int PREFILL_THREADS = 448;
+constexpr int W_MASK = 2, W_STORE = 6, W_STATE = 10;  // first warp of each four-warp group
+
+// L2 prefetch distance of the Q tiles, in row blocks ahead of their
+// shared-memory loads (0 = off).  K and V of phase O come back from L2 after
+// phase A; Q is read from DRAM once, and its shared-memory slot only frees up
+// when a5 of the block two earlier has finished, so the prefetch hides part
+// of the DRAM latency of that load.
 #ifndef LA_PREFETCH_Q
 #define LA_PREFETCH_Q 0
 #endif
-#ifndef LA_PREFETCH_KV
-#define LA_PREFETCH_KV 0
-#endif
 constexpr int PF_Q = LA_PREFETCH_Q;
-#ifndef LA_PHASE_A_Q_PREFETCH
-#define LA_PHASE_A_Q_PREFETCH 0
-#endif
-constexpr int PF_KV = LA_PREFETCH_KV;
 
 constexpr int SM_K = 0;
 constexpr int SM_V = SM_K + KV_STAGES * TILE_BYTES;
-constexpr int Q_STAGES = 2;
 constexpr int SM_Q = SM_V + KV_STAGES * TILE_BYTES;
-constexpr int SM_SHI = SM_Q + Q_STAGES * TILE_BYTES;  // one 64-column half of S as bf16 hi
-constexpr int SM_SLO = SM_SHI + HALF_BYTES;           // ... and its bf16 lo residual
+constexpr int SM_SHI = SM_Q + Q_STAGES * TILE_BYTES;  // S snapshot: bf16 hi of one half, or columns 0-63
+constexpr int SM_SLO = SM_SHI + HALF_BYTES;           // ... bf16 lo residual of that half, or columns 64-127
 constexpr int SM_CTRL = SM_SLO + HALF_BYTES;          // 229376
 constexpr int SM_CTRL_BYTES = 1024;
 constexpr int PREFILL_SMEM = SM_CTRL + SM_CTRL_BYTES + 1024;  // + alignment slack
@@ -108,13 +109,26 @@ struct PrefillParams {
     int *status;            // sticky device status word
 };
 
+// mbarriers (arrival counts in brackets)
 struct CtrlBlock {
-    uint64_t kv_full[KV_STAGES], kv_empty[KV_STAGES];
-    uint64_t q_full[Q_STAGES], q_empty[Q_STAGES];
-    uint64_t sc_full[2], p_full[2], o_full, o_empty;
-    uint64_t s_done, snap_full, snap_empty, agg_full;
-    uint64_t item_full[2], item_empty[2];
-    uint64_t fin, pub, ostage;
+    uint64_t kv_full[KV_STAGES];  // [1] producer expect_tx
+    uint64_t kv_empty[KV_STAGES]; // [1] MMA commit after the last MMA reading the stage
+    uint64_t q_full[Q_STAGES];    // [1] producer expect_tx
+    uint64_t q_empty[Q_STAGES];   // [1] MMA commit after a5 of the block
+    uint64_t sc_full[2];          // [1] a2 done: scores in buffer b & 1
+    uint64_t p_full[2];           // [4] mask warps: P in buffer b & 1
+    uint64_t o_full;              // [1] a4 + a5 done
+    uint64_t o_empty;             // [4] store warps have O in registers
+    uint64_t s_done;              // [1] a6 done
+    uint64_t snap_full;           // [4] state warps: snapshot of S in shared memory (S read)
+    uint64_t snap_empty;          // [1] a5 has read the snapshot
+    uint64_t agg_full;            // [1] phase A done: A_j in the O columns
+    uint64_t incl_ready;          // [4] state warps: INCL_j written over A_j in the O columns
+    uint64_t a_free;              // [4] store warps: INCL_j read, the O columns are free
+    uint64_t pub;                 // [4] store warps: INCL_j stores ordered before the flag
+    uint64_t item_full[2];        // [1] producer
+    uint64_t item_empty[2];       // [14] Q producer lane + MMA lane 0 + 3 x 4 warps
+    uint64_t fin;                 // [1] tear-down: every MMA done
     int item[2][8];
     uint32_t tmem_base;
     volatile int abort;
@@ -209,22 +223,32 @@ __device__ __forceinline__ void split_hi_lo(uint32_t u0, uint32_t u1, uint32_t &
     lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
 }
 
+// Load 32 consecutive TMEM columns of this warp's lanes and wait for them.
+__device__ __forceinline__ void tmem_ld_wait32(uint32_t taddr, uint32_t (&x)[32]) {
+    tmem_ld32(taddr, x);
+    tmem_wait_ld();
+    reg_fence(x);
+}
+
 // Read S from TMEM and hand it to a5 through the snapshot buffer: either the
-// whole state as bf16 (one arrival), or, when `lo`, as bf16 hi + lo one
-// 64-column half at a time (two arrivals).  The first arrival on snap_full
-// also tells the MMA warp that S has been read, so a6 may overwrite it.
+// whole state as bf16 (one arrival; columns 0-63 in `shi`, 64-127 in `slo`),
+// or, when `lo`, as bf16 hi + lo one 64-column half at a time (two arrivals).
+// The last arrival also tells the MMA warp that S has been read, so a6 may
+// overwrite it.
 __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint8_t *slo, int r, int lane, bool lo,
-                                               uint32_t &snap_n, const PrefillParams &p, CtrlBlock *cb) {
-    uint32_t x[D];
-    tmem_ld_cols<D>(trow + TM_S, x);
+                                            uint32_t &snap_n, const PrefillParams &p, CtrlBlock *cb) {
     if (!lo) {
-        if (!warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) return false;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {  // columns [64 hf, 64 hf + 64) -> shi (hf = 0) or slo (hf = 1)
+            uint32_t x[64];
+            tmem_ld_cols<64>(trow + TM_S + hf * 64, x);
+            if (hf == 0 && !warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) return false;
+            uint8_t *half = hf ? slo : shi;
 #pragma unroll
-        for (int q = 0; q < D / 8; ++q) {  // 16-byte chunks of 8 columns, two 64-column halves
-            const uint32_t off = (uint32_t)((q >> 3) * HALF_BYTES + r * 128 + (((q & 7) ^ (r & 7)) << 4));
-            *reinterpret_cast<uint4 *>(shi + off) =
-                make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
-                           bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7]));
+            for (int q = 0; q < 8; ++q)  // 16-byte chunks of 8 columns
+                *reinterpret_cast<uint4 *>(half + r * 128 + ((q ^ (r & 7)) << 4)) =
+                    make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
+                               bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7]));
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -233,18 +257,24 @@ __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint
         ++snap_n;
         return true;
     }
-#pragma unroll
+    // hi + lo, one 64-column half per arrival; a6 is issued only after a5 has
+    // used both halves, so S may be read half by half
+#pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
-        if (!warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) return false;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {  // 16-byte chunks of 8 columns
-            uint32_t hv[4], lv[4];
+        for (int qq = 0; qq < 2; ++qq) {
+            uint32_t x[32];
+            tmem_ld_wait32(trow + TM_S + hf * 64 + qq * 32, x);
+            if (qq == 0 && !warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) return false;
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-                split_hi_lo(x[hf * 64 + 8 * q + 2 * w], x[hf * 64 + 8 * q + 2 * w + 1], hv[w], lv[w]);
-            const uint32_t off = (uint32_t)(r * 128 + ((q ^ (r & 7)) << 4));
-            *reinterpret_cast<uint4 *>(shi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-            *reinterpret_cast<uint4 *>(slo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t hv[4], lv[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) split_hi_lo(x[8 * c + 2 * w], x[8 * c + 2 * w + 1], hv[w], lv[w]);
+                const uint32_t off = (uint32_t)(r * 128 + (((qq * 4 + c) ^ (r & 7)) << 4));
+                *reinterpret_cast<uint4 *>(shi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+                *reinterpret_cast<uint4 *>(slo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -255,10 +285,22 @@ __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint
     return true;
 }
 
+// Every role reads the same item from the two-slot queue the producer fills.
+__device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane, const PrefillParams &p,
+                                          CtrlBlock *cb) {
+    const int islot = it & 1;
+    if (!warp_wait(&cb->item_full[islot], (it >> 1) & 1, p, cb)) return false;
+#pragma unroll
+    for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&cb->item_empty[islot]);
+    ++it;
+    return item[IT_VALID] != 0;
+}
+
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmo,
-                  const __grid_constant__ PrefillParams p) {
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -275,27 +317,27 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             mbar_init(&cb->q_full[s], 1);
             mbar_init(&cb->q_empty[s], 1);
         }
-        mbar_init(&cb->o_full, 1);
-        mbar_init(&cb->o_empty, 4);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&cb->sc_full[s], 1);
             mbar_init(&cb->p_full[s], 4);
             mbar_init(&cb->item_full[s], 1);
-            mbar_init(&cb->item_empty[s], 9);
+            mbar_init(&cb->item_empty[s], 14);
         }
+        mbar_init(&cb->o_full, 1);
+        mbar_init(&cb->o_empty, 4);
         mbar_init(&cb->s_done, 1);
         mbar_init(&cb->snap_full, 4);
         mbar_init(&cb->snap_empty, 1);
         mbar_init(&cb->agg_full, 1);
-        mbar_init(&cb->fin, 1);
+        mbar_init(&cb->incl_ready, 4);
+        mbar_init(&cb->a_free, 4);
         mbar_init(&cb->pub, 4);
-        mbar_init(&cb->ostage, 4);
+        mbar_init(&cb->fin, 1);
         cb->abort = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
-        if (!p.out_fp32) tma_prefetch_desc(&tmo);
     }
     if (warp == 1) {
         tmem_alloc(&cb->tmem_base, TM_COLS);
@@ -308,14 +350,15 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     const int H = p.H;
 
     if (warp == 0) {
-        // ===================== producer: tickets + TMA =====================
+        // ===================== producers =====================
+        // lane 0: tickets, K and V tiles (phase A and phase O)
+        // lane 1: Q tiles of phase O, which may run ahead of K and V (for
+        //         instance into the previous item's phase A)
         if (lane == 0) {
             const uint64_t pol_first = policy_evict_first();
             const uint64_t pol_last = policy_evict_last();
-            const uint64_t pol_norm = policy_evict_normal();
-            uint32_t it = 0, kv_n = 0, q_n = 0;
+            uint32_t it = 0, kv_n = 0;
             int kv_last_fill[KV_STAGES] = {-1, -1};
-            int q_last_fill[Q_STAGES] = {-1, -1};
             const int total = *reinterpret_cast<volatile int *>(&p.hdr[HDR_TOTAL]);
             bool ok = true;
             for (;;) {
@@ -345,60 +388,20 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 const int tok0 = seg.y, tok1 = seg.z;
                 const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
                 const bool last = (seg.w & SEG_LAST) != 0;
-                // L2 prefetch of whole [128 x 128] tiles (two 64-column boxes each)
-                auto prefetch_tile = [&](const CUtensorMap *m, int b, uint64_t pol) {
-                    if (b < nblk) tma_prefetch_4d(m, 0, h, tok0 + b * BLK, 0, pol);
-                };
-                for (int b = 0; b < PF_KV; ++b) {
-                    prefetch_tile(&tmk, b, pol_last);
-                    prefetch_tile(&tmv, b, pol_last);
-                }
-                if (last)  // no phase A: the scan starts at once
-                    for (int b = 0; b < PF_Q; ++b) prefetch_tile(&tmq, b, pol_last);
-                if (!last) {  // phase A: K and V only; kept in L2 for phase O
-                    for (int b = 0; b < nblk && ok; ++b) {
+                // phase A (K and V, kept in L2 for phase O), then phase O
+                for (int pass = last ? 1 : 0; pass < 2 && ok; ++pass) {
+                    const uint64_t pol = pass == 0 ? pol_last : pol_first;
+                    for (int b = 0; b < nblk; ++b) {
                         if (cb->abort) { ok = false; break; }
                         const int s = kv_n % KV_STAGES;
                         if (!wait_or_abort(&cb->kv_empty[s], ((kv_n / KV_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
-                        if (PF_KV > 0) {
-                            prefetch_tile(&tmk, b + PF_KV, pol_last);
-                            prefetch_tile(&tmv, b + PF_KV, pol_last);
-                        }
-#if LA_PHASE_A_Q_PREFETCH
-                        prefetch_tile(&tmq, b, pol_last);  // phase O then finds Q in L2 as well as K and V
-#else
-                        if (b >= nblk - PF_Q) prefetch_tile(&tmq, b - (nblk - PF_Q), pol_last);  // phase O's first Q tiles
-#endif
                         mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
                         const int row = tok0 + b * BLK;
-                        uint8_t *kt = smem + SM_K + s * TILE_BYTES;
-                        uint8_t *vt = smem + SM_V + s * TILE_BYTES;
-                        tma_load_4d(kt, &tmk, &cb->kv_full[s], 0, h, row, 0, pol_last);
-                        tma_load_4d(vt, &tmv, &cb->kv_full[s], 0, h, row, 0, pol_last);
+                        tma_load_4d(smem + SM_K + s * TILE_BYTES, &tmk, &cb->kv_full[s], 0, h, row, 0, pol);
+                        tma_load_4d(smem + SM_V + s * TILE_BYTES, &tmv, &cb->kv_full[s], 0, h, row, 0, pol);
                         kv_last_fill[s] = kv_n / KV_STAGES;
                         ++kv_n;
                     }
-                }
-                for (int b = 0; b < nblk && ok; ++b) {  // phase O: Q, K, V
-                    if (cb->abort) { ok = false; break; }
-                    const int row = tok0 + b * BLK;
-                    if (PF_Q > 0) prefetch_tile(&tmq, b + PF_Q, pol_last);
-                    const int s = kv_n % KV_STAGES;
-                    if (!wait_or_abort(&cb->kv_empty[s], ((kv_n / KV_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
-                    mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
-                    uint8_t *kt = smem + SM_K + s * TILE_BYTES;
-                    uint8_t *vt = smem + SM_V + s * TILE_BYTES;
-                    tma_load_4d(kt, &tmk, &cb->kv_full[s], 0, h, row, 0, pol_first);
-                    tma_load_4d(vt, &tmv, &cb->kv_full[s], 0, h, row, 0, pol_first);
-                    kv_last_fill[s] = kv_n / KV_STAGES;
-                    ++kv_n;
-                    const int qs = q_n % Q_STAGES;
-                    if (!wait_or_abort(&cb->q_empty[qs], ((q_n / Q_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
-                    mbar_expect_tx(&cb->q_full[qs], TILE_BYTES);
-                    uint8_t *qt = smem + SM_Q + qs * TILE_BYTES;
-                    tma_load_4d(qt, &tmq, &cb->q_full[qs], 0, h, row, 0, pol_first);
-                    q_last_fill[qs] = q_n / Q_STAGES;
-                    ++q_n;
                 }
                 if (!ok) break;
             }
@@ -409,6 +412,36 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     int dummy = 0;
                     la_wait(&cb->kv_full[s], kv_last_fill[s] & 1, dl, &dummy);
                 }
+            if (!ok) cb->abort = 1;
+        } else if (lane == 1) {
+            const uint64_t pol_first = policy_evict_first();
+            const uint64_t pol_last = policy_evict_last();
+            uint32_t it = 0, q_n = 0;
+            int q_last_fill[Q_STAGES] = {-1, -1};
+            bool ok = true;
+            for (;;) {
+                const int islot = it & 1;
+                if (!wait_or_abort(&cb->item_full[islot], (it >> 1) & 1, p, cb)) { ok = false; break; }
+                int item[8];
+#pragma unroll
+                for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
+                mbar_arrive(&cb->item_empty[islot]);
+                ++it;
+                if (!item[IT_VALID]) break;
+                const int h = item[IT_H], tok0 = item[IT_TOK0];
+                const int nblk = (item[IT_TOK1] - tok0 + BLK - 1) / BLK;
+                for (int b = 0; b < nblk; ++b) {
+                    if (cb->abort) { ok = false; break; }
+                    if (PF_Q > 0 && b + PF_Q < nblk) tma_prefetch_4d(&tmq, 0, h, tok0 + (b + PF_Q) * BLK, 0, pol_last);
+                    const int qs = q_n % Q_STAGES;
+                    if (!wait_or_abort(&cb->q_empty[qs], ((q_n / Q_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
+                    mbar_expect_tx(&cb->q_full[qs], TILE_BYTES);
+                    tma_load_4d(smem + SM_Q + qs * TILE_BYTES, &tmq, &cb->q_full[qs], 0, h, tok0 + b * BLK, 0, pol_first);
+                    q_last_fill[qs] = q_n / Q_STAGES;
+                    ++q_n;
+                }
+                if (!ok) break;
+            }
             for (int s = 0; s < Q_STAGES; ++s)
                 if (q_last_fill[s] >= 0) {
                     const uint64_t dl = globaltimer_ns() + p.wait_limit_ns;
@@ -419,30 +452,33 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         }
     } else if (warp == 1) {
         // ===================== MMA issuer =====================
-        // Phase O runs two dependency chains per block b:
-        //   intra chain:  a2(b) -> [mask] -> a4(b)            (needs Q, K, V tiles)
-        //   state chain:  a5 half 0 (S_{<b}) -> a6(b) -> a5 half 1
-        // a4(b) initialises the block's O buffer, the a5 halves accumulate onto it.
+        // Phase O runs three dependency chains per block b:
+        //   intra chain:  a2(b) -> [mask] -> a4(b)              (needs Q, K, V tiles)
+        //   O chain:      a5(b) -> a4(b) -> [O read out] -> a5(b+1)
+        //   state chain:  [snapshot S_{<b}] -> a5(b), a6(b) -> [snapshot S_{<b+1}]
+        // a5(b) initialises the block's O buffer and a4(b) accumulates onto it,
+        // so every accumulator receives its MMAs in a fixed order and the result
+        // is deterministic.  a5 comes first so that the Q tile is released as
+        // soon as possible (a2 and a5 are its only readers) and so that a6, the
+        // state update, follows the snapshot without waiting for the mask.
         // Instead of a fixed program order, the issuing lane polls the barriers
-        // and issues whatever is ready, so the intra chain can run up to two
-        // blocks (the two O buffers) ahead of the state chain.
+        // and issues whatever is ready: a2 may run up to two blocks (the two
+        // score buffers) ahead of a4.
         constexpr uint32_t ID_QK = idesc_bf16_f32(BLK, BLK, 0, 0);    // Q (K-major) x K (K-major)
         constexpr uint32_t ID_QS = idesc_bf16_f32(BLK, D / 2, 0, 1);  // Q (K-major) x S half (MN-major)
         constexpr uint32_t ID_QF = idesc_bf16_f32(BLK, D, 0, 1);      // Q (K-major) x S (MN-major)
         constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1);        // K^T (MN) x V (MN)
         constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1);      // P (TMEM) x V (MN)
-        uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0;
+        // The whole warp runs this loop in step: every lane holds the same
+        // counters, barrier probes are combined with __all_sync, and each MMA or
+        // commit is issued by the lane that elect.sync picks.
+        uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0, afree_n = 0;
         bool ok = true;
-        while (ok) {
-            const int islot = it & 1;
-            if (!warp_wait(&cb->item_full[islot], (it >> 1) & 1, p, cb)) break;
-            int item[8];
-#pragma unroll
-            for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&cb->item_empty[islot]);
-            ++it;
-            if (!item[IT_VALID]) break;
+        int item[8];
+        auto ready = [&](uint64_t *bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_test(bar, parity)) != 0;
+        };
+        while (ok && next_item(it, item, lane, p, cb)) {
             const int tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
             const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
@@ -457,142 +493,123 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const int s = kv_n % KV_STAGES;
                     if (!warp_wait(&cb->kv_full[s], (kv_n / KV_STAGES) & 1, p, cb)) { ok = false; break; }
                     tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
-                        const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
+                    const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
+                    const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < BLK / 16; ++kk)
-                            mma_ss(tmem + TM_O, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
-                                   (b > 0 || kk > 0) ? 1u : 0u);
-                        tc_commit(&cb->kv_empty[s]);
-                    }
-                    __syncwarp();
+                    for (int kk = 0; kk < BLK / 16; ++kk)
+                        mma_ss_w(tmem + TM_O, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, (b > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit_w(&cb->kv_empty[s]);
                     ++kv_n;
                 }
                 if (!ok) break;
-                if (lane == 0) tc_commit(&cb->agg_full);
-                __syncwarp();
+                tc_commit_w(&cb->agg_full);
             }
-            // ---------------- phase O: polled two-chain schedule ----------------
+            // ---------------- phase O: polled three-chain schedule ----------------
             const bool want_final = last && p.state_out != nullptr;
             const uint32_t kv0 = kv_n, q0 = q_n, blk0 = blk_n;
             int i2 = 0, i4 = 0, i5 = 0, half = 0;  // next block of a2 / a4 / a5; a5 half pending
             uint32_t spins = 0;
             uint64_t deadline = 0;
-            while (i5 < nblk) {
-                int prog = 0;
-                if (lane == 0) {
-                    // intra chain, a4(i4): P ready and the O buffer free
-                    if (i4 < i2) {
-                        const uint32_t bn = blk0 + i4;
-                        // a4 of the first block overwrites the O columns that hold A_j:
-                        // it must wait until phase L has read A_j (first E snapshot out)
-                        const bool a_read = last || i4 > 0 || mbar_test(&cb->snap_full, snap_n & 1);
-                        if (a_read && mbar_test(&cb->p_full[bn & 1], (bn >> 1) & 1) &&
-                            mbar_test(&cb->o_empty, (bn & 1) ^ 1)) {
-                            tc_fence_after();
-                            const int s = (kv0 + i4) % KV_STAGES;
-                            const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
-#pragma unroll
-                            for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns
-                                mma_ts(tmem + TM_O, tmem + TM_SC + (bn & 1) * 128 + kk * 8, desc_mnmajor(vt, kk), ID_PV,
-                                       kk > 0 ? 1u : 0u);
-                            ++i4;
-                            prog = 1;
-                        }
-                    }
-                    // intra chain, a2(i2): its score buffer free (a4 of block i2 - 2
-                    // issued), tiles landed
-                    if (i2 < nblk && i2 < i4 + 2) {
-                        const int s = (kv0 + i2) % KV_STAGES;
-                        const uint32_t kn = (kv0 + i2) / KV_STAGES, qn = q0 + i2;
-                        if (mbar_test(&cb->kv_full[s], kn & 1) &&
-                            mbar_test(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1))
-                            prog = 2;  // a2 is issued below, after the warp zeroes ragged rows
-                    }
-                    // state chain: a5 (one full-width pass, or half 0 (+ a6) then half 1)
-                    if (prog != 2 && i5 < i4 && mbar_test(&cb->snap_full, snap_n & 1)) {
+            while (i4 < nblk) {
+                bool prog = false;
+                // O chain, a4(i4): P ready, a5 of the block issued
+                if (i4 < i5) {
+                    const uint32_t bn = blk0 + i4;
+                    if (ready(&cb->p_full[bn & 1], (bn >> 1) & 1)) {
                         tc_fence_after();
-                        const uint32_t bn = blk0 + i5;
+                        const int s = (kv0 + i4) % KV_STAGES;
+                        const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns
+                            mma_ts_w(tmem + TM_O, tmem + TM_SC + (bn & 1) * 128 + kk * 8, desc_mnmajor(vt, kk), ID_PV, 1u);
+                        tc_commit_w(&cb->o_full);
+                        tc_commit_w(&cb->kv_empty[s]);  // a2, a6 and a4 of this block are issued
+                        ++i4;
+                        prog = true;
+                    }
+                }
+                // state and O chains, a5(i5) (one full-width pass, or one half of
+                // the hi + lo pair) then a6(i5): Q landed (a2 issued), snapshot
+                // ready, the O buffer free (the previous block's O read out; for
+                // the first block of a segment with a successor, INCL read out of
+                // the O columns)
+                if (i5 < i2) {
+                    const uint32_t bn = blk0 + i5;
+                    const bool a_read = last || i5 > 0 || ready(&cb->a_free, afree_n & 1);
+                    if (a_read && ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty, (bn & 1) ^ 1)) {
+                        tc_fence_after();
                         const int s = (kv0 + i5) % KV_STAGES;
                         const uint32_t qn = q0 + i5;
                         const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
                         const uint32_t sh = sbase + SM_SHI, sl = sbase + SM_SLO;
                         const bool upd = (i5 < nblk - 1) || want_final;
-                        if (!lo) {  // O += Q S_hi, S_hi = the whole [128 x 128] snapshot buffer
+                        bool block_done = true;
+                        if (!lo) {  // O = Q S, S = the whole [128 x 128] snapshot
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(tmem + TM_O, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, 1u);
-                            tc_commit(&cb->snap_empty);
-                            ++snap_n;
-                        } else {
+                                mma_ss_w(tmem + TM_O, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, kk > 0 ? 1u : 0u);
+                        } else {  // one 64-column half of O = Q (S_hi + S_lo)
                             const uint32_t to = tmem + TM_O + half * 64;
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, 1u);
+                                mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u);
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
-                            tc_commit(&cb->snap_empty);
-                            ++snap_n;
+                                mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
+                            block_done = half == 1;
+                            half ^= 1;
                         }
-                        if (!lo || half == 0) {
+                        tc_commit_w(&cb->snap_empty);
+                        ++snap_n;
+                        if (!last && i5 == 0 && block_done) ++afree_n;
+                        if (block_done) {
+                            tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // a2 and a5 have read the Q tile
                             if (upd) {  // a6: S += K^T V (S_{<b} has been read out)
                                 const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
                                 const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                                 for (int kk = 0; kk < BLK / 16; ++kk)
-                                    mma_ss(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
-                                tc_commit(&cb->s_done);
+                                    mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                                tc_commit_w(&cb->s_done);
                             }
-                            tc_commit(&cb->kv_empty[s]);  // a2, a4 and a6 of this block are issued
-                        }
-                        if (lo && half == 0) {
-                            half = 1;
-                        } else {
-                            tc_commit(&cb->o_full);  // also: Q of this block is no longer read
-                            half = 0;
                             ++i5;
                         }
-                        prog = 1;
+                        prog = true;
                     }
                 }
-                prog = __shfl_sync(0xffffffffu, prog, 0);
-                if (prog == 2) {
+                // intra chain, a2(i2): its score buffer free (a4 of block i2 - 2
+                // issued), tiles landed
+                if (i2 < nblk && i2 < i4 + 2) {
                     const int s = (kv0 + i2) % KV_STAGES;
-                    const int valid = min(BLK, tok1 - (tok0 + i2 * BLK));
-                    if (valid < BLK) {
-                        // rows past the end of the sequence must add nothing to S or O:
-                        // zero them in K and V (they may hold the next sequence's tokens)
-                        uint8_t *kp = smem + SM_K + s * TILE_BYTES;
-                        uint8_t *vp = smem + SM_V + s * TILE_BYTES;
-                        const int nbytes = (BLK - valid) * 128;
-                        for (int hh = 0; hh < 2; ++hh)
-                            for (int o = lane * 16; o < nbytes; o += 32 * 16) {
-                                *reinterpret_cast<uint4 *>(kp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
-                                *reinterpret_cast<uint4 *>(vp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
-                            }
-                        fence_proxy_async_smem();
-                    }
-                    __syncwarp();
-                    if (lane == 0) {  // a2: Sc = Q K^T
+                    const uint32_t kn = (kv0 + i2) / KV_STAGES, qn = q0 + i2;
+                    if (ready(&cb->kv_full[s], kn & 1) && ready(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1)) {
+                        const int valid = min(BLK, tok1 - (tok0 + i2 * BLK));
+                        if (valid < BLK) {
+                            // rows past the end of the sequence must add nothing to S or O:
+                            // zero them in K and V (they may hold the next sequence's tokens)
+                            uint8_t *kp = smem + SM_K + s * TILE_BYTES;
+                            uint8_t *vp = smem + SM_V + s * TILE_BYTES;
+                            const int nbytes = (BLK - valid) * 128;
+                            for (int hh = 0; hh < 2; ++hh)
+                                for (int o = lane * 16; o < nbytes; o += 32 * 16) {
+                                    *reinterpret_cast<uint4 *>(kp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                                    *reinterpret_cast<uint4 *>(vp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                                }
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                        }
                         tc_fence_after();
-                        const uint32_t qn = q0 + i2;
                         const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
                         const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            mma_ss(tmem + TM_SC + ((blk0 + i2) & 1) * 128, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
-                                   kk > 0 ? 1u : 0u);
-                        tc_commit(&cb->sc_full[(blk0 + i2) & 1]);
+                        for (int kk = 0; kk < D / 16; ++kk)  // a2: Sc = Q K^T
+                            mma_ss_w(tmem + TM_SC + ((blk0 + i2) & 1) * 128, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
+                                     kk > 0 ? 1u : 0u);
+                        tc_commit_w(&cb->sc_full[(blk0 + i2) & 1]);
+                        ++i2;
+                        prog = true;
                     }
-                    ++i2;
                 }
-                i2 = __shfl_sync(0xffffffffu, i2, 0);
-                i4 = __shfl_sync(0xffffffffu, i4, 0);
-                i5 = __shfl_sync(0xffffffffu, i5, 0);
-                half = __shfl_sync(0xffffffffu, half, 0);
-                snap_n = __shfl_sync(0xffffffffu, snap_n, 0);
                 if (prog) {
                     spins = 0;
                     deadline = 0;
@@ -618,148 +635,150 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             blk_n = blk0 + nblk;
         }
         // Tear-down: all MMAs issued by this thread must finish before TMEM is freed.
+        __syncwarp();
+        tc_commit_w(&cb->fin);
         if (lane == 0) {
-            tc_commit(&cb->fin);
             const uint64_t dl = globaltimer_ns() + p.wait_limit_ns;
             int dummy = 0;
             la_wait(&cb->fin, 0, dl, &dummy);
         }
         __syncwarp();
-    } else if (warp < 6) {
-        // ============ warps 2-5: causal mask (a3) and output store (a7) ============
+    } else if (warp < W_STORE) {
+        // ===================== warps 2-5: causal mask (a3) =====================
         const int q4 = warp & 3;               // TMEM lane quarter this warp may access
         const int r = q4 * 32 + lane;          // tile row = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         uint32_t it = 0, blk_n = 0;
         bool ok = true;
-        uint32_t ostage_n = 0;
-        // O of block b -> out.  The O buffer is released as soon as it is in
-        // registers.  A full bf16 block is staged in the shared-memory slot of
-        // its own Q tile (o_full means every MMA that read that Q is done) and
-        // written by one TMA bulk store (full 128-byte lines); the slot goes
-        // back to the producer once the store has read it.  A ragged block
-        // (it must not write past the sequence) and fp32 outputs use direct
-        // 16-byte stores instead.
-        auto store_block = [&](uint32_t bn, int row0, int valid, int h) -> bool {
-            if (!warp_wait(&cb->o_full, bn & 1, p, cb)) return false;
-            tc_fence_after();
-            uint32_t x[D];
-            tmem_ld_cols<D>(trow + TM_O, x);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&cb->o_empty);
-            const int qslot = bn % Q_STAGES;
-            if (!p.out_fp32 && valid == BLK) {
-                uint8_t *stage = smem + SM_Q + qslot * TILE_BYTES;
-#pragma unroll
-                for (int q = 0; q < D / 8; ++q) {
-                    const uint32_t off = (uint32_t)((q >> 3) * HALF_BYTES + r * 128 + (((q & 7) ^ (r & 7)) << 4));
-                    *reinterpret_cast<uint4 *>(stage + off) =
-                        make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
-                                   bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7]));
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->ostage);
-                bool ok2 = true;
-                if (r == 0) {
-                    ok2 = wait_or_abort(&cb->ostage, ostage_n & 1, p, cb);
-                    if (ok2) {
-                        tma_store_4d(&tmo, stage, 0, h, row0, 0);
-                        bulk_commit_group();
-                        bulk_wait_read_all();
-                        mbar_arrive(&cb->q_empty[qslot]);
-                    }
-                }
-                ++ostage_n;
-                return __all_sync(0xffffffffu, ok2) != 0;
-            }
-            if (r < valid) {
-                const size_t orow = ((size_t)(row0 + r) * H + h) * D;
-                if (p.out_fp32) {
-                    float *o = reinterpret_cast<float *>(p.out) + orow;
-#pragma unroll
-                    for (int q = 0; q < D / 4; ++q)
-                        __stcs(reinterpret_cast<float4 *>(o + 4 * q),
-                               make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
-                                           __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3])));
-                } else {
-                    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out) + orow;
-#pragma unroll
-                    for (int q = 0; q < D / 8; ++q) {
-                        uint4 u;
-                        u.x = bf16x2_round(x[8 * q], x[8 * q + 1]);
-                        u.y = bf16x2_round(x[8 * q + 2], x[8 * q + 3]);
-                        u.z = bf16x2_round(x[8 * q + 4], x[8 * q + 5]);
-                        u.w = bf16x2_round(x[8 * q + 6], x[8 * q + 7]);
-                        __stcs(reinterpret_cast<uint4 *>(o + 8 * q), u);
-                    }
-                }
-            }
-            if (r == 0) mbar_arrive(&cb->q_empty[qslot]);  // the Q slot was not used here
-            return true;
-        };
-        while (ok) {
-            const int islot = it & 1;
-            if (!warp_wait(&cb->item_full[islot], (it >> 1) & 1, p, cb)) break;
-            int item[8];
-#pragma unroll
-            for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&cb->item_empty[islot]);
-            ++it;
-            if (!item[IT_VALID]) break;
-            const int h = item[IT_H], tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
-            const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
+        int item[8];
+        while (ok && next_item(it, item, lane, p, cb)) {
+            const int nblk = (item[IT_TOK1] - item[IT_TOK0] + BLK - 1) / BLK;
             for (int b = 0; b < nblk; ++b) {
-                // a3: P = bf16(Sc ⊙ M), inclusive mask; written over the first 64 score columns
-                const uint32_t bn = blk_n + b, scb = (bn & 1) * 128;
+                // P = bf16(Sc ⊙ M), inclusive mask, packed two per 32-bit column
+                // over the first 64 score columns
+                const uint32_t bn = blk_n + b, tsc = trow + TM_SC + (bn & 1) * 128;
                 if (!warp_wait(&cb->sc_full[bn & 1], (bn >> 1) & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
-                {
-                    uint32_t x[BLK];
-                    tmem_ld_cols<BLK>(trow + TM_SC + scb, x);
-                    // packed in place: x[w] <- (x[2w], x[2w+1]) only overwrites words already read
 #pragma unroll
-                    for (int w = 0; w < BLK / 2; ++w)
-                        x[w] = bf16x2_round((2 * w <= r) ? x[2 * w] : 0u, (2 * w + 1 <= r) ? x[2 * w + 1] : 0u);
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t x[64];
+                    if (hf == 1 && q4 < 2) {
+                        // rows 0-63 see none of the keys 64-127
 #pragma unroll
-                    for (int c = 0; c < BLK / 32; ++c)
-                        tmem_st16(trow + TM_SC + scb + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&x[c * 16]));
-                    tmem_wait_st();
+                        for (int w = 0; w < 32; ++w) x[w] = 0u;
+                    } else {
+                        tmem_ld_cols<64>(tsc + hf * 64, x);
+                        // in place: x[w] <- (x[2w], x[2w+1]) only overwrites words already read
+#pragma unroll
+                        for (int w = 0; w < 32; ++w) {
+                            const int c = hf * 64 + 2 * w;
+                            x[w] = bf16x2_round(c <= r ? x[2 * w] : 0u, c + 1 <= r ? x[2 * w + 1] : 0u);
+                        }
+                    }
+                    tmem_st32(tsc + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
                 }
+                tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cb->p_full[bn & 1]);
-                // a7 for the previous block, while the MMA warp works on this one
-                if (b > 0 && !store_block(blk_n + b - 1, tok0 + (b - 1) * BLK, min(BLK, tok1 - tok0 - (b - 1) * BLK), h)) {
-                    ok = false;
-                    break;
-                }
             }
-            if (ok && !store_block(blk_n + nblk - 1, tok0 + (nblk - 1) * BLK, tok1 - tok0 - (nblk - 1) * BLK, h))
-                ok = false;
             blk_n += nblk;
         }
-        if (r == 0) bulk_wait_all();  // output tiles in flight complete before exit
-    } else {
-        // ===== warps 6-9: segment hand-off (phase L), state snapshots, final state =====
+    } else if (warp < W_STATE) {
+        // ====== warps 6-9: output store (a7), publication of inclusive prefixes ======
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
-        uint32_t it = 0, blk_n = 0, snap_n = 0, upd_n = 0, agg_n = 0, pub_n = 0;
+        uint32_t it = 0, blk_n = 0, incl_n = 0, pub_n = 0;
+        bool ok = true;
+        int item[8];
+        while (ok && next_item(it, item, lane, p, cb)) {
+            const int t = item[IT_T], h = item[IT_H], tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
+            const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
+            if (!(item[IT_FLAGS] & ITF_LAST)) {
+                // INCL_j (left in the O columns by the state warps) -> workspace,
+                // then the flag that releases the next segment's look-back
+                if (!warp_wait(&cb->incl_ready, incl_n & 1, p, cb)) break;
+                ++incl_n;
+                tc_fence_after();
+                float *dst = p.incl + (size_t)t * D * D;
+#pragma unroll 1
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t x[64];
+                    tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
+                    if (hf == 1) {  // all of INCL_j is in registers: the O columns are free
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&cb->a_free);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        __stcg(reinterpret_cast<float4 *>(dst + incl_off(r, hf * 16 + c)),
+                               make_float4(__uint_as_float(x[4 * c]), __uint_as_float(x[4 * c + 1]),
+                                           __uint_as_float(x[4 * c + 2]), __uint_as_float(x[4 * c + 3])));
+                }
+                asm volatile("fence.acq_rel.gpu;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cb->pub);
+                if (r == 0) {
+                    const bool all_in = wait_or_abort(&cb->pub, pub_n & 1, p, cb);
+                    if (all_in && p.inject != LA_INJECT_SKIP_PUBLISH) {
+                        const int two = 2;
+                        int *fl = p.flags + t;
+                        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(fl), "r"(two) : "memory");
+                    }
+                }
+                ++pub_n;
+            }
+            for (int b = 0; b < nblk && ok; ++b) {
+                const uint32_t bn = blk_n + b;
+                const int row0 = tok0 + b * BLK;
+                const int valid = min(BLK, tok1 - row0);
+                if (!warp_wait(&cb->o_full, bn & 1, p, cb)) { ok = false; break; }
+                tc_fence_after();
+                const size_t orow = ((size_t)(row0 + r) * H + h) * D;
+                // two rounds of 64 columns; the O buffer is released once the
+                // second round is in registers
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t x[64];
+                    tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
+                    if (hf == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&cb->o_empty);
+                    }
+                    if (r < valid) {
+                        if (!p.out_fp32) {
+                            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out) + orow + hf * 64;
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                __stcs(reinterpret_cast<uint4 *>(o + 8 * q),
+                                       make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
+                                                  bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7])));
+                        } else {
+                            float *o = reinterpret_cast<float *>(p.out) + orow + hf * 64;
+#pragma unroll
+                            for (int q = 0; q < 16; ++q)
+                                __stcs(reinterpret_cast<float4 *>(o + 4 * q),
+                                       make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
+                                                   __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3])));
+                        }
+                    }
+                }
+            }
+            blk_n += nblk;
+        }
+    } else {
+        // ===== warps 10-13: segment hand-off (phase L), state snapshots, final state =====
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+        uint32_t it = 0, snap_n = 0, upd_n = 0, agg_n = 0;
         uint8_t *shi = smem + SM_SHI;
         uint8_t *slo = smem + SM_SLO;
-        while (true) {
-            const int islot = it & 1;
-            if (!warp_wait(&cb->item_full[islot], (it >> 1) & 1, p, cb)) break;
-            int item[8];
-#pragma unroll
-            for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&cb->item_empty[islot]);
-            ++it;
-            if (!item[IT_VALID]) break;
+        int item[8];
+        while (next_item(it, item, lane, p, cb)) {
             const int t = item[IT_T], h = item[IT_H], seq = item[IT_SEQ];
             const int tok0 = item[IT_TOK0], tok1 = item[IT_TOK1], j = item[IT_J];
             const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
@@ -801,62 +820,43 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 ++agg_n;
                 tc_fence_after();
             }
-            float *dst_incl = p.incl + (size_t)t * D * D;
 #pragma unroll 1
-            for (int hf = 0; hf < 2; ++hf) {  // two halves of 64 columns
-                float e[64];
+            for (int qq = 0; qq < 4; ++qq) {  // four groups of 32 columns
+                uint32_t e[32];
                 if (src_incl && ok) {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 x = __ldcg(reinterpret_cast<const float4 *>(src_incl + incl_off(r, hf * 16 + q)));
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 x = __ldcg(reinterpret_cast<const uint4 *>(src_incl + incl_off(r, qq * 8 + q)));
                         e[4 * q] = x.x; e[4 * q + 1] = x.y; e[4 * q + 2] = x.z; e[4 * q + 3] = x.w;
                     }
                 } else if (src_state) {
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 x = __ldg(reinterpret_cast<const float4 *>(src_state + (size_t)r * D + hf * 64 + 4 * q));
+                    for (int q = 0; q < 8; ++q) {
+                        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src_state + (size_t)r * D + qq * 32 + 4 * q));
                         e[4 * q] = x.x; e[4 * q + 1] = x.y; e[4 * q + 2] = x.z; e[4 * q + 3] = x.w;
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 64; ++q) e[q] = 0.f;
-                }
-                if (!last) {  // INCL_j = E_j + A_j  (A_j sits in an O buffer)
-                    uint32_t a[64];
-                    tmem_ld_cols<64>(trow + TM_O + hf * 64, a);
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        float4 x;
-                        x.x = e[4 * q] + __uint_as_float(a[4 * q]);
-                        x.y = e[4 * q + 1] + __uint_as_float(a[4 * q + 1]);
-                        x.z = e[4 * q + 2] + __uint_as_float(a[4 * q + 2]);
-                        x.w = e[4 * q + 3] + __uint_as_float(a[4 * q + 3]);
-                        __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, hf * 16 + q)), x);
-                    }
+                    for (int q = 0; q < 32; ++q) e[q] = 0u;
                 }
                 // S (TMEM) = E_j: the state the scan of this segment starts from
-                tmem_st32(trow + TM_S + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&e[0]));
-                tmem_st32(trow + TM_S + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&e[32]));
+                tmem_st32(trow + TM_S + qq * 32, e);
+                if (!last) {  // INCL_j = E_j + A_j, written over A_j in the O columns
+                    uint32_t a[32];
+                    tmem_ld_wait32(trow + TM_O + qq * 32, a);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) a[c] = __float_as_uint(__uint_as_float(e[c]) + __uint_as_float(a[c]));
+                    tmem_st32(trow + TM_O + qq * 32, a);
+                }
             }
             tmem_wait_st();
-            // hand E_j to a5 (this also releases A_j's O buffer and lets a6 start)
-            if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) ok = false;
-            if (!last) {
-                // publish INCL_j: every warp orders its stores and arrives; the
-                // owner of row 0 waits (bounded) for all four, then releases the flag
-                asm volatile("fence.acq_rel.gpu;" ::: "memory");
+            if (!last) {  // the store warps publish INCL_j
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->pub);
-                if (r == 0) {
-                    const bool all_in = wait_or_abort(&cb->pub, pub_n & 1, p, cb);
-                    if (all_in && ok && p.inject != LA_INJECT_SKIP_PUBLISH) {
-                        const int two = 2;
-                        int *fl = p.flags + t;
-                        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(fl), "r"(two) : "memory");
-                    }
-                }
-                ++pub_n;
+                if (lane == 0) mbar_arrive(&cb->incl_ready);
             }
+            // hand E_j to a5 of the first block
+            if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) ok = false;
             if (!__all_sync(0xffffffffu, ok && !cb->abort)) break;
 
             // ------------- phase O: state snapshots and the final state -------------
@@ -868,20 +868,22 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 ++upd_n;
                 tc_fence_after();
                 if (b < nblk - 1) {
-                    if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }  // S_{<b+1} for the next block
+                    if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }  // S_{<b+1}
                 } else {
                     // final state of the sequence -> state_out (row-major fp32)
-                    uint32_t x[D];
-                    tmem_ld_cols<D>(trow + TM_S, x);
                     float *so = p.state_out + ((size_t)seq * H + h) * D * D + (size_t)r * D;
+#pragma unroll 1
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint32_t x[32];
+                        tmem_ld_wait32(trow + TM_S + qq * 32, x);
 #pragma unroll
-                    for (int q = 0; q < D / 4; ++q)
-                        *reinterpret_cast<float4 *>(so + 4 * q) =
-                            make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
-                                        __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3]));
+                        for (int c = 0; c < 8; ++c)
+                            *reinterpret_cast<float4 *>(so + qq * 32 + 4 * c) =
+                                make_float4(__uint_as_float(x[4 * c]), __uint_as_float(x[4 * c + 1]),
+                                            __uint_as_float(x[4 * c + 2]), __uint_as_float(x[4 * c + 3]));
+                    }
                 }
             }
-            blk_n += nblk;
             if (!ok) break;
         }
     }

@@ -69,16 +69,32 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity to complete.
 // Returns false if `deadline` (globaltimer ns) passed or *abort became nonzero.
+#ifndef LA_WAIT_MODE
+#define LA_WAIT_MODE 0
+#endif
 __device__ __forceinline__ bool la_wait(uint64_t *bar, uint32_t parity, uint64_t deadline,
                                         volatile int *abort) {
     uint32_t n = 0;
-    while (!mbar_try_wait(bar, parity)) {
+    for (;;) {
+#if LA_WAIT_MODE == 2
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(1000u) : "memory");
+        if (ok) return true;
+#else
+        if (mbar_try_wait(bar, parity)) return true;
+#if LA_WAIT_MODE == 1
+        __nanosleep(LA_WAIT_SLEEP_NS);
+#endif
+#endif
         if (((++n) & 255u) == 0u) {
             if (*abort) return false;
             if (globaltimer_ns() > deadline) return false;
         }
     }
-    return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -218,6 +234,38 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Warp-collective forms: every lane of a converged warp executes the
+// instruction and elect.sync picks the one lane that issues it.  Issuing from
+// a converged warp keeps tcgen05.mma at the tensor pipe's rate; issuing from a
+// one-lane divergent branch measured about a third slower per MMA.
+__device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_w(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+        ::"r"(smem_u32(bar)) : "memory");
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]
