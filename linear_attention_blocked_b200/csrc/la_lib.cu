@@ -197,6 +197,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.state_out = state_out;
     pp.out = out;
     pp.out_fp32 = out_dtype == LA_FP32;
+    pp.out_al32 = aligned(out, 32);
     pp.H = H;
     pp.hdr = sp.hdr;
     pp.segs = sp.segs;
@@ -457,6 +458,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.state_out = state_out;
     pp.out = out;
     pp.out_fp32 = out_dtype == LA_FP32;
+    pp.out_al32 = aligned(out, 32);
     pp.H = H;
     pp.hdr = sp.hdr;
     pp.segs = sp.segs;

@@ -98,6 +98,7 @@ struct PrefillParams {
     float *state_out;       // [nseq, H, D, D] or null
     void *out;              // [T, H, D]
     int out_fp32;
+    int out_al32;           // out is 32-byte aligned: rows are written with 32-byte stores
     int H;
     int *hdr;               // workspace header
     const int4 *segs;       // [G] {seq, tok0, tok1, jinfo}
@@ -290,9 +291,9 @@ __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane
                                           CtrlBlock *cb) {
     const int islot = it & 1;
     if (!warp_wait(&cb->item_full[islot], (it >> 1) & 1, p, cb)) return false;
+    // broadcast from lane 0, so that the compiler knows the fields are warp-uniform
 #pragma unroll
-    for (int f = 0; f < 8; ++f) item[f] = cb->item[islot][f];
-    __syncwarp();
+    for (int f = 0; f < 8; ++f) item[f] = __shfl_sync(0xffffffffu, cb->item[islot][f], 0);
     if (lane == 0) mbar_arrive(&cb->item_empty[islot]);
     ++it;
     return item[IT_VALID] != 0;
@@ -305,7 +306,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     CtrlBlock *cb = reinterpret_cast<CtrlBlock *>(smem + SM_CTRL);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // warp index and TMEM base through a shuffle: provably warp-uniform values,
+    // so role branches and MMA operands stay in uniform registers
+    const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0), lane = threadIdx.x & 31;
     const uint32_t sbase = smem_u32(smem);
 
     if (threadIdx.x == 0) {
@@ -346,7 +349,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = cb->tmem_base;
+    const uint32_t tmem = __shfl_sync(0xffffffffu, cb->tmem_base, 0);
     const int H = p.H;
 
     if (warp == 0) {
@@ -737,32 +740,52 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 if (!warp_wait(&cb->o_full, bn & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
                 const size_t orow = ((size_t)(row0 + r) * H + h) * D;
-                // two rounds of 64 columns; the O buffer is released once the
-                // second round is in registers
+                if (!p.out_fp32) {
+                    // both 64-column rounds into registers (packed to bf16 as they
+                    // arrive), release the O buffer, then write the row with 32-byte
+                    // stores: full sectors, and no store queued ahead of the TMEM loads
+                    uint32_t w[64];
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t x[64];
-                    tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
-                    if (hf == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&cb->o_empty);
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t x[64];
+                        tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) w[hf * 32 + c] = bf16x2_round(x[2 * c], x[2 * c + 1]);
                     }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&cb->o_empty);
                     if (r < valid) {
-                        if (!p.out_fp32) {
-                            __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out) + orow + hf * 64;
+                        uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow);
+                        if (p.out_al32) {
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                __stcs(reinterpret_cast<uint4 *>(o + 8 * q),
-                                       make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
-                                                  bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7])));
+                            for (int q = 0; q < 8; ++q) st_global_cs_v8(o + 8 * q, &w[8 * q]);
                         } else {
-                            float *o = reinterpret_cast<float *>(p.out) + orow + hf * 64;
 #pragma unroll
                             for (int q = 0; q < 16; ++q)
-                                __stcs(reinterpret_cast<float4 *>(o + 4 * q),
-                                       make_float4(__uint_as_float(x[4 * q]), __uint_as_float(x[4 * q + 1]),
-                                                   __uint_as_float(x[4 * q + 2]), __uint_as_float(x[4 * q + 3])));
+                                __stcs(reinterpret_cast<uint4 *>(o + 4 * q), make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t x[64];
+                        tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
+                        if (hf == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&cb->o_empty);
+                        }
+                        if (r < valid) {
+                            uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(p.out) + orow + hf * 64);
+                            if (p.out_al32) {
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) st_global_cs_v8(o + 8 * q, &x[8 * q]);
+                            } else {
+#pragma unroll
+                                for (int q = 0; q < 16; ++q)
+                                    __stcs(reinterpret_cast<uint4 *>(o + 4 * q), make_uint4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+                            }
                         }
                     }
                 }

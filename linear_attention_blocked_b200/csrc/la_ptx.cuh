@@ -343,6 +343,14 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 32-byte global store with the streaming hint (a full sector per thread);
+// `addr` must be 32-byte aligned.
+__device__ __forceinline__ void st_global_cs_v8(void *addr, const uint32_t *v) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"l"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                   "r"(v[7]) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Shared-memory matrix descriptors (tcgen05 "matrix descriptor" format):
 //   bits  0-13 start address >> 4

@@ -229,3 +229,21 @@ def test_empty_problems():
     out, st = la.prefill_varlen(zt, zt, zt, cu, 0, state_in=sin3)
     assert torch.equal(st, sin3)
     assert la.get_device_status() == la.LA_OK
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_output_only_16_byte_aligned(oracle_mod, dtype):
+    """An output buffer that is 16- but not 32-byte aligned (the minimum the C
+    ABI accepts) takes the 16-byte store path and gives the same result."""
+    B, N, H = 1, 640, 2
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=61, device="cuda")
+    esz = torch.finfo(dtype).bits // 8
+    flat = torch.empty(B * N * H * D + 64, dtype=dtype, device="cuda")
+    shift = (16 - flat.data_ptr() % 32) % 32 // esz  # first element 16 bytes past a 32-byte boundary
+    out = flat[shift:shift + B * N * H * D].view(B, N, H, D)
+    assert out.data_ptr() % 32 == 16
+    la.set_segment_len(256)
+    out2, _ = la.prefill(q, k, v, out=out, out_dtype=dtype)
+    assert out2.data_ptr() == out.data_ptr()
+    ref, _ = _oracle_prefill(oracle_mod, q[0], k[0], v[0], np.array([0, N], np.int32))
+    check_out(to_np(out[0]), ref, bf16_out=dtype == torch.bfloat16, what="16-byte aligned out")
