@@ -124,9 +124,8 @@ struct CtrlBlock {
     uint64_t snap_full;           // [4] state warps: snapshot of S in shared memory (S read)
     uint64_t snap_empty;          // [1] a5 has read the snapshot
     uint64_t agg_full;            // [1] phase A done: A_j in the O columns
-    uint64_t incl_ready;          // [4] state warps: INCL_j written over A_j in the O columns
-    uint64_t a_free;              // [4] store warps: INCL_j read, the O columns are free
-    uint64_t pub;                 // [4] store warps: INCL_j stores ordered before the flag
+    uint64_t a_free;              // [4] state warps: A_j read, the O columns are free
+    uint64_t incl_stored;         // [4] state warps: INCL_j written to the workspace
     uint64_t item_full[2];        // [1] producer
     uint64_t item_empty[2];       // [14] Q producer lane + MMA lane 0 + 3 x 4 warps
     uint64_t fin;                 // [1] tear-down: every MMA done
@@ -332,9 +331,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         mbar_init(&cb->snap_full, 4);
         mbar_init(&cb->snap_empty, 1);
         mbar_init(&cb->agg_full, 1);
-        mbar_init(&cb->incl_ready, 4);
         mbar_init(&cb->a_free, 4);
-        mbar_init(&cb->pub, 4);
+        mbar_init(&cb->incl_stored, 4);
         mbar_init(&cb->fin, 1);
         cb->abort = 0;
         fence_mbarrier_init();
@@ -692,42 +690,22 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
-        uint32_t it = 0, blk_n = 0, incl_n = 0, pub_n = 0;
+        uint32_t it = 0, blk_n = 0, pub_n = 0;
         bool ok = true;
         int item[8];
         while (ok && next_item(it, item, lane, p, cb)) {
             const int t = item[IT_T], h = item[IT_H], tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
             if (!(item[IT_FLAGS] & ITF_LAST)) {
-                // INCL_j (left in the O columns by the state warps) -> workspace,
-                // then the flag that releases the next segment's look-back
-                if (!warp_wait(&cb->incl_ready, incl_n & 1, p, cb)) break;
-                ++incl_n;
-                tc_fence_after();
-                float *dst = p.incl + (size_t)t * D * D;
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    uint32_t x[64];
-                    tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
-                    if (hf == 1) {  // all of INCL_j is in registers: the O columns are free
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&cb->a_free);
-                    }
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        __stcg(reinterpret_cast<float4 *>(dst + incl_off(r, hf * 16 + c)),
-                               make_float4(__uint_as_float(x[4 * c]), __uint_as_float(x[4 * c + 1]),
-                                           __uint_as_float(x[4 * c + 2]), __uint_as_float(x[4 * c + 3])));
-                }
-                asm volatile("fence.acq_rel.gpu;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->pub);
+                // the state warps have written INCL_j: release the flag the next
+                // segment's look-back waits for (this thread's acquire on the
+                // barrier orders their stores before its release)
                 if (r == 0) {
-                    const bool all_in = wait_or_abort(&cb->pub, pub_n & 1, p, cb);
+                    const bool all_in = wait_or_abort(&cb->incl_stored, pub_n & 1, p, cb);
                     if (all_in && p.inject != LA_INJECT_SKIP_PUBLISH) {
                         const int two = 2;
                         int *fl = p.flags + t;
+                        asm volatile("fence.acq_rel.gpu;" ::: "memory");
                         asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(fl), "r"(two) : "memory");
                     }
                 }
@@ -843,43 +821,75 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 ++agg_n;
                 tc_fence_after();
             }
+            // E_j -> S (TMEM); INCL_j = E_j + A_j -> workspace straight from registers;
+            // E_j as bf16 -> the snapshot buffer for a5 of the first block (one
+            // bf16 term: written here; hi + lo: through snapshot_state below)
+            const bool snap_here = !lo;
+            if (snap_here && !warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) ok = false;
+            float *dst_incl = p.incl + (size_t)t * D * D;
 #pragma unroll 1
-            for (int qq = 0; qq < 4; ++qq) {  // four groups of 32 columns
-                uint32_t e[32];
+            for (int hf = 0; hf < 2; ++hf) {  // two halves of 64 columns
+                uint32_t e[64];
                 if (src_incl && ok) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 x = __ldcg(reinterpret_cast<const uint4 *>(src_incl + incl_off(r, qq * 8 + q)));
+                    for (int q = 0; q < 16; ++q) {
+                        const uint4 x = __ldcg(reinterpret_cast<const uint4 *>(src_incl + incl_off(r, hf * 16 + q)));
                         e[4 * q] = x.x; e[4 * q + 1] = x.y; e[4 * q + 2] = x.z; e[4 * q + 3] = x.w;
                     }
                 } else if (src_state) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src_state + (size_t)r * D + qq * 32 + 4 * q));
+                    for (int q = 0; q < 16; ++q) {
+                        const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src_state + (size_t)r * D + hf * 64 + 4 * q));
                         e[4 * q] = x.x; e[4 * q + 1] = x.y; e[4 * q + 2] = x.z; e[4 * q + 3] = x.w;
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) e[q] = 0u;
+                    for (int q = 0; q < 64; ++q) e[q] = 0u;
                 }
-                // S (TMEM) = E_j: the state the scan of this segment starts from
-                tmem_st32(trow + TM_S + qq * 32, e);
-                if (!last) {  // INCL_j = E_j + A_j, written over A_j in the O columns
-                    uint32_t a[32];
-                    tmem_ld_wait32(trow + TM_O + qq * 32, a);
+                tmem_st32(trow + TM_S + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&e[0]));
+                tmem_st32(trow + TM_S + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&e[32]));
+                if (snap_here) {
+                    uint8_t *half = hf ? slo : shi;
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) a[c] = __float_as_uint(__uint_as_float(e[c]) + __uint_as_float(a[c]));
-                    tmem_st32(trow + TM_O + qq * 32, a);
+                    for (int q = 0; q < 8; ++q)  // 16-byte chunks of 8 columns
+                        *reinterpret_cast<uint4 *>(half + r * 128 + ((q ^ (r & 7)) << 4)) =
+                            make_uint4(bf16x2_round(e[8 * q], e[8 * q + 1]), bf16x2_round(e[8 * q + 2], e[8 * q + 3]),
+                                       bf16x2_round(e[8 * q + 4], e[8 * q + 5]), bf16x2_round(e[8 * q + 6], e[8 * q + 7]));
+                }
+                if (!last) {
+#pragma unroll
+                    for (int qq = 0; qq < 2; ++qq) {
+                        uint32_t a[32];
+                        tmem_ld_wait32(trow + TM_O + hf * 64 + qq * 32, a);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, hf * 16 + qq * 8 + c)),
+                                   make_float4(__uint_as_float(e[qq * 32 + 4 * c]) + __uint_as_float(a[4 * c]),
+                                               __uint_as_float(e[qq * 32 + 4 * c + 1]) + __uint_as_float(a[4 * c + 1]),
+                                               __uint_as_float(e[qq * 32 + 4 * c + 2]) + __uint_as_float(a[4 * c + 2]),
+                                               __uint_as_float(e[qq * 32 + 4 * c + 3]) + __uint_as_float(a[4 * c + 3])));
+                    }
                 }
             }
-            tmem_wait_st();
-            if (!last) {  // the store warps publish INCL_j
+            if (!last) {  // A_j has been read: the O columns are free for a5 of the first block
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->incl_ready);
+                if (lane == 0) mbar_arrive(&cb->a_free);
             }
-            // hand E_j to a5 of the first block
-            if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) ok = false;
+            tmem_wait_st();
+            if (snap_here) {
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cb->snap_full);
+                ++snap_n;
+            } else if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) {
+                ok = false;
+            }
+            if (!last) {  // INCL_j is written: the store warps release the flag
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&cb->incl_stored);
+            }
             if (!__all_sync(0xffffffffu, ok && !cb->abort)) break;
 
             // ------------- phase O: state snapshots and the final state -------------
