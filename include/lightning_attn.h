@@ -132,6 +132,51 @@ LA_API la_status la_decode_step(const void *q, const void *k, const void *v, flo
                          cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * State slots and the mixed prefill/decode step ("MiniMax-01技术报告解读",
+ * §3.3 item 2: prefill and decode requests are served on separate CUDA
+ * streams, with the length-1 tokens routed to the decode kernel; item 1: the
+ * decode kernel updates the prefix-KV cache in place).
+ *
+ * A state pool is device fp32 [n_slots, H, d, d]: one running state per
+ * request.  `slots` (DEVICE int32) maps each sequence or decode row to its
+ * slot; a slot outside [0, n_slots) computes nothing for that sequence or
+ * row and records LA_ERR_INVALID_ARGUMENT in the sticky device word.  Two
+ * sequences or rows of one call must not name the same slot (the results
+ * are then undefined; nothing checks it).
+ *
+ * la_prefill_varlen_slots: la_prefill_varlen where sequence i starts from
+ *   state_pool[slots[i]] and leaves its final state there (in place).
+ *   A zero-length sequence leaves its slot unchanged.
+ * la_decode_step_slots: la_decode_step where row b updates state_pool[slots[b]].
+ * la_mixed_step: one batch of requests, rows [0, prefill_tokens) of q, k, v
+ *   and out packed as prefill chunks (cu_seqlens, prefill_slots), rows
+ *   [prefill_tokens, prefill_tokens + n_decode) one decode token each
+ *   (decode_slots).  The prefill is launched on prefill_stream and the
+ *   decode on decode_stream; when the two streams differ, prefill_stream
+ *   then waits (cudaStreamWaitEvent) for the decode, so work queued on
+ *   prefill_stream after the call sees both results.  The workspace is the
+ *   la_prefill_varlen workspace for (n_prefill, prefill_tokens).  Argument
+ *   errors of either part are returned before anything is launched.
+ * ------------------------------------------------------------------------- */
+LA_API la_status la_prefill_varlen_slots(const void *q, const void *k, const void *v,
+                                  const int *cu_seqlens, const int *slots, int nseq,
+                                  int total_tokens, int max_seqlen, int H, int d, int block,
+                                  float *state_pool, int n_slots, void *out,
+                                  la_dtype out_dtype, void *workspace, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+LA_API la_status la_decode_step_slots(const void *q, const void *k, const void *v,
+                               float *state_pool, int n_slots, const int *slots, void *out,
+                               la_dtype out_dtype, int B, int H, int d, cudaStream_t stream);
+
+LA_API la_status la_mixed_step(const void *q, const void *k, const void *v,
+                        const int *cu_seqlens, const int *prefill_slots, int n_prefill,
+                        int prefill_tokens, int max_seqlen, const int *decode_slots,
+                        int n_decode, int H, int d, float *state_pool, int n_slots, void *out,
+                        la_dtype out_dtype, void *workspace, size_t ws_bytes,
+                        cudaStream_t prefill_stream, cudaStream_t decode_stream);
+
+/* ---------------------------------------------------------------------------
  * la_prefill without a workspace argument, for callers that cannot allocate
  * device memory when they call: e.g. a plugin inside a host framework that
  * owns the allocator and offers no allocation hook, or a serving process that

@@ -7,12 +7,18 @@ ABI (include/lightning_attn.h).  Entry points:
   prefill(q, k, v, ...)                      la_prefill          [B, N, H, 128]
   prefill_varlen(q, k, v, cu_seqlens, ...)   la_prefill_varlen   [T, H, 128] packed
   decode_step(q, k, v, state, ...)           la_decode_step      [B, H, 128]
+  prefill_varlen_slots / decode_step_slots   the same on a pool of per-request states
+  mixed_step(q, k, v, cu_seqlens, ...)       la_mixed_step: prefill chunks and decode tokens
+                                             of one batch on two streams (plan with
+                                             serving.plan_batch)
   get_device_status()                        la_get_device_status
 """
 from ._binding import (D, DEFAULT_BLOCK, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
                        LA_ERR_INVALID_ARGUMENT, LA_ERR_TIMEOUT, LA_ERR_UNSUPPORTED,
                        LA_ERR_WORKSPACE, LA_FP32, LA_INJECT_NONE, LA_INJECT_SKIP_PUBLISH, LA_OK,
-                       LAError, debug_inject, decode_step, get_device_status, kernel_launches,
-                       last_segment_len, lib, library_path, prefill, prefill_varlen,
+                       LAError, debug_inject, decode_step, decode_step_slots, get_device_status,
+                       kernel_launches, last_segment_len, lib, library_path, mixed_step, prefill,
+                       prefill_varlen, prefill_varlen_slots,
                        set_segment_len, set_wait_limit_ns, status_string, varlen_workspace_size,
                        workspace_size)
+from .serving import BatchPlan, plan_batch  # noqa: F401,E402

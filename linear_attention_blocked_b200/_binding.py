@@ -23,7 +23,8 @@ DEFAULT_BLOCK = 128
 EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_workspace_size",
             "la_prefill_varlen", "la_decode_step", "la_get_device_status", "la_status_string",
             "la_set_wait_limit_ns", "la_set_segment_len", "la_debug_inject",
-            "la_last_segment_len", "la_kernel_launches", "la_prefill_noalloc")
+            "la_last_segment_len", "la_kernel_launches", "la_prefill_noalloc",
+            "la_prefill_varlen_slots", "la_decode_step_slots", "la_mixed_step")
 
 
 class LAError(RuntimeError):
@@ -64,6 +65,14 @@ def lib():
         L.la_prefill_noalloc.restype = c_int
         L.la_decode_step.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
         L.la_decode_step.restype = c_int
+        L.la_prefill_varlen_slots.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                              vp, c_int, vp, c_int, vp, sz, vp]
+        L.la_prefill_varlen_slots.restype = c_int
+        L.la_decode_step_slots.argtypes = [vp, vp, vp, vp, c_int, vp, vp, c_int, c_int, c_int, c_int, vp]
+        L.la_decode_step_slots.restype = c_int
+        L.la_mixed_step.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, vp, c_int, c_int, c_int, vp, c_int,
+                                    vp, c_int, vp, sz, vp, vp]
+        L.la_mixed_step.restype = c_int
         L.la_get_device_status.argtypes = [vp]
         L.la_get_device_status.restype = c_int
         L.la_status_string.argtypes = [c_int]
@@ -209,6 +218,97 @@ def decode_step(q, k, v, state, out=None, out_dtype=torch.bfloat16, stream=None)
     st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), _out_code(out.dtype),
                               B, H, d, _stream_handle(stream))
     _check(st, "la_decode_step")
+    return out
+
+
+def _need_pool(state_pool, H, d):
+    if state_pool.dim() != 4:
+        raise ValueError("state_pool must be [n_slots, H, d, d]")
+    _need(state_pool, "state_pool", torch.float32, (state_pool.shape[0], H, d, d))
+    return int(state_pool.shape[0])
+
+
+def prefill_varlen_slots(q, k, v, cu_seqlens, slots, max_seqlen: int, state_pool, out=None,
+                         out_dtype=torch.bfloat16, workspace=None, stream=None):
+    """la_prefill_varlen_slots: sequence i starts from state_pool[slots[i]] and
+    leaves its final state there.  slots: device int32 [nseq]."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, d]")
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (T, H, d))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    nseq = cu_seqlens.numel() - 1
+    _need(slots, "slots", torch.int32, (nseq,))
+    n_slots = _need_pool(state_pool, H, d)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=out_dtype, device=q.device)
+    _need(out, "out", out.dtype, (T, H, d))
+    ws_bytes = varlen_workspace_size(nseq, T, max_seqlen, H, d)
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, q.device)
+    st = lib().la_prefill_varlen_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(slots), nseq, T,
+                                       int(max_seqlen), H, d, 0, _ptr(state_pool), n_slots, _ptr(out),
+                                       _out_code(out.dtype), _ptr(workspace),
+                                       workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "la_prefill_varlen_slots")
+    return out
+
+
+def decode_step_slots(q, k, v, state_pool, slots, out=None, out_dtype=torch.bfloat16, stream=None):
+    """la_decode_step_slots: row b updates state_pool[slots[b]] in place."""
+    if q.dim() != 3:
+        raise ValueError("q must be [B, H, d]")
+    B, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (B, H, d))
+    _need(slots, "slots", torch.int32, (B,))
+    n_slots = _need_pool(state_pool, H, d)
+    if out is None:
+        out = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
+    _need(out, "out", out.dtype, (B, H, d))
+    st = lib().la_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(state_pool), n_slots, _ptr(slots),
+                                    _ptr(out), _out_code(out.dtype), B, H, d, _stream_handle(stream))
+    _check(st, "la_decode_step_slots")
+    return out
+
+
+def mixed_step(q, k, v, cu_seqlens, prefill_slots, max_seqlen: int, decode_slots, state_pool, out=None,
+               out_dtype=torch.bfloat16, workspace=None, prefill_stream=None, decode_stream=None):
+    """la_mixed_step on one packed batch: rows [0, T_p) are prefill chunks
+    (cu_seqlens, prefill_slots), the last n_decode rows one decode token each
+    (decode_slots).  Prefill runs on prefill_stream, decode on decode_stream;
+    prefill_stream then waits for the decode."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, d]")
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (T, H, d))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    n_prefill = cu_seqlens.numel() - 1
+    _need(prefill_slots, "prefill_slots", torch.int32, (n_prefill,))
+    _need(decode_slots, "decode_slots", torch.int32)
+    n_decode = decode_slots.numel()
+    T_p = T - n_decode
+    if T_p < 0:
+        raise ValueError("fewer rows than decode tokens")
+    n_slots = _need_pool(state_pool, H, d)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=out_dtype, device=q.device)
+    _need(out, "out", out.dtype, (T, H, d))
+    ws_bytes = varlen_workspace_size(max(n_prefill, 1), T_p, max_seqlen, H, d)
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, q.device)
+    if prefill_stream is None:
+        prefill_stream = torch.cuda.current_stream()
+    if decode_stream is None:
+        decode_stream = prefill_stream
+    st = lib().la_mixed_step(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), _ptr(prefill_slots), n_prefill, T_p,
+                             int(max_seqlen), _ptr(decode_slots), n_decode, H, d, _ptr(state_pool), n_slots,
+                             _ptr(out), _out_code(out.dtype), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream_handle(prefill_stream),
+                             _stream_handle(decode_stream))
+    _check(st, "la_mixed_step")
     return out
 
 

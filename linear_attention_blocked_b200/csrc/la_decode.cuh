@@ -33,10 +33,14 @@ __device__ __forceinline__ void st_stream_f4(float *p, float4 v) {
                  "f"(v.w) : "memory");
 }
 
+// Row b of q/k/v/out updates state b, or, with `slots`, state slots[b] of a
+// pool of n_slots (sequence, H heads) states; a slot outside [0, n_slots)
+// skips the row and records LA_ERR_INVALID_ARGUMENT in the status word.
 __global__ void __launch_bounds__(DEC_THREADS)
 la_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, float *__restrict__ state, void *__restrict__ out,
-                 int out_fp32, long long npairs) {
+                 int out_fp32, long long npairs, int H, const int *__restrict__ slots, int n_slots,
+                 int *status) {
     constexpr int Dd = 128;
     __shared__ float red[8][Dd];
     __shared__ float qs[Dd], ks[Dd];
@@ -44,7 +48,17 @@ la_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
     const int g = tid >> 5, c = tid & 31;
     for (long long pair = blockIdx.x; pair < npairs; pair += gridDim.x) {
         const size_t vec = (size_t)pair * Dd;
-        float *S = state + (size_t)pair * Dd * Dd;
+        long long spair = pair;
+        if (slots) {
+            const long long b = pair / H;
+            const int slot = slots[b];
+            if (slot < 0 || slot >= n_slots) {  // uniform across the block
+                if (tid == 0 && pair % H == 0) atomicCAS(status, 0, 1);
+                continue;
+            }
+            spair = (long long)slot * H + (pair - b * H);
+        }
+        float *S = state + (size_t)spair * Dd * Dd;
         float4 s[DEC_ROWS_PER_THREAD];
 #pragma unroll
         for (int m = 0; m < DEC_ROWS_PER_THREAD; ++m)

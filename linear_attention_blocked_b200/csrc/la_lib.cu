@@ -129,7 +129,8 @@ la_status check_common(int H, int d, int block, la_dtype out_dtype) {
 la_status prefill_impl(const void *q, const void *k, const void *v, const int *cu, int fixed_len,
                        int nseq, long long T, int max_seqlen, int H, int d, int block,
                        const float *state_in, void *out, la_dtype out_dtype, float *state_out,
-                       void *workspace, size_t ws_bytes, cudaStream_t stream) {
+                       void *workspace, size_t ws_bytes, cudaStream_t stream,
+                       const int *slots = nullptr, int n_slots = 0) {
     la_status st = check_common(H, d, block, out_dtype);
     if (st != LA_OK) return st;
     if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -141,7 +142,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
         if (p && !aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
     const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
     const size_t n_in = (size_t)T * H * la::D * 2, n_out = (size_t)T * H * la::D * esz;
-    const size_t n_state = (size_t)nseq * H * la::D * la::D * 4;
+    if (slots && (n_slots <= 0 || !aligned(slots, 4) || state_in != state_out || !state_out))
+        return LA_ERR_INVALID_ARGUMENT;
+    const size_t n_state = (size_t)(slots ? n_slots : nseq) * H * la::D * la::D * 4;
     if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
     const void *ins[3] = {q, k, v};
@@ -181,6 +184,8 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     sp.flags = reinterpret_cast<int *>(ws + w.flags);
     sp.state_in = state_in;
     sp.state_out = state_out;
+    sp.slots = slots;
+    sp.n_slots = n_slots;
     sp.status = status;
     la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
@@ -195,6 +200,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     la::PrefillParams pp;
     pp.state_in = state_in;
     pp.state_out = state_out;
+    pp.slots = slots;
     pp.out = out;
     pp.out_fp32 = out_dtype == LA_FP32;
     pp.out_al32 = aligned(out, 32);
@@ -218,6 +224,36 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
     la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
+
+// Shared body of la_decode_step / la_decode_step_slots.
+la_status decode_impl(const void *q, const void *k, const void *v, float *state, const int *slots, int n_slots,
+                      void *out, la_dtype out_dtype, int B, int H, int d, cudaStream_t stream) {
+    la_status st = check_common(H, d, 0, out_dtype);
+    if (st != LA_OK) return st;
+    if (B < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (B == 0) return LA_OK;
+    if (!q || !k || !v || !state || !out) return LA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[5] = {q, k, v, state, out};
+    for (const void *p : ptrs)
+        if (!aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+    if (slots && (n_slots <= 0 || !aligned(slots, 4))) return LA_ERR_INVALID_ARGUMENT;
+    const long long npairs = (long long)B * H;
+    const long long nstates = (slots ? (long long)n_slots : (long long)B) * H;
+    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
+    if (ranges_overlap(out, npairs * la::D * esz, state, nstates * la::D * la::D * 4))
+        return LA_ERR_INVALID_ARGUMENT;
+    const long long grid = npairs < (1LL << 30) ? npairs : (1LL << 30);
+    int *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_la_status) != cudaSuccess)
+        return LA_ERR_CUDA;
+    la::la_decode_kernel<<<(unsigned)grid, la::DEC_THREADS, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), state, out, out_dtype == LA_FP32, npairs, H, slots, n_slots,
+        status);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;
@@ -265,28 +301,77 @@ la_status la_prefill_varlen(const void *q, const void *k, const void *v, const i
                         out, out_dtype, state_out, workspace, ws_bytes, stream);
 }
 
+la_status la_prefill_varlen_slots(const void *q, const void *k, const void *v, const int *cu_seqlens,
+                                  const int *slots, int nseq, int total_tokens, int max_seqlen, int H, int d,
+                                  int block, float *state_pool, int n_slots, void *out, la_dtype out_dtype,
+                                  void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!cu_seqlens || nseq < 0 || total_tokens < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (nseq > 0 && (!slots || !state_pool)) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARGUMENT;
+    if (nseq == 0) return total_tokens == 0 ? LA_OK : LA_ERR_INVALID_ARGUMENT;
+    return prefill_impl(q, k, v, cu_seqlens, 0, nseq, total_tokens, max_seqlen, H, d, block, state_pool,
+                        out, out_dtype, state_pool, workspace, ws_bytes, stream, slots, n_slots);
+}
+
 la_status la_decode_step(const void *q, const void *k, const void *v, float *state, void *out,
                          la_dtype out_dtype, int B, int H, int d, cudaStream_t stream) {
+    return decode_impl(q, k, v, state, nullptr, 0, out, out_dtype, B, H, d, stream);
+}
+
+la_status la_decode_step_slots(const void *q, const void *k, const void *v, float *state_pool, int n_slots,
+                               const int *slots, void *out, la_dtype out_dtype, int B, int H, int d,
+                               cudaStream_t stream) {
+    if (B > 0 && !slots) return LA_ERR_INVALID_ARGUMENT;
+    return decode_impl(q, k, v, state_pool, slots, n_slots, out, out_dtype, B, H, d, stream);
+}
+
+la_status la_mixed_step(const void *q, const void *k, const void *v, const int *cu_seqlens,
+                        const int *prefill_slots, int n_prefill, int prefill_tokens, int max_seqlen,
+                        const int *decode_slots, int n_decode, int H, int d, float *state_pool, int n_slots,
+                        void *out, la_dtype out_dtype, void *workspace, size_t ws_bytes,
+                        cudaStream_t prefill_stream, cudaStream_t decode_stream) {
     la_status st = check_common(H, d, 0, out_dtype);
     if (st != LA_OK) return st;
-    if (B < 0) return LA_ERR_INVALID_ARGUMENT;
-    if (B == 0) return LA_OK;
-    if (!q || !k || !v || !state || !out) return LA_ERR_INVALID_ARGUMENT;
-    const void *ptrs[5] = {q, k, v, state, out};
-    for (const void *p : ptrs)
-        if (!aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
-    const long long npairs = (long long)B * H;
-    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
-    if (ranges_overlap(out, npairs * la::D * esz, state, npairs * la::D * la::D * 4))
+    if (n_prefill < 0 || n_decode < 0 || prefill_tokens < 0 || n_slots <= 0 || !state_pool)
         return LA_ERR_INVALID_ARGUMENT;
-    const long long grid = npairs < (1LL << 30) ? npairs : (1LL << 30);
-    la::la_decode_kernel<<<(unsigned)grid, la::DEC_THREADS, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-        static_cast<const __nv_bfloat16 *>(v), state, out, out_dtype == LA_FP32, npairs);
-    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
-    ++g_launches;
+    if ((long long)prefill_tokens + n_decode > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    if (n_prefill == 0 && prefill_tokens != 0) return LA_ERR_INVALID_ARGUMENT;
+    if (n_decode > 0 && (!decode_slots || !q || !k || !v || !out)) return LA_ERR_INVALID_ARGUMENT;
+    // rows [0, prefill_tokens): packed prefill chunks; rows [prefill_tokens, + n_decode): one
+    // decode token per decode slot
+    const size_t row = (size_t)H * la::D;
+    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
+    if (n_decode > 0) {  // the decode part's checks, before anything is queued
+        const void *ptrs[5] = {q, k, v, out, state_pool};
+        for (const void *p : ptrs)
+            if (!aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+        if (!aligned(decode_slots, 4)) return LA_ERR_INVALID_ARGUMENT;
+        const size_t n_out = ((size_t)prefill_tokens + n_decode) * row * esz;
+        if (ranges_overlap(out, n_out, state_pool, (size_t)n_slots * H * la::D * la::D * 4))
+            return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (n_prefill > 0) {
+        st = la_prefill_varlen_slots(q, k, v, cu_seqlens, prefill_slots, n_prefill, prefill_tokens, max_seqlen, H,
+                                     d, 0, state_pool, n_slots, out, out_dtype, workspace, ws_bytes, prefill_stream);
+        if (st != LA_OK) return st;
+    }
+    if (n_decode > 0) {
+        const size_t off = (size_t)prefill_tokens * row;
+        st = decode_impl(static_cast<const uint16_t *>(q) + off, static_cast<const uint16_t *>(k) + off,
+                         static_cast<const uint16_t *>(v) + off, state_pool, decode_slots, n_slots,
+                         static_cast<uint8_t *>(out) + off * esz, out_dtype, n_decode, H, d, decode_stream);
+        if (st != LA_OK) return st;
+        if (decode_stream != prefill_stream) {
+            // join: work queued on the prefill stream after this call sees both results
+            static thread_local cudaEvent_t ev = nullptr;
+            if (!ev && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return LA_ERR_CUDA;
+            if (cudaEventRecord(ev, decode_stream) != cudaSuccess) return LA_ERR_CUDA;
+            if (cudaStreamWaitEvent(prefill_stream, ev, 0) != cudaSuccess) return LA_ERR_CUDA;
+        }
+    }
     return LA_OK;
 }
+
 
 la_status la_get_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return LA_ERR_CUDA;
@@ -443,6 +528,8 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     sp.flags = reinterpret_cast<int *>(ws + w.flags);
     sp.state_in = state_in;
     sp.state_out = state_out;
+    sp.slots = nullptr;
+    sp.n_slots = 0;
     sp.status = status;
     la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
@@ -456,6 +543,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     la::PrefillParams pp;
     pp.state_in = state_in;
     pp.state_out = state_out;
+    pp.slots = nullptr;
     pp.out = out;
     pp.out_fp32 = out_dtype == LA_FP32;
     pp.out_al32 = aligned(out, 32);

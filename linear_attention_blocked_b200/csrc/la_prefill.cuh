@@ -94,8 +94,9 @@ constexpr int HDR_BYTES = 256;
 constexpr int SEG_LAST = 1 << 30;  // flag bit in SegInfo::jinfo
 
 struct PrefillParams {
-    const float *state_in;  // [nseq, H, D, D] or null
-    float *state_out;       // [nseq, H, D, D] or null
+    const float *state_in;  // [nseq, H, D, D] or null (or a pool of states, see slots)
+    float *state_out;       // [nseq, H, D, D] or null (or a pool of states, see slots)
+    const int *slots;       // null, or [nseq]: sequence i reads and writes state slots[i]
     void *out;              // [T, H, D]
     int out_fp32;
     int out_al32;           // out is 32-byte aligned: rows are written with 32-byte stores
@@ -791,7 +792,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const float *src_state = nullptr;  // row-major [D][D] (state_in) ...
             const float *src_incl = nullptr;   // ... or interleaved (predecessor)
             if (j == 0) {
-                if (p.state_in) src_state = p.state_in + ((size_t)seq * H + h) * D * D;
+                if (p.state_in) src_state = p.state_in + ((size_t)(p.slots ? p.slots[seq] : seq) * H + h) * D * D;
             } else {
                 const int pred = t - H;
                 const int *fl = p.flags + pred;
@@ -904,7 +905,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }  // S_{<b+1}
                 } else {
                     // final state of the sequence -> state_out (row-major fp32)
-                    float *so = p.state_out + ((size_t)seq * H + h) * D * D + (size_t)r * D;
+                    float *so = p.state_out + ((size_t)(p.slots ? p.slots[seq] : seq) * H + h) * D * D + (size_t)r * D;
 #pragma unroll 1
                     for (int qq = 0; qq < 4; ++qq) {
                         uint32_t x[32];
@@ -944,6 +945,8 @@ struct ScheduleParams {
     int *flags;
     const float *state_in;
     float *state_out;
+    const int *slots;       // null, or [nseq] state slots in a pool of n_slots
+    int n_slots;
     int *status;
 };
 
@@ -964,6 +967,9 @@ __global__ void __launch_bounds__(SCHED_THREADS, 1) la_schedule_kernel(const Sch
             if (len < 0 || len > s.max_seqlen) bad = 1;
         }
     }
+    if (s.slots)
+        for (int i = tid; i < s.nseq; i += SCHED_THREADS)
+            if (s.slots[i] < 0 || s.slots[i] >= s.n_slots) bad = 1;
     bad = __syncthreads_or(bad);
     if (bad) {
         if (tid == 0) {
@@ -1016,8 +1022,9 @@ __global__ void __launch_bounds__(SCHED_THREADS, 1) la_schedule_kernel(const Sch
     const int G = carry_sh;
     // 3. reset the hand-off flags of this launch's items
     for (int e = tid; e < G * s.H; e += SCHED_THREADS) s.flags[e] = 0;
-    // 4. empty sequences: the final state is the carried-in state
-    if (s.state_out) {
+    // 4. empty sequences: the final state is the carried-in state (nothing to
+    //    do when the states are updated in place)
+    if (s.state_out && s.state_out != s.state_in) {
         for (int i = 0; i < s.nseq; ++i) {
             if (cu_at(s, i + 1) != cu_at(s, i)) continue;
             const size_t n = (size_t)s.H * D * D, off = (size_t)i * n;

@@ -130,3 +130,32 @@ def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 128, 1, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         la.prefill(q, q, q)
+
+
+def test_slot_and_mixed_argument_errors(L):
+    """The state-pool entry points reject bad arguments before launching."""
+    V = ctypes.c_void_p
+    fake = V(1 << 20)       # never dereferenced: validation fails first
+    bad = la.LA_ERR_INVALID_ARGUMENT
+    # decode rows without a slot map
+    assert L.la_decode_step_slots(fake, fake, fake, fake, 4, None, fake, 0, 2, 2, 128, None) == bad
+    # a pool with no slot
+    assert L.la_decode_step_slots(fake, fake, fake, fake, 0, fake, fake, 0, 2, 2, 128, None) == bad
+    # unsupported head dimension
+    assert L.la_decode_step_slots(fake, fake, fake, fake, 4, fake, fake, 0, 2, 2, 64, None) == la.LA_ERR_UNSUPPORTED
+    # prefill sequences without a slot map or without a pool
+    assert L.la_prefill_varlen_slots(fake, fake, fake, fake, None, 2, 10, 8, 2, 128, 0, fake, 4, fake, 0,
+                                     fake, 1 << 30, None) == bad
+    assert L.la_prefill_varlen_slots(fake, fake, fake, fake, fake, 2, 10, 8, 2, 128, 0, None, 4, fake, 0,
+                                     fake, 1 << 30, None) == bad
+    # mixed step: empty pool, negative counts, prefill tokens without prefill sequences
+    args = lambda **kw: dict(dict(q=fake, k=fake, v=fake, cu=fake, ps=fake, n_p=1, T_p=10, maxlen=10, ds=fake,
+                                  n_d=2, H=2, d=128, pool=fake, n_slots=4, out=fake, od=0, ws=fake,
+                                  wsb=1 << 30, sp=None, sd=None), **kw)
+    call = lambda a: L.la_mixed_step(*a.values())
+    assert call(args(n_slots=0)) == bad
+    assert call(args(n_d=-1)) == bad
+    assert call(args(n_p=0)) == bad
+    assert call(args(ds=None)) == bad
+    assert call(args(pool=None)) == bad
+    assert call(args(d=64)) == la.LA_ERR_UNSUPPORTED
