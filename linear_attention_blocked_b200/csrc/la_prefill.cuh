@@ -40,9 +40,10 @@
 // 128 rows of 128 bytes, written by one TMA box {64, 1, 128, 2} of the 4-D
 // view {64, H, T, 2} of the [T, H, 128] tensor (the halves are its outer
 // dimension).
-// TMEM (512 columns x 128 lanes x 32 bit): Sc0 [0,128) | Sc1 [128,256)
-//   (double-buffered scores; P overwrites the first 64 columns of its buffer in
-//   place) | O [256,384) | S [384,512).
+// TMEM (512 columns x 128 lanes x 32 bit): Sc [0,128) (scores; P overwrites
+//   the first 64 columns in place) | O0 [128,256) | O1 [256,384) (block b
+//   accumulates in O_{b&1}, so O of block b is read out while b+1 runs) |
+//   S [384,512).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -70,6 +71,12 @@ constexpr int W_MASK = 2, W_STORE = 6, W_STATE = 10;  // first warp of each four
 #endif
 constexpr int PF_Q = LA_PREFETCH_Q;
 
+// The scores a2(b+1) are issued only after a4(b): they fill the gap while
+// the tensor pipe waits on the next a5 instead of delaying it, and, since the
+// pipe runs MMAs in issue order, a4(b) has read P(b) before a2(b+1)
+// overwrites the score buffer -- one score buffer suffices, which leaves the
+// TMEM for two O buffers.
+
 constexpr int SM_K = 0;
 constexpr int SM_V = SM_K + KV_STAGES * TILE_BYTES;
 constexpr int SM_Q = SM_V + KV_STAGES * TILE_BYTES;
@@ -79,7 +86,7 @@ constexpr int SM_CTRL = SM_SLO + HALF_BYTES;          // 229376
 constexpr int SM_CTRL_BYTES = 1024;
 constexpr int PREFILL_SMEM = SM_CTRL + SM_CTRL_BYTES + 1024;  // + alignment slack
 
-constexpr uint32_t TM_SC = 0, TM_O = 256, TM_S = 384, TM_COLS = 512;  // SC1 = TM_SC + 128
+constexpr uint32_t TM_SC = 0, TM_O = 128, TM_S = 384, TM_COLS = 512;  // O buffer 1 = TM_O + 128
 
 // device status codes (match la_status)
 constexpr int ST_INVALID = 1;
@@ -117,10 +124,10 @@ struct CtrlBlock {
     uint64_t kv_empty[KV_STAGES]; // [1] MMA commit after the last MMA reading the stage
     uint64_t q_full[Q_STAGES];    // [1] producer expect_tx
     uint64_t q_empty[Q_STAGES];   // [1] MMA commit after a5 of the block
-    uint64_t sc_full[2];          // [1] a2 done: scores in buffer b & 1
-    uint64_t p_full[2];           // [4] mask warps: P in buffer b & 1
-    uint64_t o_full;              // [1] a4 + a5 done
-    uint64_t o_empty;             // [4] store warps have O in registers
+    uint64_t sc_full;             // [1] a2 done: scores in the score buffer
+    uint64_t p_full;              // [4] mask warps: P written over the scores
+    uint64_t o_full[2];           // [1] a5 + a4 of a block done, O in buffer b & 1
+    uint64_t o_empty[2];          // [4] store warps have O buffer b & 1 in registers
     uint64_t s_done;              // [1] a6 done
     uint64_t snap_full;           // [4] state warps: snapshot of S in shared memory (S read)
     uint64_t snap_empty;          // [1] a5 has read the snapshot
@@ -321,13 +328,13 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             mbar_init(&cb->q_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&cb->sc_full[s], 1);
-            mbar_init(&cb->p_full[s], 4);
+            mbar_init(&cb->o_full[s], 1);
+            mbar_init(&cb->o_empty[s], 4);
             mbar_init(&cb->item_full[s], 1);
             mbar_init(&cb->item_empty[s], 14);
         }
-        mbar_init(&cb->o_full, 1);
-        mbar_init(&cb->o_empty, 4);
+        mbar_init(&cb->sc_full, 1);
+        mbar_init(&cb->p_full, 4);
         mbar_init(&cb->s_done, 1);
         mbar_init(&cb->snap_full, 4);
         mbar_init(&cb->snap_empty, 1);
@@ -488,7 +495,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             if (!last) {
                 // phase A: A_j = sum_b K_b^T V_b, accumulated in the O columns once
                 // the previous block's output has been read out
-                if (!warp_wait(&cb->o_empty, (blk_n & 1) ^ 1, p, cb)) break;
+                // (the O buffer of this item's first block; free once the block two
+                // before it has been read out)
+                if (!warp_wait(&cb->o_empty[blk_n & 1], ((blk_n >> 1) & 1) ^ 1, p, cb)) break;
                 tc_fence_after();
                 for (int b = 0; b < nblk; ++b) {
                     if (cb->abort) { ok = false; break; }
@@ -499,7 +508,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BLK / 16; ++kk)
-                        mma_ss_w(tmem + TM_O, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, (b > 0 || kk > 0) ? 1u : 0u);
+                        mma_ss_w(tmem + TM_O + (blk_n & 1) * 128, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
+                                 (b > 0 || kk > 0) ? 1u : 0u);
                     tc_commit_w(&cb->kv_empty[s]);
                     ++kv_n;
                 }
@@ -517,14 +527,14 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 // O chain, a4(i4): P ready, a5 of the block issued
                 if (i4 < i5) {
                     const uint32_t bn = blk0 + i4;
-                    if (ready(&cb->p_full[bn & 1], (bn >> 1) & 1)) {
+                    if (ready(&cb->p_full, bn & 1)) {
                         tc_fence_after();
                         const int s = (kv0 + i4) % KV_STAGES;
                         const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns
-                            mma_ts_w(tmem + TM_O, tmem + TM_SC + (bn & 1) * 128 + kk * 8, desc_mnmajor(vt, kk), ID_PV, 1u);
-                        tc_commit_w(&cb->o_full);
+                            mma_ts_w(tmem + TM_O + (bn & 1) * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV, 1u);
+                        tc_commit_w(&cb->o_full[bn & 1]);
                         tc_commit_w(&cb->kv_empty[s]);  // a2, a6 and a4 of this block are issued
                         ++i4;
                         prog = true;
@@ -538,7 +548,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 if (i5 < i2) {
                     const uint32_t bn = blk0 + i5;
                     const bool a_read = last || i5 > 0 || ready(&cb->a_free, afree_n & 1);
-                    if (a_read && ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty, (bn & 1) ^ 1)) {
+                    if (a_read && ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty[bn & 1], ((bn >> 1) & 1) ^ 1)) {
                         tc_fence_after();
                         const int s = (kv0 + i5) % KV_STAGES;
                         const uint32_t qn = q0 + i5;
@@ -549,9 +559,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         if (!lo) {  // O = Q S, S = the whole [128 x 128] snapshot
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss_w(tmem + TM_O, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, kk > 0 ? 1u : 0u);
+                                mma_ss_w(tmem + TM_O + (bn & 1) * 128, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF,
+                                         kk > 0 ? 1u : 0u);
                         } else {  // one 64-column half of O = Q (S_hi + S_lo)
-                            const uint32_t to = tmem + TM_O + half * 64;
+                            const uint32_t to = tmem + TM_O + (bn & 1) * 128 + half * 64;
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk)
                                 mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u);
@@ -581,7 +592,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
                 // intra chain, a2(i2): its score buffer free (a4 of block i2 - 2
                 // issued), tiles landed
-                if (i2 < nblk && i2 < i4 + 2) {
+                if (i2 < nblk && i2 <= i4) {
                     const int s = (kv0 + i2) % KV_STAGES;
                     const uint32_t kn = (kv0 + i2) / KV_STAGES, qn = q0 + i2;
                     if (ready(&cb->kv_full[s], kn & 1) && ready(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1)) {
@@ -605,9 +616,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)  // a2: Sc = Q K^T
-                            mma_ss_w(tmem + TM_SC + ((blk0 + i2) & 1) * 128, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
+                            mma_ss_w(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
                                      kk > 0 ? 1u : 0u);
-                        tc_commit_w(&cb->sc_full[(blk0 + i2) & 1]);
+                        tc_commit_w(&cb->sc_full);
                         ++i2;
                         prog = true;
                     }
@@ -658,8 +669,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             for (int b = 0; b < nblk; ++b) {
                 // P = bf16(Sc ⊙ M), inclusive mask, packed two per 32-bit column
                 // over the first 64 score columns
-                const uint32_t bn = blk_n + b, tsc = trow + TM_SC + (bn & 1) * 128;
-                if (!warp_wait(&cb->sc_full[bn & 1], (bn >> 1) & 1, p, cb)) { ok = false; break; }
+                const uint32_t bn = blk_n + b, tsc = trow + TM_SC;
+                if (!warp_wait(&cb->sc_full, bn & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -682,7 +693,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->p_full[bn & 1]);
+                if (lane == 0) mbar_arrive(&cb->p_full);
             }
             blk_n += nblk;
         }
@@ -716,7 +727,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 const uint32_t bn = blk_n + b;
                 const int row0 = tok0 + b * BLK;
                 const int valid = min(BLK, tok1 - row0);
-                if (!warp_wait(&cb->o_full, bn & 1, p, cb)) { ok = false; break; }
+                if (!warp_wait(&cb->o_full[bn & 1], (bn >> 1) & 1, p, cb)) { ok = false; break; }
+                const uint32_t tob = trow + TM_O + (bn & 1) * 128;  // this block's O buffer
                 tc_fence_after();
                 const size_t orow = ((size_t)(row0 + r) * H + h) * D;
                 if (!p.out_fp32) {
@@ -727,13 +739,13 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         uint32_t x[64];
-                        tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
+                        tmem_ld_cols<64>(tob + hf * 64, x);
 #pragma unroll
                         for (int c = 0; c < 32; ++c) w[hf * 32 + c] = bf16x2_round(x[2 * c], x[2 * c + 1]);
                     }
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&cb->o_empty);
+                    if (lane == 0) mbar_arrive(&cb->o_empty[bn & 1]);
                     if (r < valid) {
                         uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow);
                         if (p.out_al32) {
@@ -749,11 +761,11 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                     for (int hf = 0; hf < 2; ++hf) {
                         uint32_t x[64];
-                        tmem_ld_cols<64>(trow + TM_O + hf * 64, x);
+                        tmem_ld_cols<64>(tob + hf * 64, x);
                         if (hf == 1) {
                             tc_fence_before();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(&cb->o_empty);
+                            if (lane == 0) mbar_arrive(&cb->o_empty[bn & 1]);
                         }
                         if (r < valid) {
                             uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(p.out) + orow + hf * 64);
@@ -776,7 +788,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int q4 = warp & 3;
         const int r = q4 * 32 + lane;
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
-        uint32_t it = 0, snap_n = 0, upd_n = 0, agg_n = 0;
+        uint32_t it = 0, snap_n = 0, upd_n = 0, agg_n = 0, blk_n = 0;
         uint8_t *shi = smem + SM_SHI;
         uint8_t *slo = smem + SM_SLO;
         int item[8];
@@ -861,7 +873,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                     for (int qq = 0; qq < 2; ++qq) {
                         uint32_t a[32];
-                        tmem_ld_wait32(trow + TM_O + hf * 64 + qq * 32, a);
+                        tmem_ld_wait32(trow + TM_O + (blk_n & 1) * 128 + hf * 64 + qq * 32, a);  // A_j: first block's O buffer
 #pragma unroll
                         for (int c = 0; c < 8; ++c)
                             __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, hf * 16 + qq * 8 + c)),
@@ -918,6 +930,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                 }
             }
+            blk_n += nblk;
             if (!ok) break;
         }
     }
