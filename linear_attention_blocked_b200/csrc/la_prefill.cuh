@@ -6,7 +6,7 @@
 // and take items in ticket order from a device counter.  For an item
 //
 //   phase A (only if a later segment of the same sequence exists):
-//       local KV sum  A_j = sum_b K_b^T V_b    (tcgen05, fp32, in the O columns)
+//       local KV sum  A_j = sum_b K_b^T V_b    (tcgen05, fp32, in an O buffer)
 //   phase L (look-back, LASP+ "gather + global prefix" on SMs instead of ranks):
 //       E_j = state_in (j = 0)  or  INCL_{j-1} published by the item that
 //       owns segment j-1 (bounded spin on its flag);  INCL_j = E_j + A_j is
@@ -24,9 +24,10 @@
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
 //               loads Q
-//   warp 1      TMEM allocator + MMA issuer (lane 0 issues)
+//   warp 1      TMEM allocator + MMA issuer (the whole warp runs the schedule;
+//               elect.sync picks the lane that issues each MMA or commit)
 //   warps 2-5   causal mask (a3)
-//   warps 6-9   output store (a7) and publication of inclusive prefixes
+//   warps 6-9   output store (a7) and the flag that publishes INCL_j
 //   warps 10-13 segment hand-off (phase L), state snapshots for a5, final state
 // A warp may only touch the 32 TMEM lanes of its quarter (warp % 4), so each
 // group of four covers all 128 rows.  Every group has its own chain of TMEM
@@ -62,10 +63,9 @@ constexpr int PREFILL_THREADS = 448;
 constexpr int W_MASK = 2, W_STORE = 6, W_STATE = 10;  // first warp of each four-warp group
 
 // L2 prefetch distance of the Q tiles, in row blocks ahead of their
-// shared-memory loads (0 = off).  K and V of phase O come back from L2 after
-// phase A; Q is read from DRAM once, and its shared-memory slot only frees up
-// when a5 of the block two earlier has finished, so the prefetch hides part
-// of the DRAM latency of that load.
+// shared-memory loads.  Q is the one tile phase O reads from DRAM (K and V
+// come back from L2 after phase A); prefetching it two or four blocks ahead
+// measured slower, so the default is 0 (off).
 #ifndef LA_PREFETCH_Q
 #define LA_PREFETCH_Q 0
 #endif
@@ -131,8 +131,8 @@ struct CtrlBlock {
     uint64_t s_done;              // [1] a6 done
     uint64_t snap_full;           // [4] state warps: snapshot of S in shared memory (S read)
     uint64_t snap_empty;          // [1] a5 has read the snapshot
-    uint64_t agg_full;            // [1] phase A done: A_j in the O columns
-    uint64_t a_free;              // [4] state warps: A_j read, the O columns are free
+    uint64_t agg_full;            // [1] phase A done: A_j in the first block's O buffer
+    uint64_t a_free;              // [4] state warps: A_j read, that O buffer is free
     uint64_t incl_stored;         // [4] state warps: INCL_j written to the workspace
     uint64_t item_full[2];        // [1] producer
     uint64_t item_empty[2];       // [14] Q producer lane + MMA lane 0 + 3 x 4 warps
@@ -462,17 +462,16 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
     } else if (warp == 1) {
         // ===================== MMA issuer =====================
         // Phase O runs three dependency chains per block b:
-        //   intra chain:  a2(b) -> [mask] -> a4(b)              (needs Q, K, V tiles)
-        //   O chain:      a5(b) -> a4(b) -> [O read out] -> a5(b+1)
+        //   intra chain:  a4(b-1) -> a2(b) -> [mask] -> a4(b)   (needs Q, K, V tiles)
+        //   O chain:      a5(b) -> a4(b) -> [O_{b&1} read out] -> a5(b+2)
         //   state chain:  [snapshot S_{<b}] -> a5(b), a6(b) -> [snapshot S_{<b+1}]
         // a5(b) initialises the block's O buffer and a4(b) accumulates onto it,
         // so every accumulator receives its MMAs in a fixed order and the result
         // is deterministic.  a5 comes first so that the Q tile is released as
         // soon as possible (a2 and a5 are its only readers) and so that a6, the
         // state update, follows the snapshot without waiting for the mask.
-        // Instead of a fixed program order, the issuing lane polls the barriers
-        // and issues whatever is ready: a2 may run up to two blocks (the two
-        // score buffers) ahead of a4.
+        // Instead of a fixed program order, the warp polls the barriers and
+        // issues whatever is ready; a2(b) waits for a4(b-1) (see TM_O).
         constexpr uint32_t ID_QK = idesc_bf16_f32(BLK, BLK, 0, 0);    // Q (K-major) x K (K-major)
         constexpr uint32_t ID_QS = idesc_bf16_f32(BLK, D / 2, 0, 1);  // Q (K-major) x S half (MN-major)
         constexpr uint32_t ID_QF = idesc_bf16_f32(BLK, D, 0, 1);      // Q (K-major) x S (MN-major)
@@ -493,10 +492,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
             const bool lo = (item[IT_FLAGS] & ITF_LO) != 0;
             if (!last) {
-                // phase A: A_j = sum_b K_b^T V_b, accumulated in the O columns once
-                // the previous block's output has been read out
-                // (the O buffer of this item's first block; free once the block two
-                // before it has been read out)
+                // phase A: A_j = sum_b K_b^T V_b, accumulated in the O buffer of this
+                // item's first block once the block two before it has been read out
                 if (!warp_wait(&cb->o_empty[blk_n & 1], ((blk_n >> 1) & 1) ^ 1, p, cb)) break;
                 tc_fence_after();
                 for (int b = 0; b < nblk; ++b) {
@@ -542,9 +539,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
                 // state and O chains, a5(i5) (one full-width pass, or one half of
                 // the hi + lo pair) then a6(i5): Q landed (a2 issued), snapshot
-                // ready, the O buffer free (the previous block's O read out; for
-                // the first block of a segment with a successor, INCL read out of
-                // the O columns)
+                // ready, the block's O buffer free (block i5 - 2 read out; for the
+                // first block of a segment with a successor, A_j read out of it)
                 if (i5 < i2) {
                     const uint32_t bn = blk0 + i5;
                     const bool a_read = last || i5 > 0 || ready(&cb->a_free, afree_n & 1);
@@ -884,7 +880,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                 }
             }
-            if (!last) {  // A_j has been read: the O columns are free for a5 of the first block
+            if (!last) {  // A_j has been read: its O buffer is free for a5 of the first block
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cb->a_free);
