@@ -7,7 +7,9 @@ iid N(0,1)*128^-0.5, fp32 accumulation, bf16 output plus the final fp32
 (segment table + TMA staging + the four tcgen05 contractions + masking +
 cross-SM segment hand-off + epilogue).  In the same run the fused batched
 decode step is timed on its own workload (256 sequences x 64 heads, fp32
-states initialised by a 4096-token prefill) and reported under "decode".
+states initialised by a 4096-token prefill) and reported under "decode", and
+the local-prefix step of sequence parallelism (la_kv_aggregate) on the
+prefill's k and v under "kv_aggregate".
 
   python bench.py [--gpus N] [--steps K] [--warmup W]      # CUDA path
   python bench.py --impl reference ...                     # fp64 CPU oracle arm
@@ -63,6 +65,11 @@ def prefill_flops(tok_heads: int, block: int, frac_phase_a: float):
     return tok_heads * alg, tok_heads * exe
 
 
+def aggregate_bytes(tok_heads: int, pairs: int) -> int:
+    """Read k and v (bf16), write one fp32 d x d sum per (sequence, head)."""
+    return tok_heads * D * 2 * 2 + pairs * D * D * 4
+
+
 def decode_bytes(pairs: int) -> int:
     """Read + write the fp32 state, read q, k, v and write o (bf16)."""
     return pairs * (2 * D * D * 4 + 4 * D * 2)
@@ -81,6 +88,7 @@ def load_peaks():
 KERNEL_SOURCES = {
     "la_prefill_kernel": ("la_prefill.cuh", "la_ptx.cuh", "la_lib.cu"),
     "la_decode_kernel": ("la_decode.cuh", "la_lib.cu"),
+    "la_kv_aggregate_kernel": ("la_aggregate.cuh", "la_prefill.cuh", "la_ptx.cuh", "la_lib.cu"),
 }
 
 
@@ -341,6 +349,9 @@ def run_cuda(args, world, rank, local):
     if rank == 0 or world > 1:
         dec = bench_decode(la, dev, stream, args, hbm_peak, world)
 
+    # ---------------- local prefix of sequence parallelism on the same k, v
+    agg = bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world)
+
     status2 = la.get_device_status()
     if rank != 0:
         return 0
@@ -369,11 +380,40 @@ def run_cuda(args, world, rank, local):
         "gpu_launches": int(launches),
         "clocks": clocks,
         "decode": dec,
+        "kv_aggregate": agg,
         "cpu_baseline": cpu,
         "device_status": [int(status), int(status2)],
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world):
+    """la_kv_aggregate (local prefix of sequence parallelism: sum of k_t^T v_t
+    per head) over the prefill workload's k and v (1.07 GB, larger than L2)."""
+    agg = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(256, la.lib().la_kv_aggregate_workspace_size(B, N, H, D)), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        la.kv_aggregate(k, v, out=agg, workspace=ws)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(20, min(args.steps, 500))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        la.kv_aggregate(k, v, out=agg, workspace=ws)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    byts = aggregate_bytes(B * N * H, B * H)
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"workload": "kv_aggregate B=1 H=64 N=32768 d=128 (the prefill workload's k, v)",
+            "ms_per_call": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "kernel": "la_kv_aggregate_kernel",
+                         "traffic": recorded_traffic("la_kv_aggregate_kernel", "aggregate_B1_H64_N32768"),
+                         "bytes_per_launch": byts,
+                         "duration": "CUDA events around each la_kv_aggregate call (aggregate + reduce)"}}
 
 
 def bench_decode(la, dev, stream, args, hbm_peak, world):

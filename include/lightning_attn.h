@@ -204,6 +204,50 @@ LA_API la_status la_prefill_noalloc(const void *q, const void *k, const void *v,
                                     float *state_out, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Sequence parallelism across ranks ("MiniMax-01技术报告解读", §3.2 item 3,
+ * LASP+: each rank forms the local prefix of its part of the sequence, the
+ * local prefixes are all-gathered, and each rank adds up the global prefix
+ * of the ranks before it, then runs its own blocked scan from there).
+ * Rank r holds tokens [n_0 + ... + n_{r-1}, + n_r) of every sequence of the
+ * batch.  Per rank:
+ *
+ *   la_kv_aggregate(k_r, v_r) -> A_r           (local prefix, this library)
+ *   AllGather(A_r) -> A_0 ... A_{W-1}          (the caller's collective)
+ *   la_state_prefix(A, r, S_in) -> P_r         (global prefix, this library)
+ *   la_prefill(q_r, k_r, v_r, state_in = P_r)  (the local scan)
+ *
+ * and la_state_prefix(A, W, S_in) is the final state of the whole sequence.
+ * The rank's outputs equal the rows of the single-GPU result for its tokens.
+ *
+ * la_kv_aggregate: A[b][h][i][j] = sum_t k[b][t][h][i] * v[b][t][h][j] over
+ *   the N tokens of each sequence (the state increment S_out - S_in of a
+ *   prefill of those tokens).  k, v: bf16 [B, N, H, d] contiguous (read
+ *   only; may be NULL when N == 0).  agg: fp32 [B, H, d, d] row-major, fully
+ *   written (zeros when N == 0), must not overlap k, v or the workspace.
+ *   workspace: at least la_kv_aggregate_workspace_size(B, N, H, d) bytes
+ *   (at most 2 x 148 x 64 KiB), 16-byte aligned, caller-owned scratch whose
+ *   contents before and after the call do not matter; may be NULL when the
+ *   size is 0.  fp32 accumulation on the tensor cores, summed in a fixed
+ *   order (the result does not depend on timing).  Asynchronous on `stream`;
+ *   argument errors are returned before any launch; a device-side wait that
+ *   ran out is reported by la_get_device_status.
+ * la_state_prefix: out = (state_in or 0) + parts[0] + ... + parts[count-1],
+ *   elementwise in that order, in fp32.  parts: fp32 [count][nstates][d][d]
+ *   contiguous (NULL when count == 0); state_in: fp32 [nstates][d][d] or
+ *   NULL; out: fp32 [nstates][d][d], may equal state_in, must not overlap
+ *   parts or partially overlap state_in.  nstates = B * H.  Asynchronous on
+ *   `stream`.
+ * ------------------------------------------------------------------------- */
+LA_API size_t la_kv_aggregate_workspace_size(int B, int N, int H, int d);
+
+LA_API la_status la_kv_aggregate(const void *k, const void *v, int B, int N, int H, int d,
+                                 float *agg, void *workspace, size_t ws_bytes,
+                                 cudaStream_t stream);
+
+LA_API la_status la_state_prefix(const float *parts, int count, const float *state_in,
+                                 float *out, int nstates, int d, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status.
  * la_get_device_status synchronises `stream`, then returns and clears the
  * sticky device word of the current device (LA_ERR_TIMEOUT,

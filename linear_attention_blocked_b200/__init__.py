@@ -11,14 +11,18 @@ ABI (include/lightning_attn.h).  Entry points:
   mixed_step(q, k, v, cu_seqlens, ...)       la_mixed_step: prefill chunks and decode tokens
                                              of one batch on two streams (plan with
                                              serving.plan_batch)
+  kv_aggregate(k, v)                         la_kv_aggregate: sum_t k_t^T v_t per (sequence, head)
+  state_prefix(parts, count, state_in)       la_state_prefix: state_in + parts[0] + ... + parts[count-1]
+  lasp_prefill(q, k, v, group=...)           sequence parallelism across ranks (seqpar.py)
   get_device_status()                        la_get_device_status
 """
 from ._binding import (D, DEFAULT_BLOCK, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
                        LA_ERR_INVALID_ARGUMENT, LA_ERR_TIMEOUT, LA_ERR_UNSUPPORTED,
                        LA_ERR_WORKSPACE, LA_FP32, LA_INJECT_NONE, LA_INJECT_SKIP_PUBLISH, LA_OK,
                        LAError, debug_inject, decode_step, decode_step_slots, get_device_status,
-                       kernel_launches, last_segment_len, lib, library_path, mixed_step, prefill,
-                       prefill_varlen, prefill_varlen_slots,
-                       set_segment_len, set_wait_limit_ns, status_string, varlen_workspace_size,
-                       workspace_size)
+                       kernel_launches, kv_aggregate, last_segment_len, lib, library_path, mixed_step,
+                       prefill, prefill_varlen, prefill_varlen_slots,
+                       set_segment_len, set_wait_limit_ns, state_prefix, status_string,
+                       varlen_workspace_size, workspace_size)
+from .seqpar import lasp_prefill  # noqa: F401,E402
 from .serving import BatchPlan, plan_batch  # noqa: F401,E402

@@ -24,7 +24,8 @@ EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_worksp
             "la_prefill_varlen", "la_decode_step", "la_get_device_status", "la_status_string",
             "la_set_wait_limit_ns", "la_set_segment_len", "la_debug_inject",
             "la_last_segment_len", "la_kernel_launches", "la_prefill_noalloc",
-            "la_prefill_varlen_slots", "la_decode_step_slots", "la_mixed_step")
+            "la_prefill_varlen_slots", "la_decode_step_slots", "la_mixed_step",
+            "la_kv_aggregate_workspace_size", "la_kv_aggregate", "la_state_prefix")
 
 
 class LAError(RuntimeError):
@@ -73,6 +74,12 @@ def lib():
         L.la_mixed_step.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, vp, c_int, c_int, c_int, vp, c_int,
                                     vp, c_int, vp, sz, vp, vp]
         L.la_mixed_step.restype = c_int
+        L.la_kv_aggregate_workspace_size.argtypes = [c_int] * 4
+        L.la_kv_aggregate_workspace_size.restype = sz
+        L.la_kv_aggregate.argtypes = [vp, vp, c_int, c_int, c_int, c_int, vp, vp, sz, vp]
+        L.la_kv_aggregate.restype = c_int
+        L.la_state_prefix.argtypes = [vp, c_int, vp, vp, c_int, c_int, vp]
+        L.la_state_prefix.restype = c_int
         L.la_get_device_status.argtypes = [vp]
         L.la_get_device_status.restype = c_int
         L.la_status_string.argtypes = [c_int]
@@ -309,6 +316,53 @@ def mixed_step(q, k, v, cu_seqlens, prefill_slots, max_seqlen: int, decode_slots
                              workspace.numel() * workspace.element_size(), _stream_handle(prefill_stream),
                              _stream_handle(decode_stream))
     _check(st, "la_mixed_step")
+    return out
+
+
+def kv_aggregate(k, v, out=None, workspace=None, stream=None):
+    """la_kv_aggregate on [B, N, H, d] bf16 k, v: returns fp32 [B, H, d, d]
+    with A[b, h] = sum over the N tokens of k_t^T v_t."""
+    if k.dim() != 4:
+        raise ValueError("k must be [B, N, H, d]")
+    B, N, H, d = k.shape
+    _need(k, "k", torch.bfloat16, (B, N, H, d))
+    _need(v, "v", torch.bfloat16, (B, N, H, d))
+    if out is None:
+        out = torch.empty((B, H, d, d), dtype=torch.float32, device=k.device)
+    _need(out, "out", torch.float32, (B, H, d, d))
+    ws_bytes = int(lib().la_kv_aggregate_workspace_size(B, N, H, d))
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, k.device)
+    st = lib().la_kv_aggregate(_ptr(k), _ptr(v), B, N, H, d, _ptr(out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "la_kv_aggregate")
+    return out
+
+
+def state_prefix(parts, count: int, state_in=None, out=None, stream=None):
+    """la_state_prefix: (state_in or 0) + parts[0] + ... + parts[count-1].
+    parts: fp32 [W, ...states..., d, d] (W >= count); returns fp32 states of
+    the shape of parts[0]."""
+    if parts.dim() < 3:
+        raise ValueError("parts must be [W, ..., d, d]")
+    shape = tuple(parts.shape[1:])
+    d = shape[-1]
+    _need(parts, "parts", torch.float32, (parts.shape[0],) + shape)
+    if shape[-2] != d:
+        raise ValueError("states must be square")
+    if not 0 <= count <= parts.shape[0]:
+        raise ValueError("count must lie in [0, W]")
+    nstates = 1
+    for x in shape[:-2]:
+        nstates *= int(x)
+    if state_in is not None:
+        _need(state_in, "state_in", torch.float32, shape)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.float32, device=parts.device)
+    _need(out, "out", torch.float32, shape)
+    st = lib().la_state_prefix(_ptr(parts), int(count), _ptr(state_in), _ptr(out), nstates, d,
+                               _stream_handle(stream))
+    _check(st, "la_state_prefix")
     return out
 
 

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "lightning_attn.h"
+#include "la_aggregate.cuh"
 #include "la_decode.cuh"
 #include "la_prefill.cuh"
 
@@ -259,6 +260,27 @@ la_status decode_impl(const void *q, const void *k, const void *v, float *state,
     return LA_OK;
 }
 
+// Cut the block list of la_kv_aggregate into equal ranges, one per CTA.
+// Depends on the shape only, so the workspace size is a pure function of it.
+struct AggPlan {
+    long long total = 0, per_cta = 1;
+    int ctas = 0;
+    int nblk = 0;
+};
+
+AggPlan agg_plan(long long npairs, int N) {
+    AggPlan a;
+    a.nblk = (int)(((long long)N + la::BLK - 1) / la::BLK);
+    a.total = npairs * a.nblk;
+    if (a.total == 0) return a;
+    const long long c = a.total < la::AGG_CTAS ? a.total : la::AGG_CTAS;
+    a.per_cta = (a.total + c - 1) / c;
+    a.ctas = (int)((a.total + a.per_cta - 1) / a.per_cta);
+    return a;
+}
+
+size_t agg_ws_bytes(const AggPlan &a) { return (size_t)2 * a.ctas * la::D * la::D * sizeof(float); }
+
 }  // namespace
 
 extern "C" {
@@ -416,6 +438,88 @@ la_status la_debug_inject(int mode) {
 int la_last_segment_len(void) { return g_last_seg_len.load(); }
 
 unsigned long long la_kernel_launches(void) { return g_launches.load(); }
+
+size_t la_kv_aggregate_workspace_size(int B, int N, int H, int d) {
+    (void)d;
+    if (B <= 0 || N <= 0 || H <= 0) return 0;
+    return agg_ws_bytes(agg_plan((long long)B * H, N));
+}
+
+la_status la_kv_aggregate(const void *k, const void *v, int B, int N, int H, int d, float *agg, void *workspace,
+                          size_t ws_bytes, cudaStream_t stream) {
+    la_status st = check_common(H, d, 0, LA_FP32);
+    if (st != LA_OK) return st;
+    if (B < 0 || N < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (B == 0) return LA_OK;
+    const long long T = (long long)B * N;
+    if (T > 0x7fffffffLL || (long long)B * H > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    if (!agg || !aligned(agg, 16)) return LA_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return LA_ERR_INVALID_ARGUMENT;
+    const size_t n_in = (size_t)T * H * la::D * 2, n_agg = (size_t)B * H * la::D * la::D * 4;
+    if (ranges_overlap(agg, n_agg, k, n_in) || ranges_overlap(agg, n_agg, v, n_in)) return LA_ERR_INVALID_ARGUMENT;
+    const AggPlan a = agg_plan((long long)B * H, N);
+    const size_t need = agg_ws_bytes(a);
+    if (need > 0) {
+        if (!workspace || ws_bytes < need) return LA_ERR_WORKSPACE;
+        if (!aligned(workspace, 16)) return LA_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(workspace, need, agg, n_agg)) return LA_ERR_INVALID_ARGUMENT;
+    }
+    int *status = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void **>(&status), g_la_status) != cudaSuccess) return LA_ERR_CUDA;
+    if (a.ctas > 0) {
+        CUtensorMap mk, mv;
+        if (!encode_qkv_map(&mk, k, (int)T, H) || !encode_qkv_map(&mv, v, (int)T, H)) return LA_ERR_CUDA;
+        la::AggParams p;
+        p.out = agg;
+        p.partial = static_cast<float *>(workspace);
+        p.N = N;
+        p.H = H;
+        p.nblk = a.nblk;
+        p.total = a.total;
+        p.per_cta = a.per_cta;
+        p.wait_limit_ns = g_wait_limit_ns.load();
+        p.status = status;
+        static std::once_flag attr_once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(attr_once, [] {
+            attr_err = cudaFuncSetAttribute(la::la_kv_aggregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            la::AGG_SMEM);
+        });
+        if (attr_err != cudaSuccess) return LA_ERR_CUDA;
+        la::la_kv_aggregate_kernel<<<a.ctas, la::AGG_THREADS, la::AGG_SMEM, stream>>>(mk, mv, p);
+        if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+        ++g_launches;
+    }
+    // sums of the pairs that range boundaries cut (zeros when N == 0)
+    la::la_agg_reduce_kernel<<<dim3((unsigned)((long long)B * H), la::AGG_RED_SLICES), la::AGG_RED_THREADS, 0,
+                               stream>>>(agg, static_cast<const float *>(workspace), a.nblk, a.per_cta);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
+
+la_status la_state_prefix(const float *parts, int count, const float *state_in, float *out, int nstates, int d,
+                          cudaStream_t stream) {
+    if (d <= 0 || nstates < 0 || count < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (d != la::D) return LA_ERR_UNSUPPORTED;
+    if (nstates == 0) return LA_OK;
+    if (!out || !aligned(out, 16)) return LA_ERR_INVALID_ARGUMENT;
+    if (count > 0 && (!parts || !aligned(parts, 16))) return LA_ERR_INVALID_ARGUMENT;
+    if (state_in && !aligned(state_in, 16)) return LA_ERR_INVALID_ARGUMENT;
+    const size_t n = (size_t)nstates * la::D * la::D * 4;
+    if (ranges_overlap(out, n, parts, (size_t)count * n)) return LA_ERR_INVALID_ARGUMENT;
+    if (state_in && state_in != out && ranges_overlap(out, n, state_in, n)) return LA_ERR_INVALID_ARGUMENT;
+    const long long n4 = (long long)nstates * (la::D * la::D / 4);
+    long long blocks = (n4 + la::PREFIX_THREADS - 1) / la::PREFIX_THREADS;
+    const long long cap = (long long)device_sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    la::la_state_prefix_kernel<<<(unsigned)blocks, la::PREFIX_THREADS, 0, stream>>>(
+        reinterpret_cast<const float4 *>(parts), count, reinterpret_cast<const float4 *>(state_in),
+        reinterpret_cast<float4 *>(out), n4);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
 
 }  // extern "C"
 

@@ -159,3 +159,29 @@ def test_slot_and_mixed_argument_errors(L):
     assert call(args(ds=None)) == bad
     assert call(args(pool=None)) == bad
     assert call(args(d=64)) == la.LA_ERR_UNSUPPORTED
+
+
+def test_sequence_parallel_argument_errors(L):
+    """la_kv_aggregate and la_state_prefix reject bad arguments before launching."""
+    V = ctypes.c_void_p
+    fake = V(1 << 20)
+    bad = la.LA_ERR_INVALID_ARGUMENT
+    ws = L.la_kv_aggregate_workspace_size(1, 32768, 64, 128)
+    assert ws == 2 * 148 * 128 * 128 * 4             # two partial slots per CTA range
+    assert L.la_kv_aggregate_workspace_size(2, 0, 4, 128) == 0
+    assert L.la_kv_aggregate_workspace_size(1, 384, 100, 128) == 2 * 100 * 128 * 128 * 4
+    assert L.la_kv_aggregate(fake, fake, 1, 100, 2, 64, fake, fake, ws, None) == la.LA_ERR_UNSUPPORTED
+    assert L.la_kv_aggregate(fake, fake, -1, 100, 2, 128, fake, fake, ws, None) == bad
+    assert L.la_kv_aggregate(fake, fake, 1, 100, 2, 128, None, fake, ws, None) == bad          # no output
+    assert L.la_kv_aggregate(None, fake, 1, 100, 2, 128, fake, fake, ws, None) == bad          # no k
+    assert L.la_kv_aggregate(fake, fake, 1, 100, 2, 128, V((1 << 20) + 8), fake, ws, None) == bad  # misaligned
+    assert L.la_kv_aggregate(fake, fake, 1, 100, 2, 128, V(1 << 30), None, 0, None) == la.LA_ERR_WORKSPACE
+    assert L.la_kv_aggregate(fake, fake, 1, 100, 2, 128, fake, V(1 << 30), ws, None) == bad   # output inside k
+    assert L.la_kv_aggregate(fake, fake, 0, 100, 2, 128, fake, None, 0, None) == la.LA_OK    # nothing to do
+    assert L.la_state_prefix(fake, 1, None, fake, 4, 64, None) == la.LA_ERR_UNSUPPORTED
+    assert L.la_state_prefix(fake, -1, None, fake, 4, 128, None) == bad
+    assert L.la_state_prefix(None, 2, None, fake, 4, 128, None) == bad                        # no parts
+    assert L.la_state_prefix(fake, 2, None, fake, 4, 128, None) == bad                        # out inside parts
+    assert L.la_state_prefix(fake, 2, None, V((1 << 30) + 4), 4, 128, None) == bad            # misaligned
+    assert L.la_state_prefix(fake, 2, V((1 << 30) + 1024), V(1 << 30), 4, 128, None) == bad   # partial overlap
+    assert L.la_state_prefix(fake, 2, None, fake, 0, 128, None) == la.LA_OK

@@ -1,0 +1,158 @@
+"""GPU parity of the sequence-parallel steps (LASP+ across ranks) against the
+fp64 oracle: the local prefix la_kv_aggregate equals the oracle's final state
+from a zero state; the global prefix la_state_prefix is the ordered fp32 sum
+it is defined as; and ranks emulated one after another on one GPU (local
+prefix, gather, global prefix, local scan) reproduce the oracle's result for
+the whole sequences.  One more test runs lasp_prefill itself under a one-rank
+NCCL process group."""
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+
+import la_inputs
+import linear_attention_blocked_b200 as la
+from parity_util import check_out, check_state, to_np
+
+pytestmark = pytest.mark.gpu
+
+D = 128
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _cu(B, N):
+    return (np.arange(B + 1) * N).astype(np.int32)
+
+
+def _oracle_state(oracle_mod, k, v, heads=None):
+    """Final state from a zero state over each sequence of [B, N, H, D] k, v."""
+    B, N, H, _ = k.shape
+    K = la_inputs.bits(k.reshape(B * N, H, D))
+    V = la_inputs.bits(v.reshape(B * N, H, D))
+    _, st = oracle_mod.recurrent(K, K, V, _cu(B, N), heads=heads)
+    return st
+
+
+# (B, N, H): every pair cut into one-block pieces; pairs cut at ragged points;
+# one whole pair per CTA; ragged tails inside and at the end of the batch;
+# single tokens; more pairs than CTAs.
+@pytest.mark.parametrize("B,N,H", [(1, 1000, 3), (2, 129, 5), (1, 384, 100), (1, 640, 64), (3, 1, 2),
+                                   (2, 300, 7), (4, 2050, 40)])
+def test_kv_aggregate_matches_oracle(oracle_mod, B, N, H):
+    _, k, v = la_inputs.qkv((B, N, H, D), seed=500 + N + H, device="cuda")
+    agg = la.kv_aggregate(k, v)
+    assert la.get_device_status() == la.LA_OK
+    check_state(to_np(agg), _oracle_state(oracle_mod, k, v), what=f"A for B={B} N={N} H={H}")
+
+
+def test_kv_aggregate_full_size_sampled_heads(oracle_mod):
+    """B=1, N=32768, H=64 (the single-sequence prefill workload), three heads
+    checked against the oracle, every head against la_prefill's final state."""
+    B, N, H = 1, 32768, 64
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=42, device="cuda")
+    agg = la.kv_aggregate(k, v)
+    _, st = la.prefill(q, k, v)
+    assert la.get_device_status() == la.LA_OK
+    heads = [0, 17, 63]
+    check_state(to_np(agg[:, heads]), _oracle_state(oracle_mod, k, v, heads=heads), what="sampled heads")
+    check_state(to_np(agg), to_np(st), what="A vs prefill final state (all heads)")
+
+
+def test_kv_aggregate_empty_and_deterministic():
+    B, H = 2, 3
+    k = torch.empty((B, 0, H, D), dtype=torch.bfloat16, device="cuda")
+    agg = la.kv_aggregate(k, k.clone())
+    assert torch.count_nonzero(agg) == 0
+    _, k, v = la_inputs.qkv((B, 777, H, D), seed=9, device="cuda")
+    a1 = la.kv_aggregate(k, v)
+    a2 = la.kv_aggregate(k, v)
+    assert torch.equal(a1, a2)
+    assert la.get_device_status() == la.LA_OK
+
+
+@pytest.mark.parametrize("count", [0, 1, 3, 4])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_state_prefix_is_the_ordered_fp32_sum(count, with_state):
+    W, B, H = 4, 2, 3
+    gen = torch.Generator(device="cuda").manual_seed(11 + count)
+    parts = torch.randn((W, B, H, D, D), generator=gen, device="cuda")
+    sin = torch.randn((B, H, D, D), generator=gen, device="cuda") if with_state else None
+    out = la.state_prefix(parts, count, sin)
+    # the same additions in the same order in fp32 on the host: bit-exact
+    ref = to_np(sin).astype(np.float32) if with_state else np.zeros((B, H, D, D), np.float32)
+    p = parts.cpu().numpy()
+    for i in range(count):
+        ref = (ref + p[i]).astype(np.float32)
+    assert np.array_equal(out.cpu().numpy(), ref)
+    if with_state:  # in place
+        la.state_prefix(parts, count, sin, out=sin)
+        assert np.array_equal(sin.cpu().numpy(), ref)
+
+
+def test_emulated_ranks_reproduce_the_whole_sequence(oracle_mod):
+    """Three ranks with parts of 700, 1500 and 829 tokens, run one after the
+    other on this GPU: local prefixes, their stack standing in for the
+    AllGather, global prefixes, local scans seeded with them."""
+    B, H = 2, 4
+    lens = [700, 1500, 829]
+    N = sum(lens)
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=321, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(322)
+    sin = torch.randn((B, H, D, D), generator=gen, device="cuda") * 0.1
+    bounds = np.concatenate([[0], np.cumsum(lens)])
+    shard = lambda t, r: t[:, bounds[r]:bounds[r + 1]].contiguous()
+    parts = torch.stack([la.kv_aggregate(shard(k, r), shard(v, r)) for r in range(len(lens))])
+    outs = []
+    for r in range(len(lens)):
+        prefix = la.state_prefix(parts, r, sin)
+        o, _ = la.prefill(shard(q, r), shard(k, r), shard(v, r), state_in=prefix, out_dtype=torch.float32,
+                          want_state=False)
+        outs.append(o)
+    final = la.state_prefix(parts, len(lens), sin)
+    assert la.get_device_status() == la.LA_OK
+    Q, K, V = (la_inputs.bits(t.reshape(B * N, H, D)) for t in (q, k, v))
+    ref, rst = oracle_mod.recurrent(Q, K, V, _cu(B, N), state_in=to_np(sin))
+    got = torch.cat(outs, dim=1).reshape(B * N, H, D)
+    check_out(to_np(got), ref, bf16_out=False, what="rank outputs")
+    check_state(to_np(final), rst, what="final state")
+
+
+_ONE_RANK = r"""
+import os, sys
+sys.path.insert(0, os.environ["LA_ROOT"])
+import torch, torch.distributed as dist
+import la_inputs
+import linear_attention_blocked_b200 as la
+torch.cuda.set_device(0)
+dist.init_process_group("nccl", init_method="tcp://127.0.0.1:" + os.environ["LA_PORT"], rank=0, world_size=1)
+B, N, H, D = 2, 1000, 8, 128
+q, k, v = la_inputs.qkv((B, N, H, D), seed=77, device="cuda")
+sin = torch.randn((B, H, D, D), device="cuda") * 0.1
+out, final = la.lasp_prefill(q, k, v, state_in=sin)
+ref, st = la.prefill(q, k, v, state_in=sin)
+torch.cuda.synchronize()
+same = torch.equal(out, ref)
+rel = float((final - st).norm() / st.norm())
+dist.destroy_process_group()
+print("RESULT", int(same), rel, la.get_device_status())
+"""
+
+
+def test_lasp_prefill_under_one_rank_nccl_group():
+    """With one rank the global prefix is the carried-in state itself, so the
+    output must equal la_prefill's bit for bit; the final state differs from
+    la_prefill's only in summation order."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    env = dict(os.environ, LA_ROOT=ROOT, LA_PORT=str(port), NCCL_NVLS_ENABLE="0")
+    res = subprocess.run([sys.executable, "-c", _ONE_RANK], env=env, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    line = [x for x in res.stdout.splitlines() if x.startswith("RESULT")][-1].split()
+    assert line[1] == "1", "output differs from la_prefill"
+    assert float(line[2]) <= 1e-5
+    assert int(line[3]) == la.LA_OK

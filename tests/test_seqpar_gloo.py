@@ -1,0 +1,98 @@
+"""Sequence parallelism across ranks (LASP+) on CPU ranks (gloo, world sizes
+2 and 3): lasp_prefill's exchange -- local prefixes all-gathered in rank
+order, the global prefix of the ranks before this one, the local scan seeded
+with it -- reproduces the oracle's result for the whole sequences.  The
+device steps are host stand-ins built from the oracle (fp64), so what is
+checked here is the rank logic; the CUDA steps are checked on the GPU."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import la_inputs
+
+D = 8  # small head dimension: the oracle takes any d
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class _HostOps:
+    """The three device steps of a rank, computed by the oracle in fp64."""
+
+    @staticmethod
+    def _packed(t):
+        B, n, H, d = t.shape
+        return la_inputs.bits(t.reshape(B * n, H, d)), (np.arange(B + 1) * n).astype(np.int32)
+
+    @staticmethod
+    def kv_aggregate(k, v):
+        import oracle
+        K, cu = _HostOps._packed(k)
+        V, _ = _HostOps._packed(v)
+        _, st = oracle.recurrent(K, K, V, cu)  # final state from zero = sum of k_t^T v_t
+        return torch.from_numpy(st)
+
+    @staticmethod
+    def state_prefix(parts, count, state_in):
+        acc = torch.zeros(parts.shape[1:], dtype=torch.float64) if state_in is None else state_in.clone()
+        for i in range(count):
+            acc += parts[i]
+        return acc
+
+    @staticmethod
+    def prefill(q, k, v, state_in, out_dtype):
+        import oracle
+        B, n, H, d = q.shape
+        Q, cu = _HostOps._packed(q)
+        K, _ = _HostOps._packed(k)
+        V, _ = _HostOps._packed(v)
+        out, _ = oracle.recurrent(Q, K, V, cu, state_in=state_in.numpy())
+        return torch.from_numpy(out).reshape(B, n, H, d)
+
+
+def _worker(rank, world, port, lens, result_path):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from linear_attention_blocked_b200 import seqpar
+        B, H = 2, 3
+        N = sum(lens)
+        q, k, v = la_inputs.qkv((B, N, H, D), seed=61, scale=0.5)
+        sin = torch.from_numpy(np.random.default_rng(62).standard_normal((B, H, D, D)) * 0.3)
+        a = sum(lens[:rank])
+        part = lambda t: t[:, a:a + lens[rank]].contiguous()
+        out, final = seqpar.lasp_prefill(part(q), part(k), part(v), state_in=sin, ops=_HostOps)
+        shares = [None] * world
+        dist.all_gather_object(shares, (out.numpy(), final.numpy()))
+        if rank == 0:
+            Q, cu = _HostOps._packed(q)
+            K, _ = _HostOps._packed(k)
+            V, _ = _HostOps._packed(v)
+            ref, rst = oracle.recurrent(Q, K, V, cu, state_in=sin.numpy())
+            ref = ref.reshape(B, N, H, D)
+            got = np.concatenate([o for o, _ in shares], axis=1)
+            scale = np.abs(ref).max()
+            ok = got.shape == ref.shape and np.abs(got - ref).max() <= 1e-10 * scale
+            for _, f in shares:
+                ok &= np.abs(f - rst).max() <= 1e-10 * np.abs(rst).max()
+            with open(result_path, "w") as fh:
+                fh.write("ok" if ok else f"mismatch {np.abs(got - ref).max()}")
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lens", [[40, 77], [130, 1, 59]])
+def test_ranks_reproduce_the_whole_sequence(tmp_path, oracle_mod, lens):
+    result = tmp_path / "result.txt"
+    mp.start_processes(_worker, args=(len(lens), _free_port(), lens, str(result)), nprocs=len(lens), join=True,
+                       start_method="spawn")
+    assert result.read_text() == "ok"
