@@ -14,6 +14,7 @@ ABI (include/lightning_attn.h).  Entry points:
   kv_aggregate(k, v)                         la_kv_aggregate: sum_t k_t^T v_t per (sequence, head)
   state_prefix(parts, count, state_in)       la_state_prefix: state_in + parts[0] + ... + parts[count-1]
   lasp_prefill(q, k, v, group=...)           sequence parallelism across ranks (seqpar.py)
+  lasp_prefill_varlen(q, k, v, cu, bounds)   the same for a packed batch cut at any token
   get_device_status()                        la_get_device_status
 """
 from ._binding import (D, DEFAULT_BLOCK, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
@@ -24,5 +25,5 @@ from ._binding import (D, DEFAULT_BLOCK, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa
                        prefill, prefill_varlen, prefill_varlen_slots,
                        set_segment_len, set_wait_limit_ns, state_prefix, status_string,
                        varlen_workspace_size, workspace_size)
-from .seqpar import lasp_prefill  # noqa: F401,E402
+from .seqpar import lasp_prefill, lasp_prefill_varlen, plan_varlen_rank, split_tokens  # noqa: F401,E402
 from .serving import BatchPlan, plan_batch  # noqa: F401,E402

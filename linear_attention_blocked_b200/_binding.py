@@ -341,27 +341,38 @@ def kv_aggregate(k, v, out=None, workspace=None, stream=None):
 
 def state_prefix(parts, count: int, state_in=None, out=None, stream=None):
     """la_state_prefix: (state_in or 0) + parts[0] + ... + parts[count-1].
-    parts: fp32 [W, ...states..., d, d] (W >= count); returns fp32 states of
-    the shape of parts[0]."""
-    if parts.dim() < 3:
-        raise ValueError("parts must be [W, ..., d, d]")
-    shape = tuple(parts.shape[1:])
-    d = shape[-1]
-    _need(parts, "parts", torch.float32, (parts.shape[0],) + shape)
-    if shape[-2] != d:
+    parts: fp32 [W, ...states..., d, d] with W >= count, or None when count is
+    0 (then the call copies state_in into out, or zeroes out).  Returns fp32
+    states of the shape of one part (or of state_in / out)."""
+    if parts is not None:
+        if parts.dim() < 3:
+            raise ValueError("parts must be [W, ..., d, d]")
+        shape = tuple(parts.shape[1:])
+        _need(parts, "parts", torch.float32, (parts.shape[0],) + shape)
+        if not 0 <= count <= parts.shape[0]:
+            raise ValueError("count must lie in [0, W]")
+        device = parts.device
+    else:
+        if count != 0:
+            raise ValueError("count must be 0 without parts")
+        ref = state_in if state_in is not None else out
+        if ref is None:
+            raise ValueError("need parts, state_in or out to know the shape")
+        shape = tuple(ref.shape)
+        device = ref.device
+    if len(shape) < 2 or shape[-1] != shape[-2]:
         raise ValueError("states must be square")
-    if not 0 <= count <= parts.shape[0]:
-        raise ValueError("count must lie in [0, W]")
+    d = shape[-1]
     nstates = 1
     for x in shape[:-2]:
         nstates *= int(x)
     if state_in is not None:
         _need(state_in, "state_in", torch.float32, shape)
     if out is None:
-        out = torch.empty(shape, dtype=torch.float32, device=parts.device)
+        out = torch.empty(shape, dtype=torch.float32, device=device)
     _need(out, "out", torch.float32, shape)
-    st = lib().la_state_prefix(_ptr(parts), int(count), _ptr(state_in), _ptr(out), nstates, d,
-                               _stream_handle(stream))
+    st = lib().la_state_prefix(_ptr(parts) if count > 0 else None, int(count), _ptr(state_in), _ptr(out),
+                               nstates, d, _stream_handle(stream))
     _check(st, "la_state_prefix")
     return out
 

@@ -13,11 +13,25 @@ of the batch as [B, n_r, H, 128] tensors; the parts may differ in length.  The
 rank's output equals the rows of the single-GPU prefill of the whole sequences
 for its tokens, and every rank returns the final state of the whole sequences.
 
+Packed variable-length batches (lasp_prefill_varlen): the packed token axis
+is cut into contiguous rank ranges at arbitrary points, so a sequence may
+start on one rank and end several ranks later.  Each rank forms the local
+prefix of the one sequence that is still open at the end of its range, the
+local prefixes are all-gathered, and the sequence carried into the rank's
+range starts from its carried-in state plus the local prefixes of the ranks
+it spanned before; every other sequence of the range starts from its own
+carried-in state.  The planning is plain host arithmetic on cu_seqlens
+(plan_varlen_rank); the device steps are la_kv_aggregate, la_state_prefix
+and la_prefill_varlen.
+
 The device steps run in the CUDA library (la_kv_aggregate, la_state_prefix,
-la_prefill); the collective is torch.distributed's.
+la_prefill, la_prefill_varlen); the collective is torch.distributed's.
 """
 from __future__ import annotations
 
+from dataclasses import dataclass
+
+import numpy as np
 import torch
 import torch.distributed as dist
 
@@ -25,20 +39,25 @@ from . import _binding
 
 
 class DeviceOps:
-    """The three device steps of one rank, as this library's CUDA entry points."""
+    """The device steps of one rank, as this library's CUDA entry points."""
 
     @staticmethod
     def kv_aggregate(k, v):
         return _binding.kv_aggregate(k, v)
 
     @staticmethod
-    def state_prefix(parts, count, state_in):
-        return _binding.state_prefix(parts, count, state_in)
+    def state_prefix(parts, count, state_in, out=None):
+        return _binding.state_prefix(parts, count, state_in, out=out)
 
     @staticmethod
     def prefill(q, k, v, state_in, out_dtype):
         out, _ = _binding.prefill(q, k, v, state_in=state_in, out_dtype=out_dtype, want_state=False)
         return out
+
+    @staticmethod
+    def prefill_varlen(q, k, v, cu_seqlens, max_seqlen, state_in, out_dtype):
+        cu = torch.from_numpy(np.ascontiguousarray(cu_seqlens, dtype=np.int32)).to(q.device)
+        return _binding.prefill_varlen(q, k, v, cu, max_seqlen, state_in=state_in, out_dtype=out_dtype)
 
 
 def lasp_prefill(q, k, v, group=None, state_in=None, out_dtype=torch.bfloat16, want_state: bool = True,
@@ -66,3 +85,134 @@ def lasp_prefill(q, k, v, group=None, state_in=None, out_dtype=torch.bfloat16, w
     out = ops.prefill(q, k, v, prefix, out_dtype)
     final = ops.state_prefix(parts, world, state_in) if want_state else None
     return out, final
+
+
+# --------------------------------------------------------------------------- packed batches
+def split_tokens(total_tokens: int, world: int) -> np.ndarray:
+    """Rank boundaries [world + 1] cutting the packed token axis into ranges
+    whose lengths differ by at most one token."""
+    return (np.arange(world + 1, dtype=np.int64) * int(total_tokens)) // int(world)
+
+
+@dataclass
+class VarlenRankPlan:
+    rank: int
+    tok0: int                 # this rank holds packed tokens [tok0, tok1)
+    tok1: int
+    seq0: int                 # its local sequences are global sequences seq0 .. seq1-1
+    seq1: int
+    local_cu: np.ndarray      # int32 [seq1 - seq0 + 1], offsets into the rank's tokens
+    max_seqlen: int
+    carried_from: int         # rank where local sequence 0 began (== rank: not carried in)
+    open_tail: tuple | None   # (a, b): the rank's tokens of the sequence continuing past tok1
+    ends_here: np.ndarray     # bool [seq1 - seq0]: that sequence's final state is formed here
+
+    @property
+    def n_local(self) -> int:
+        return self.seq1 - self.seq0
+
+
+def plan_varlen_rank(cu_seqlens, bounds, rank: int) -> VarlenRankPlan:
+    """Which sequences rank `rank` sees, and how they continue across ranks.
+
+    cu_seqlens: int [nseq + 1] of the whole packed batch; bounds: int
+    [world + 1], non-decreasing from 0 to the total token count.  A non-empty
+    sequence belongs to every rank whose range it overlaps; an empty sequence
+    at position p belongs to the first rank with p < tok1 (the last rank when
+    p is the end of the batch), which also reports its final state (= its
+    carried-in state).
+    """
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    bd = np.asarray(bounds, dtype=np.int64)
+    world = len(bd) - 1
+    if cu.ndim != 1 or len(cu) < 1 or cu[0] != 0 or np.any(np.diff(cu) < 0):
+        raise ValueError("cu_seqlens must start at 0 and not decrease")
+    if world < 1 or bd[0] != 0 or bd[-1] != cu[-1] or np.any(np.diff(bd) < 0):
+        raise ValueError("bounds must run from 0 to the token count without decreasing")
+    if not 0 <= rank < world:
+        raise ValueError("rank out of range")
+    tok0, tok1 = int(bd[rank]), int(bd[rank + 1])
+    starts, ends = cu[:-1], cu[1:]
+    nonempty = ends > starts
+    overlap = np.maximum(starts, tok0) < np.minimum(ends, tok1)  # shares at least one token
+    # owner rank of each empty sequence: first rank whose range ends after p
+    owner = np.searchsorted(bd[1:], starts, side="right")
+    owner = np.minimum(owner, world - 1)
+    mine = overlap | (~nonempty & (owner == rank))
+    idx = np.nonzero(mine)[0]
+    if len(idx) == 0:
+        seq0 = seq1 = int(np.searchsorted(starts, tok0, side="left"))
+        return VarlenRankPlan(rank, tok0, tok1, seq0, seq1, np.zeros(1, np.int32), 0, rank, None,
+                              np.zeros(0, bool))
+    seq0, seq1 = int(idx[0]), int(idx[-1]) + 1
+    if len(idx) != seq1 - seq0:
+        raise AssertionError("local sequences are not contiguous")
+    local_cu = (np.clip(cu[seq0:seq1 + 1], tok0, tok1) - tok0).astype(np.int32)
+    lens = np.diff(local_cu)
+    carried_from = rank
+    if cu[seq0] < tok0:  # the first sequence began on an earlier rank
+        carried_from = int(np.searchsorted(bd[1:], cu[seq0], side="right"))
+    open_tail = None
+    if cu[seq1] > tok1:  # the last sequence continues on a later rank
+        open_tail = (int(local_cu[-2]), int(local_cu[-1]))
+    ends_here = cu[seq0 + 1:seq1 + 1] <= tok1
+    if open_tail is not None:
+        ends_here[-1] = False
+    return VarlenRankPlan(rank, tok0, tok1, seq0, seq1, local_cu, int(lens.max()) if len(lens) else 0,
+                          carried_from, open_tail, ends_here.astype(bool))
+
+
+def varlen_local_prefix(plan: VarlenRankPlan, k, v, ops=DeviceOps):
+    """Step 1 on one rank: the local prefix [H, d, d] of the sequence still
+    open at the end of its range (zero when every sequence ends there)."""
+    _, H, d = k.shape
+    a, b = plan.open_tail if plan.open_tail is not None else (0, 0)
+    return ops.kv_aggregate(k[a:b].reshape(1, b - a, H, d), v[a:b].reshape(1, b - a, H, d))[0]
+
+
+def varlen_local_scan(plan: VarlenRankPlan, q, k, v, parts, state_in=None, out_dtype=torch.bfloat16,
+                      ops=DeviceOps):
+    """Step 3 on one rank, given every rank's local prefix (parts [W, H, d,
+    d], rank order): the carried-in states of the rank's sequences, then its
+    local scan.  Returns (out [tokens, H, d], local final states)."""
+    _, H, d = q.shape
+    if plan.n_local == 0:
+        return q.new_empty((0, H, d), dtype=out_dtype), parts.new_empty((0, H, d, d))
+    sin = parts.new_empty((plan.n_local, H, d, d))
+    s0 = None if state_in is None else state_in[plan.seq0]
+    cf, r = plan.carried_from, plan.rank
+    if cf < r:  # global prefix of the sequence carried into this range
+        ops.state_prefix(parts[cf:r], r - cf, s0, sin[0])
+    else:
+        ops.state_prefix(None, 0, s0, sin[0])
+    if plan.n_local > 1:
+        rest = None if state_in is None else state_in[plan.seq0 + 1:plan.seq1]
+        ops.state_prefix(None, 0, rest, sin[1:])
+    return ops.prefill_varlen(q, k, v, plan.local_cu, plan.max_seqlen, sin, out_dtype)
+
+
+def lasp_prefill_varlen(q, k, v, cu_seqlens, bounds, group=None, state_in=None, out_dtype=torch.bfloat16,
+                        ops=DeviceOps):
+    """Prefill of this rank's range [bounds[r], bounds[r+1]) of a packed batch.
+
+    q, k, v: [bounds[r+1] - bounds[r], H, d] bf16 (this rank's tokens);
+    cu_seqlens, bounds: host int arrays of the whole batch (the same on every
+    rank); state_in: fp32 [nseq, H, d, d] carried-in states of all sequences
+    (the same on every rank), or None for zero.  Returns (out [tokens, H, d],
+    local final states [seq1 - seq0, H, d, d], plan): row i of the states is
+    the final state of global sequence plan.seq0 + i where plan.ends_here[i]
+    (the other rows, at most the last one, are only this rank's part).
+    """
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if len(bounds) != world + 1:
+        raise ValueError("bounds must hold world + 1 entries")
+    plan = plan_varlen_rank(cu_seqlens, bounds, rank)
+    if q.dim() != 3 or q.shape[0] != plan.tok1 - plan.tok0:
+        raise ValueError("q must be [this rank's tokens, H, d]")
+    _, H, d = q.shape
+    local = varlen_local_prefix(plan, k, v, ops)
+    gathered = local.new_empty((world * H, d, d))  # rank-major
+    dist.all_gather_into_tensor(gathered, local.contiguous(), group=group)
+    out, st = varlen_local_scan(plan, q, k, v, gathered.view(world, H, d, d), state_in, out_dtype, ops)
+    return out, st, plan

@@ -120,6 +120,37 @@ def test_emulated_ranks_reproduce_the_whole_sequence(oracle_mod):
     check_state(to_np(final), rst, what="final state")
 
 
+@pytest.mark.parametrize("lens,world", [([300, 0, 1290, 77, 0, 2100, 1, 129], 3),
+                                        ([40, 5000, 60], 4)])
+def test_emulated_ranks_on_a_packed_batch(oracle_mod, lens, world):
+    """A packed batch cut evenly into ranges at arbitrary tokens (sequences
+    spanning several ranks, empty sequences), run through the same two steps
+    lasp_prefill_varlen runs on each rank, with a stack of the local prefixes
+    standing in for the AllGather."""
+    from linear_attention_blocked_b200 import seqpar
+    H = 4
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    T = int(cu[-1])
+    q, k, v = la_inputs.qkv((T, H, D), seed=410 + world, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(411)
+    sin = torch.randn((len(lens), H, D, D), generator=gen, device="cuda") * 0.1
+    bounds = seqpar.split_tokens(T, world)
+    plans = [seqpar.plan_varlen_rank(cu, bounds, r) for r in range(world)]
+    rng = lambda t, p: t[p.tok0:p.tok1].contiguous()
+    parts = torch.stack([seqpar.varlen_local_prefix(p, rng(k, p), rng(v, p)) for p in plans])
+    outs, final = [], torch.full((len(lens), H, D, D), float("nan"), device="cuda")
+    for p in plans:
+        o, st = seqpar.varlen_local_scan(p, rng(q, p), rng(k, p), rng(v, p), parts, sin, torch.float32)
+        outs.append(o)
+        for i in np.nonzero(p.ends_here)[0]:
+            final[p.seq0 + i] = st[i]
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = oracle_mod.recurrent(la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v), cu,
+                                    state_in=to_np(sin))
+    check_out(to_np(torch.cat(outs, 0)), ref, bf16_out=False, what="packed outputs")
+    check_state(to_np(final), rst, what="final states")
+
+
 _ONE_RANK = r"""
 import os, sys
 sys.path.insert(0, os.environ["LA_ROOT"])
@@ -136,6 +167,13 @@ ref, st = la.prefill(q, k, v, state_in=sin)
 torch.cuda.synchronize()
 same = torch.equal(out, ref)
 rel = float((final - st).norm() / st.norm())
+import numpy as np
+cu = la_inputs.cu_seqlens_from_lengths([700, 0, 1300])
+qp, kp, vp = (t.reshape(-1, H, D)[:2000].contiguous() for t in (q, k, v))
+sinp = torch.randn((3, H, D, D), device="cuda") * 0.1
+outp, stp, plan = la.seqpar.lasp_prefill_varlen(qp, kp, vp, cu, np.array([0, 2000]), state_in=sinp)
+refp, rstp = la.prefill_varlen(qp, kp, vp, torch.from_numpy(cu).cuda(), 1300, state_in=sinp)
+same = same and torch.equal(outp, refp) and torch.equal(stp, rstp) and bool(plan.ends_here.all())
 dist.destroy_process_group()
 print("RESULT", int(same), rel, la.get_device_status())
 """
@@ -143,8 +181,9 @@ print("RESULT", int(same), rel, la.get_device_status())
 
 def test_lasp_prefill_under_one_rank_nccl_group():
     """With one rank the global prefix is the carried-in state itself, so the
-    output must equal la_prefill's bit for bit; the final state differs from
-    la_prefill's only in summation order."""
+    output must equal la_prefill's bit for bit (and the packed form's outputs
+    and states those of la_prefill_varlen); the final state of the
+    equal-length form differs from la_prefill's only in summation order."""
     import socket
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -153,6 +192,6 @@ def test_lasp_prefill_under_one_rank_nccl_group():
     res = subprocess.run([sys.executable, "-c", _ONE_RANK], env=env, capture_output=True, text=True, timeout=300)
     assert res.returncode == 0, res.stderr[-2000:]
     line = [x for x in res.stdout.splitlines() if x.startswith("RESULT")][-1].split()
-    assert line[1] == "1", "output differs from la_prefill"
+    assert line[1] == "1", "output differs from la_prefill / la_prefill_varlen"
     assert float(line[2]) <= 1e-5
     assert int(line[3]) == la.LA_OK

@@ -1,9 +1,11 @@
 """Sequence parallelism across ranks (LASP+) on CPU ranks (gloo, world sizes
-2 and 3): lasp_prefill's exchange -- local prefixes all-gathered in rank
+2 to 4): lasp_prefill's exchange -- local prefixes all-gathered in rank
 order, the global prefix of the ranks before this one, the local scan seeded
-with it -- reproduces the oracle's result for the whole sequences.  The
-device steps are host stand-ins built from the oracle (fp64), so what is
-checked here is the rank logic; the CUDA steps are checked on the GPU."""
+with it -- reproduces the oracle's result for the whole sequences, and so
+does lasp_prefill_varlen on packed batches cut at arbitrary token positions
+(sequences spanning several ranks, empty sequences, empty ranks).  The device
+steps are host stand-ins built from the oracle (fp64), so what is checked
+here is the rank logic; the CUDA steps are checked on the GPU."""
 import os
 import socket
 
@@ -41,10 +43,14 @@ class _HostOps:
         return torch.from_numpy(st)
 
     @staticmethod
-    def state_prefix(parts, count, state_in):
-        acc = torch.zeros(parts.shape[1:], dtype=torch.float64) if state_in is None else state_in.clone()
+    def state_prefix(parts, count, state_in, out=None):
+        shape = parts.shape[1:] if parts is not None else (state_in if state_in is not None else out).shape
+        acc = torch.zeros(shape, dtype=torch.float64) if state_in is None else state_in.clone()
         for i in range(count):
             acc += parts[i]
+        if out is not None:
+            out.copy_(acc)
+            return out
         return acc
 
     @staticmethod
@@ -56,6 +62,13 @@ class _HostOps:
         V, _ = _HostOps._packed(v)
         out, _ = oracle.recurrent(Q, K, V, cu, state_in=state_in.numpy())
         return torch.from_numpy(out).reshape(B, n, H, d)
+
+    @staticmethod
+    def prefill_varlen(q, k, v, cu_seqlens, max_seqlen, state_in, out_dtype):
+        import oracle
+        out, st = oracle.recurrent(la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v), cu_seqlens,
+                                   state_in=state_in.numpy())
+        return torch.from_numpy(out), torch.from_numpy(st)
 
 
 def _worker(rank, world, port, lens, result_path):
@@ -95,4 +108,56 @@ def test_ranks_reproduce_the_whole_sequence(tmp_path, oracle_mod, lens):
     result = tmp_path / "result.txt"
     mp.start_processes(_worker, args=(len(lens), _free_port(), lens, str(result)), nprocs=len(lens), join=True,
                        start_method="spawn")
+    assert result.read_text() == "ok"
+
+
+def _varlen_worker(rank, world, port, lens, bounds, result_path):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from linear_attention_blocked_b200 import seqpar
+        H = 2
+        cu = la_inputs.cu_seqlens_from_lengths(lens)
+        T = int(cu[-1])
+        q, k, v = la_inputs.qkv((T, H, D), seed=63, scale=0.5)
+        sin = torch.from_numpy(np.random.default_rng(64).standard_normal((len(lens), H, D, D)) * 0.3)
+        a, b = int(bounds[rank]), int(bounds[rank + 1])
+        out, st, plan = seqpar.lasp_prefill_varlen(q[a:b].contiguous(), k[a:b].contiguous(), v[a:b].contiguous(),
+                                                   cu, bounds, state_in=sin, ops=_HostOps)
+        shares = [None] * world
+        dist.all_gather_object(shares, (out.double().numpy(), st.double().numpy(), plan.seq0, plan.ends_here))
+        if rank == 0:
+            ref, rst = oracle.recurrent(la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v), cu,
+                                        state_in=sin.numpy())
+            got = np.concatenate([o for o, _, _, _ in shares], axis=0)
+            ok = got.shape == ref.shape and np.abs(got - ref).max() <= 1e-10 * np.abs(ref).max()
+            final = np.full(rst.shape, np.nan)
+            seen = np.zeros(len(lens), int)
+            for _, s_, seq0, ends in shares:
+                for i in np.nonzero(ends)[0]:
+                    final[seq0 + i] = s_[i]
+                    seen[seq0 + i] += 1
+            ok &= bool(np.all(seen == 1))
+            ok &= bool(np.abs(final - rst).max() <= 1e-10 * np.abs(rst).max())
+            with open(result_path, "w") as fh:
+                fh.write("ok" if ok else f"mismatch seen={seen.tolist()}")
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lens,bounds", [
+    ([50, 0, 130, 7, 0, 200, 1], None),                 # cut evenly into 3 ranks
+    ([20, 400, 30], None),                              # the long sequence spans all 4 ranks
+    ([50, 0, 130, 7, 0, 200, 1], [0, 50, 50, 300, 388]),  # cuts on sequence edges, an empty rank
+    ([3, 0, 0], [0, 3, 3]),                             # trailing empty sequences on the last rank
+])
+def test_varlen_ranks_reproduce_the_packed_batch(tmp_path, oracle_mod, lens, bounds):
+    from linear_attention_blocked_b200 import seqpar
+    T = sum(lens)
+    world = 4 if bounds is None and len(lens) == 3 else (3 if bounds is None else len(bounds) - 1)
+    bounds = np.asarray(bounds if bounds is not None else seqpar.split_tokens(T, world))
+    result = tmp_path / "result.txt"
+    mp.start_processes(_varlen_worker, args=(world, _free_port(), lens, bounds, str(result)), nprocs=world,
+                       join=True, start_method="spawn")
     assert result.read_text() == "ok"
