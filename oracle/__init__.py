@@ -3,5 +3,5 @@
 Only the test suite, the entry module's smoke check and the benchmark's
 CPU-baseline leg import this package; the product package never does.
 """
-from .oracle import (blocked, build, decode_step, max_threads, quadratic,  # noqa: F401
+from .oracle import (backward, blocked, build, decode_step, max_threads, quadratic,  # noqa: F401
                      recurrent, segmented)

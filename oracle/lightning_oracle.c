@@ -23,6 +23,9 @@
  *        §3.2 item 1 (data packing: samples joined end to end),
  *        §3.3 items 1-2 (decode: length-1 tokens, KV update fused with the
  *        prefix-KV cache).
+ *   Gradients: [P5] §3.2 item 3 trains the model with LASP+ but the pages
+ *   give no backward formulas; lao_backward writes out the derivatives of
+ *   the forward definition below, term by term.
  *   The pages print no formula; the formula used is the plainest reading of
  *   that prose: O = (Q K^T ⊙ M) V with the inclusive causal mask
  *   M[t][s] = 1 iff s <= t, no scale, feature map, normalisation or decay
@@ -361,4 +364,105 @@ int lao_decode_step(const uint16_t *q, const uint16_t *k, const uint16_t *v,
         }
     }
     return 0;
+}
+
+/*
+ * Gradients of the forward definition (lao_quadratic) for a loss L with
+ * dL/do_t = g_t (dout, bf16 bits [T][H][d]) and dL/dS_out = G_S (dstate_out,
+ * double [nseq][nh][d][d] or NULL = 0), where
+ *   o_t   = sum_{s <= t} (q_t . k_s) v_s + q_t S_in,
+ *   S_out = S_in + sum_s k_s^T v_s.
+ * Differentiating term by term:
+ *   dq_t = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T
+ *   dk_s = sum_{t >= s} (g_t . v_s) q_t + v_s G_S^T
+ *   dv_s = sum_{t >= s} (q_t . k_s) g_t + k_s G_S
+ *   dS_in = sum_t q_t^T g_t + G_S
+ * (row vectors; (x M^T)[a] = sum_b M[a][b] x[b]).  Plain O(n^2 d) loops per
+ * (sequence, head).  dq, dk, dv: double [T][nh][d]; dstate_in: double
+ * [nseq][nh][d][d] or NULL.
+ */
+int lao_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                 const int32_t *cu_seqlens, int nseq, int H, int d,
+                 const int32_t *heads, int nh, const double *state_in,
+                 const double *dstate_out, double *dq, double *dk, double *dv,
+                 double *dstate_in, int nthreads)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        const int t0 = cu_seqlens[i], n = cu_seqlens[i + 1] - cu_seqlens[i];
+        const size_t nd = (size_t)(n > 0 ? n : 1) * d;
+        double *Q = (double *)malloc(nd * sizeof(double));
+        double *K = (double *)malloc(nd * sizeof(double));
+        double *V = (double *)malloc(nd * sizeof(double));
+        double *G = (double *)malloc(nd * sizeof(double));
+        if (!Q || !K || !V || !G) {
+            bad = 1;
+            free(Q); free(K); free(V); free(G);
+            continue;
+        }
+        for (int t = 0; t < n; ++t)
+            for (int a = 0; a < d; ++a) {
+                Q[(size_t)t * d + a] = widen_bf16(ROW(q, t0 + t, h)[a]);
+                K[(size_t)t * d + a] = widen_bf16(ROW(k, t0 + t, h)[a]);
+                V[(size_t)t * d + a] = widen_bf16(ROW(v, t0 + t, h)[a]);
+                G[(size_t)t * d + a] = widen_bf16(ROW(dout, t0 + t, h)[a]);
+            }
+        const double *Sin = state_in ? state_in + (size_t)p * d * d : NULL;
+        const double *GS = dstate_out ? dstate_out + (size_t)p * d * d : NULL;
+        for (int t = 0; t < n; ++t) {
+            /* dq_t = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T */
+            double *o = dq + ((size_t)(t0 + t) * nh + j) * d;
+            for (int a = 0; a < d; ++a) o[a] = 0.0;
+            for (int s2 = 0; s2 <= t; ++s2) {
+                double w = 0.0;
+                for (int b = 0; b < d; ++b) w += G[(size_t)t * d + b] * V[(size_t)s2 * d + b];
+                for (int a = 0; a < d; ++a) o[a] += w * K[(size_t)s2 * d + a];
+            }
+            if (Sin)
+                for (int a = 0; a < d; ++a)
+                    for (int b = 0; b < d; ++b) o[a] += Sin[(size_t)a * d + b] * G[(size_t)t * d + b];
+        }
+        for (int s2 = 0; s2 < n; ++s2) {
+            /* dk_s = sum_{t >= s} (g_t . v_s) q_t + v_s G_S^T
+               dv_s = sum_{t >= s} (q_t . k_s) g_t + k_s G_S */
+            double *ok = dk + ((size_t)(t0 + s2) * nh + j) * d;
+            double *ov = dv + ((size_t)(t0 + s2) * nh + j) * d;
+            for (int a = 0; a < d; ++a) ok[a] = ov[a] = 0.0;
+            for (int t = s2; t < n; ++t) {
+                double wk = 0.0, wv = 0.0;
+                for (int b = 0; b < d; ++b) {
+                    wk += G[(size_t)t * d + b] * V[(size_t)s2 * d + b];
+                    wv += Q[(size_t)t * d + b] * K[(size_t)s2 * d + b];
+                }
+                for (int a = 0; a < d; ++a) {
+                    ok[a] += wk * Q[(size_t)t * d + a];
+                    ov[a] += wv * G[(size_t)t * d + a];
+                }
+            }
+            if (GS)
+                for (int a = 0; a < d; ++a)
+                    for (int b = 0; b < d; ++b) {
+                        ok[a] += GS[(size_t)a * d + b] * V[(size_t)s2 * d + b];
+                        ov[b] += K[(size_t)s2 * d + a] * GS[(size_t)a * d + b];
+                    }
+        }
+        if (dstate_in) {
+            /* dS_in = sum_t q_t^T g_t + G_S */
+            double *D = dstate_in + (size_t)p * d * d;
+            for (size_t e = 0; e < (size_t)d * d; ++e) D[e] = GS ? GS[e] : 0.0;
+            for (int t = 0; t < n; ++t)
+                for (int a = 0; a < d; ++a)
+                    for (int b = 0; b < d; ++b)
+                        D[(size_t)a * d + b] += Q[(size_t)t * d + a] * G[(size_t)t * d + b];
+        }
+        free(Q); free(K); free(V); free(G);
+    }
+    return bad ? -1 : 0;
 }

@@ -77,6 +77,9 @@ def _bind(path: str):
     lib.lao_segmented.restype = c_int
     lib.lao_decode_step.argtypes = [u16p, u16p, u16p, c_int, c_int, c_int, f64p, f64p, c_int]
     lib.lao_decode_step.restype = c_int
+    lib.lao_backward.argtypes = [u16p, u16p, u16p, u16p, i32p, c_int, c_int, c_int, i32p, c_int,
+                                 f64p, f64p, f64p, f64p, f64p, f64p, c_int]
+    lib.lao_backward.restype = c_int
     lib.lao_max_threads.argtypes = []
     lib.lao_max_threads.restype = c_int
     return lib
@@ -175,3 +178,30 @@ def decode_step(q, k, v, state, threads=None, lib=None):
     if rc != 0:
         raise ValueError("lao_decode_step rejected its arguments")
     return out, st
+
+
+def backward(q, k, v, dout, cu_seqlens, heads=None, state_in=None, dstate_out=None, threads=None,
+             lib=None):
+    """Gradients of the forward definition for dL/dO = dout (bf16 bits, like
+    q) and dL/dS_out = dstate_out (float64 [nseq, nh, d, d] or None).
+    Returns (dq, dk, dv [T, nh, d], dstate_in [nseq, nh, d, d])."""
+    q, k, v, cu, nseq, T, H, d, hs, nh, state_in = _prep(q, k, v, cu_seqlens, heads, state_in)
+    g = np.ascontiguousarray(dout, dtype=np.uint16)
+    if g.shape != q.shape:
+        raise ValueError("dout must have the shape of q")
+    if dstate_out is not None:
+        dstate_out = np.ascontiguousarray(dstate_out, dtype=np.float64)
+        if dstate_out.shape != (nseq, nh, d, d):
+            raise ValueError(f"dstate_out must be [nseq, nheads, d, d] = {(nseq, nh, d, d)}")
+    dq, dk, dv = (np.zeros((T, nh, d), dtype=np.float64) for _ in range(3))
+    dsin = np.zeros((nseq, nh, d, d), dtype=np.float64)
+    rc = (lib or _load()).lao_backward(_ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+                                       _ptr(v, ctypes.c_uint16), _ptr(g, ctypes.c_uint16),
+                                       _ptr(cu, ctypes.c_int32), nseq, H, d, _ptr(hs, ctypes.c_int32), nh,
+                                       _ptr(state_in, ctypes.c_double), _ptr(dstate_out, ctypes.c_double),
+                                       _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double),
+                                       _ptr(dv, ctypes.c_double), _ptr(dsin, ctypes.c_double),
+                                       int(threads or 0))
+    if rc != 0:
+        raise ValueError("lao_backward rejected its arguments")
+    return dq, dk, dv, dsin

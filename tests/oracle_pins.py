@@ -10,7 +10,10 @@ the oracle handle ``lib`` (None = the real oracle) disagrees with
   * brute force in pure Python on tiny inputs,
   * identities of the method (block-size invariance, segment (LASP+)
     decomposition, packed-sequence independence, causality, state carry,
-    decode after prefill).
+    decode after prefill),
+  * for the gradients: hand-worked examples, torch autograd of the dense
+    forward expression (a library routine), and Euler's identity for the
+    parts of the loss linear in one argument, using the forward oracle.
 
 The same functions run in test_oracle_pins.py (real oracle) and in
 test_oracle_mutations.py (oracle copies with a planted mistake, each of which
@@ -294,6 +297,95 @@ def pin_linearity(orc, lib=None):
     assert np.array_equal(o4, -o) and np.array_equal(s4, -s)
 
 
+# -------------------------------------------------------------------------- gradients
+def pin_backward_golden(orc, lib=None):
+    """The hand-worked gradient examples (d = 1 and d = 2), exact."""
+    g = load_golden()
+    for name in ("backward_d1", "backward_d2"):
+        c = g[name]
+        d = c["q"].shape[1]
+        cu = np.array([0, c["q"].shape[0]], np.int32)
+        dq, dk, dv, dsin = orc.backward(_b(c["q"]), _b(c["k"]), _b(c["v"]), _b(c["dout"]), cu,
+                                        state_in=c["state_in"].reshape(1, 1, d, d),
+                                        dstate_out=c["dstate_out"].reshape(1, 1, d, d), lib=lib)
+        assert np.array_equal(dq[:, 0], c["dq"]), (name, "dq", dq[:, 0])
+        assert np.array_equal(dk[:, 0], c["dk"]), (name, "dk", dk[:, 0])
+        assert np.array_equal(dv[:, 0], c["dv"]), (name, "dv", dv[:, 0])
+        assert np.array_equal(dsin[0, 0], c["dstate_in"]), (name, "dS_in", dsin[0, 0])
+
+
+def _autograd_reference(Qf, Kf, Vf, Gf, cu, Sin, GS):
+    """torch autograd (a library routine) of the dense forward expression, one
+    sequence at a time, in fp64."""
+    import torch
+    outs = [np.zeros_like(Qf) for _ in range(3)]
+    dsin = np.zeros_like(Sin)
+    for i in range(len(cu) - 1):
+        a, b = int(cu[i]), int(cu[i + 1])
+        for h in range(Qf.shape[1]):
+            q, k, v = (torch.tensor(x[a:b, h], dtype=torch.float64, requires_grad=True) for x in (Qf, Kf, Vf))
+            s_in = torch.tensor(Sin[i, h], dtype=torch.float64, requires_grad=True)
+            o = torch.tril(q @ k.T) @ v + q @ s_in
+            s_out = s_in + k.T @ v
+            loss = (torch.tensor(Gf[a:b, h]) * o).sum() + (torch.tensor(GS[i, h]) * s_out).sum()
+            loss.backward()
+            for dst, x in zip(outs, (q, k, v)):
+                dst[a:b, h] = x.grad.numpy()
+            dsin[i, h] = s_in.grad.numpy()
+    return outs + [dsin]
+
+
+def pin_backward_autograd(orc, lib=None):
+    """Packed sequences (one empty) with carried-in states and state
+    gradients: the oracle's gradients equal torch autograd's to rounding."""
+    H, d = 2, 5
+    cu = np.array([0, 7, 7, 30, 41], np.int32)
+    T = int(cu[-1])
+    Q, K, V = _rand_bits(T, H, d, seed=31)
+    G, _, _ = _rand_bits(T, H, d, seed=32)
+    rng = np.random.default_rng(33)
+    Sin = rng.standard_normal((4, H, d, d))
+    GS = rng.standard_normal((4, H, d, d))
+    got = orc.backward(Q, K, V, G, cu, state_in=Sin, dstate_out=GS, lib=lib)
+    ref = _autograd_reference(_f(Q), _f(K), _f(V), _f(G), cu, Sin, GS)
+    for name, x, y in zip(("dq", "dk", "dv", "dS_in"), got, ref):
+        assert _rel(x, y) < 1e-12, (name, _rel(x, y))
+    # without carried-in state and state gradient: the same as zeros
+    got0 = orc.backward(Q, K, V, G, cu, lib=lib)
+    ref0 = _autograd_reference(_f(Q), _f(K), _f(V), _f(G), cu, np.zeros_like(Sin), np.zeros_like(GS))
+    for x, y in zip(got0, ref0):
+        assert _rel(x, y) < 1e-12
+
+
+def pin_backward_homogeneity(orc, lib=None):
+    """Euler's identity for the pieces of the loss L = <g, o> + <G, S_out>
+    that are linear in one argument, with o and S_out from the (separately
+    pinned) forward oracle:
+      sum q.dq = <g, o>;   sum k.dk = sum v.dv = <g, o_intra> + <G, S_out - S_in>;
+      <S_in, dS_in> = <g, o - o_intra> + <G, S_in>."""
+    H, d = 1, 6
+    cu = np.array([0, 19, 40], np.int32)
+    T = int(cu[-1])
+    Q, K, V = _rand_bits(T, H, d, seed=35)
+    G, _, _ = _rand_bits(T, H, d, seed=36)
+    rng = np.random.default_rng(37)
+    Sin = rng.standard_normal((2, H, d, d))
+    GS = rng.standard_normal((2, H, d, d))
+    dq, dk, dv, dsin = orc.backward(Q, K, V, G, cu, state_in=Sin, dstate_out=GS, lib=lib)
+    o, s_out = orc.quadratic(Q, K, V, cu, state_in=Sin, lib=lib)
+    o_intra, kv = orc.quadratic(Q, K, V, cu, lib=lib)
+    g = _f(G)
+    L_o, L_intra = float((g * o).sum()), float((g * o_intra).sum())
+    assert abs(float((_f(Q) * dq).sum()) - L_o) < 1e-11 * max(1.0, abs(L_o))
+    rhs = L_intra + float((GS * kv).sum())
+    for x, dx in ((_f(K), dk), (_f(V), dv)):
+        assert abs(float((x * dx).sum()) - rhs) < 1e-11 * max(1.0, abs(rhs))
+    rhs_s = (L_o - L_intra) + float((GS * Sin).sum())
+    assert abs(float((Sin * dsin).sum()) - rhs_s) < 1e-11 * max(1.0, abs(rhs_s))
+    assert np.allclose(s_out - Sin, kv, rtol=0, atol=1e-12)
+
+
 ALL_PINS = [pin_golden, pin_single_token, pin_constant_kv, pin_one_hot_q, pin_exact_integers,
             pin_brute_force, pin_forms_agree, pin_causality_and_packing,
-            pin_state_carry_and_decode, pin_linearity]
+            pin_state_carry_and_decode, pin_linearity, pin_backward_golden, pin_backward_autograd,
+            pin_backward_homogeneity]

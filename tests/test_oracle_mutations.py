@@ -37,6 +37,22 @@ MUTANTS = [
     ("decode_update_index", "S[(size_t)a * d + b] += ka * widen_bf16(vp[b]);",
      "S[(size_t)a * d + b] += ka * widen_bf16(vp[a]);", 0),
     ("widen_wrong_shift", "((uint32_t)bits) << 16", "((uint32_t)bits) << 15", 0),
+    ("backward_dq_strict_mask", "for (int s2 = 0; s2 <= t; ++s2) {", "for (int s2 = 0; s2 < t; ++s2) {", 0),
+    ("backward_dq_state_transposed", "o[a] += Sin[(size_t)a * d + b] * G[(size_t)t * d + b];",
+     "o[a] += Sin[(size_t)b * d + a] * G[(size_t)t * d + b];", 0),
+    ("backward_dkdv_strict_mask", "for (int t = s2; t < n; ++t) {", "for (int t = s2 + 1; t < n; ++t) {", 0),
+    ("backward_dk_wrong_factor", "ok[a] += wk * Q[(size_t)t * d + a];", "ok[a] += wk * K[(size_t)t * d + a];", 0),
+    ("backward_dv_wrong_score", "wv += Q[(size_t)t * d + b] * K[(size_t)s2 * d + b];",
+     "wv += Q[(size_t)t * d + b] * Q[(size_t)s2 * d + b];", 0),
+    ("backward_dk_drops_state_grad", "ok[a] += GS[(size_t)a * d + b] * V[(size_t)s2 * d + b];",
+     "ok[a] += 0.0 * GS[(size_t)a * d + b] * V[(size_t)s2 * d + b];", 0),
+    ("backward_dk_state_grad_transposed", "ok[a] += GS[(size_t)a * d + b] * V[(size_t)s2 * d + b];",
+     "ok[a] += GS[(size_t)b * d + a] * V[(size_t)s2 * d + b];", 0),
+    ("backward_dv_state_grad_transposed", "ov[b] += K[(size_t)s2 * d + a] * GS[(size_t)a * d + b];",
+     "ov[b] += K[(size_t)s2 * d + a] * GS[(size_t)b * d + a];", 0),
+    ("backward_dsin_drops_state_grad", "D[e] = GS ? GS[e] : 0.0;", "D[e] = 0.0;", 0),
+    ("backward_dsin_transposed", "D[(size_t)a * d + b] += Q[(size_t)t * d + a] * G[(size_t)t * d + b];",
+     "D[(size_t)b * d + a] += Q[(size_t)t * d + a] * G[(size_t)t * d + b];", 0),
 ]
 
 
