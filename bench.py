@@ -9,7 +9,8 @@ cross-SM segment hand-off + epilogue).  In the same run the fused batched
 decode step is timed on its own workload (256 sequences x 64 heads, fp32
 states initialised by a 4096-token prefill) and reported under "decode", and
 the local-prefix step of sequence parallelism (la_kv_aggregate) on the
-prefill's k and v under "kv_aggregate".
+prefill's k and v under "kv_aggregate", and the gradients of the prefill
+(la_prefill_backward) under "backward".
 
   python bench.py [--gpus N] [--steps K] [--warmup W]      # CUDA path
   python bench.py --impl reference ...                     # fp64 CPU oracle arm
@@ -68,6 +69,11 @@ def prefill_flops(tok_heads: int, block: int, frac_phase_a: float):
 def aggregate_bytes(tok_heads: int, pairs: int) -> int:
     """Read k and v (bf16), write one fp32 d x d sum per (sequence, head)."""
     return tok_heads * D * 2 * 2 + pairs * D * D * 4
+
+
+def backward_bytes(tok_heads: int) -> int:
+    """Read q, k, v and dout, write dq, dk and dv (all bf16)."""
+    return tok_heads * D * 2 * 7
 
 
 def decode_bytes(pairs: int) -> int:
@@ -351,6 +357,8 @@ def run_cuda(args, world, rank, local):
 
     # ---------------- local prefix of sequence parallelism on the same k, v
     agg = bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world)
+    # ---------------- gradients of the prefill on the same q, k, v
+    bwd = bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world)
 
     status2 = la.get_device_status()
     if rank != 0:
@@ -381,6 +389,7 @@ def run_cuda(args, world, rank, local):
         "clocks": clocks,
         "decode": dec,
         "kv_aggregate": agg,
+        "backward": bwd,
         "cpu_baseline": cpu,
         "device_status": [int(status), int(status2)],
     }
@@ -414,6 +423,39 @@ def bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world):
                          "traffic": recorded_traffic("la_kv_aggregate_kernel", "aggregate_B1_H64_N32768"),
                          "bytes_per_launch": byts,
                          "duration": "CUDA events around each la_kv_aggregate call (aggregate + reduce)"}}
+
+
+def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
+    """la_prefill_backward (dq, dk, dv, dS_in for a random dout; no carried-in
+    state or state gradient) on the prefill workload, bf16 gradients."""
+    g, _, _ = la_inputs.qkv((B, N, H, D), SEED + 11, device=dev)
+    grads = [torch.empty_like(q) for _ in range(3)]
+    ws = torch.empty(la.backward_workspace_size(B, N, H, D), dtype=torch.uint8, device=dev)
+
+    def call():
+        la.prefill_backward(q, k, v, g, dq=grads[0], dk=grads[1], dv=grads[2], workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(5, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    byts = backward_bytes(B * N * H)
+    gbs = byts / (ms * 1e-3) / 1e9
+    del g, grads, ws
+    return {"workload": "prefill backward B=1 H=64 N=32768 d=128, bf16 dq/dk/dv + fp32 dS_in",
+            "ms_per_call": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (three scans) + la_kv_aggregate_kernel (two sums)",
+                         "traffic": None, "bytes_per_launch": byts,
+                         "duration": "CUDA events around each la_prefill_backward call (about ten kernels)"}}
 
 
 def bench_decode(la, dev, stream, args, hbm_peak, world):

@@ -248,6 +248,44 @@ LA_API la_status la_state_prefix(const float *parts, int count, const float *sta
                                  float *out, int nstates, int d, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Gradients of la_prefill.  The pages train the model with LASP+
+ * ("MiniMax-01技术报告解读", §3.2 item 3) but give no backward formulas; these
+ * are the derivatives of the forward definition at the top of this file for
+ * a loss L with dL/do_t = g_t (dout) and dL/dS_out = G (dstate_out):
+ *
+ *   dq_t  = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T
+ *   dk_s  = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
+ *   dv_s  = sum_{t >= s} (q_t . k_s) g_t + k_s G
+ *   dS_in = sum_t q_t^T g_t + G
+ *
+ * computed as three blocked scans: dq is a forward scan of (dout, v, k)
+ * from S_in^T; dk and dv scan forward too, starting from the sum over all
+ * tokens (W_k = sum_t g_t^T q_t + G^T, W_v = sum_t q_t^T g_t + G, each one
+ * la_kv_aggregate) and removing the earlier tokens as they go (an exclusive
+ * mask and a subtracted state update), which leaves the sums over t >= s.
+ * dS_in is W_v.
+ *
+ * q, k, v, dout: bf16 [B, N, H, d] contiguous (read only).  state_in,
+ * dstate_out: fp32 [B, H, d, d] row-major or NULL (= 0).  dq, dk, dv: [B, N,
+ * H, d] in grad_dtype (bf16 or fp32), fully written; they must not overlap
+ * each other, the inputs, the states or the workspace.  dstate_in: fp32
+ * [B, H, d, d] or NULL (not computed).  workspace: at least
+ * la_prefill_backward_workspace_size(B, N, H, d) bytes, 256-byte aligned,
+ * caller-owned scratch.  fp32 accumulation on the tensor cores.  Enqueues
+ * about a dozen kernels on `stream` and returns; argument errors are
+ * returned before any launch; device-side problems are reported by
+ * la_get_device_status.
+ * ------------------------------------------------------------------------- */
+LA_API size_t la_prefill_backward_workspace_size(int B, int N, int H, int d);
+
+LA_API la_status la_prefill_backward(const void *q, const void *k, const void *v,
+                                     const void *dout, int B, int N, int H, int d,
+                                     const float *state_in, const float *dstate_out,
+                                     void *dq, void *dk, void *dv, la_dtype grad_dtype,
+                                     float *dstate_in, void *workspace, size_t ws_bytes,
+                                     cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Status.
  * la_get_device_status synchronises `stream`, then returns and clears the
  * sticky device word of the current device (LA_ERR_TIMEOUT,

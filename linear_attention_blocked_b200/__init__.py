@@ -15,9 +15,10 @@ ABI (include/lightning_attn.h).  Entry points:
   state_prefix(parts, count, state_in)       la_state_prefix: state_in + parts[0] + ... + parts[count-1]
   lasp_prefill(q, k, v, group=...)           sequence parallelism across ranks (seqpar.py)
   lasp_prefill_varlen(q, k, v, cu, bounds)   the same for a packed batch cut at any token
+  prefill_backward(q, k, v, dout, ...)       la_prefill_backward: dq, dk, dv, dS_in
   get_device_status()                        la_get_device_status
 """
-from ._binding import (D, DEFAULT_BLOCK, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
+from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, prefill_backward, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
                        LA_ERR_INVALID_ARGUMENT, LA_ERR_TIMEOUT, LA_ERR_UNSUPPORTED,
                        LA_ERR_WORKSPACE, LA_FP32, LA_INJECT_NONE, LA_INJECT_SKIP_PUBLISH, LA_OK,
                        LAError, debug_inject, decode_step, decode_step_slots, get_device_status,

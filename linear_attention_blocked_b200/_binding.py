@@ -25,7 +25,8 @@ EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_worksp
             "la_set_wait_limit_ns", "la_set_segment_len", "la_debug_inject",
             "la_last_segment_len", "la_kernel_launches", "la_prefill_noalloc",
             "la_prefill_varlen_slots", "la_decode_step_slots", "la_mixed_step",
-            "la_kv_aggregate_workspace_size", "la_kv_aggregate", "la_state_prefix")
+            "la_kv_aggregate_workspace_size", "la_kv_aggregate", "la_state_prefix",
+            "la_prefill_backward_workspace_size", "la_prefill_backward")
 
 
 class LAError(RuntimeError):
@@ -80,6 +81,11 @@ def lib():
         L.la_kv_aggregate.restype = c_int
         L.la_state_prefix.argtypes = [vp, c_int, vp, vp, c_int, c_int, vp]
         L.la_state_prefix.restype = c_int
+        L.la_prefill_backward_workspace_size.argtypes = [c_int] * 4
+        L.la_prefill_backward_workspace_size.restype = sz
+        L.la_prefill_backward.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, c_int, vp,
+                                          vp, sz, vp]
+        L.la_prefill_backward.restype = c_int
         L.la_get_device_status.argtypes = [vp]
         L.la_get_device_status.restype = c_int
         L.la_status_string.argtypes = [c_int]
@@ -375,6 +381,43 @@ def state_prefix(parts, count: int, state_in=None, out=None, stream=None):
                                nstates, d, _stream_handle(stream))
     _check(st, "la_state_prefix")
     return out
+
+
+def backward_workspace_size(B: int, N: int, H: int, d: int = D) -> int:
+    return int(lib().la_prefill_backward_workspace_size(B, N, H, d))
+
+
+def prefill_backward(q, k, v, dout, state_in=None, dstate_out=None, grad_dtype=torch.bfloat16,
+                     want_dstate_in: bool = True, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """la_prefill_backward on [B, N, H, d] bf16 tensors: gradients of
+    la_prefill for dL/dout and dL/dstate_out.  Returns (dq, dk, dv,
+    dstate_in or None)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, N, H, d]")
+    B, N, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, name, torch.bfloat16, (B, N, H, d))
+    for name, t in (("state_in", state_in), ("dstate_out", dstate_out)):
+        if t is not None:
+            _need(t, name, torch.float32, (B, H, d, d))
+    grads = []
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if t is None:
+            t = torch.empty((B, N, H, d), dtype=grad_dtype, device=q.device)
+        _need(t, name, t.dtype, (B, N, H, d))
+        grads.append(t)
+    if len({t.dtype for t in grads}) != 1:
+        raise TypeError("dq, dk and dv must share one dtype")
+    dsin = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device) if want_dstate_in else None
+    ws_bytes = backward_workspace_size(B, N, H, d)
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, q.device)
+    st = lib().la_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, N, H, d, _ptr(state_in),
+                                   _ptr(dstate_out), _ptr(grads[0]), _ptr(grads[1]), _ptr(grads[2]),
+                                   _out_code(grads[0].dtype), _ptr(dsin), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(st, "la_prefill_backward")
+    return grads[0], grads[1], grads[2], dsin
 
 
 def get_device_status(stream=None) -> int:

@@ -298,4 +298,22 @@ la_state_prefix_kernel(const float4 *__restrict__ parts, int count, const float4
     }
 }
 
+// out[s] = in[s]^T for nstates D x D fp32 matrices (32 x 32 tiles through
+// shared memory; grid (nstates, (D/32)^2), 32 x 8 threads).
+constexpr int TRANSPOSE_TILE = 32;
+
+__global__ void __launch_bounds__(256)
+la_state_transpose_kernel(const float *__restrict__ in, float *__restrict__ out) {
+    __shared__ float tile[TRANSPOSE_TILE][TRANSPOSE_TILE + 1];
+    constexpr int TILES = D / TRANSPOSE_TILE;
+    const size_t base = (size_t)blockIdx.x * D * D;
+    const int ti = blockIdx.y / TILES, tj = blockIdx.y % TILES;  // tile row / column of `in`
+    const int x = threadIdx.x & 31, y0 = threadIdx.x >> 5;
+    for (int y = y0; y < TRANSPOSE_TILE; y += 8)
+        tile[y][x] = in[base + (size_t)(ti * TRANSPOSE_TILE + y) * D + tj * TRANSPOSE_TILE + x];
+    __syncthreads();
+    for (int y = y0; y < TRANSPOSE_TILE; y += 8)
+        out[base + (size_t)(tj * TRANSPOSE_TILE + y) * D + ti * TRANSPOSE_TILE + x] = tile[x][y];
+}
+
 }  // namespace la

@@ -131,7 +131,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
                        int nseq, long long T, int max_seqlen, int H, int d, int block,
                        const float *state_in, void *out, la_dtype out_dtype, float *state_out,
                        void *workspace, size_t ws_bytes, cudaStream_t stream,
-                       const int *slots = nullptr, int n_slots = 0) {
+                       const int *slots = nullptr, int n_slots = 0, bool anti = false) {
     la_status st = check_common(H, d, block, out_dtype);
     if (st != LA_OK) return st;
     if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -218,13 +218,19 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(la::la_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(la::la_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         la::PREFILL_SMEM);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(la::la_prefill_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, la::PREFILL_SMEM);
     });
     if (attr_err != cudaSuccess) return LA_ERR_CUDA;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    if (anti)
+        la::la_prefill_kernel<true><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    else
+        la::la_prefill_kernel<false><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;
@@ -280,6 +286,38 @@ AggPlan agg_plan(long long npairs, int N) {
 }
 
 size_t agg_ws_bytes(const AggPlan &a) { return (size_t)2 * a.ctas * la::D * la::D * sizeof(float); }
+
+la_status launch_transpose(const float *in, float *out, long long nstates, cudaStream_t stream) {
+    if (nstates <= 0) return LA_OK;
+    const int tiles = (la::D / la::TRANSPOSE_TILE) * (la::D / la::TRANSPOSE_TILE);
+    la::la_state_transpose_kernel<<<dim3((unsigned)nstates, tiles), 256, 0, stream>>>(in, out);
+    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    ++g_launches;
+    return LA_OK;
+}
+
+// Workspace of la_prefill_backward: one prefill workspace (reused by the
+// three scans, which run in stream order), one la_kv_aggregate workspace and
+// three [B, H, D, D] fp32 states.
+struct BwdLayout {
+    size_t prefill, agg, st0, st1, st2, total;
+};
+
+BwdLayout bwd_layout(int B, int N, int H) {
+    BwdLayout w;
+    const long long T = (long long)B * N;
+    const int L = choose_seg_len(B, T, H);
+    const size_t pre = ws_layout(gmax_for(B, T, L), H).total;
+    const size_t agg = agg_ws_bytes(agg_plan((long long)B * H, N));
+    const size_t st = (size_t)B * H * la::D * la::D * sizeof(float);
+    w.prefill = 0;
+    w.agg = round_up(pre, 256);
+    w.st0 = w.agg + round_up(agg, 256);
+    w.st1 = w.st0 + round_up(st, 256);
+    w.st2 = w.st1 + round_up(st, 256);
+    w.total = w.st2 + st;
+    return w;
+}
 
 }  // namespace
 
@@ -498,6 +536,94 @@ la_status la_kv_aggregate(const void *k, const void *v, int B, int N, int H, int
     return LA_OK;
 }
 
+size_t la_prefill_backward_workspace_size(int B, int N, int H, int d) {
+    (void)d;
+    if (B <= 0 || N < 0 || H <= 0) return la::HDR_BYTES;
+    return bwd_layout(B, N, H).total;
+}
+
+la_status la_prefill_backward(const void *q, const void *k, const void *v, const void *dout, int B, int N, int H,
+                              int d, const float *state_in, const float *dstate_out, void *dq, void *dk, void *dv,
+                              la_dtype grad_dtype, float *dstate_in, void *workspace, size_t ws_bytes,
+                              cudaStream_t stream) {
+    la_status st = check_common(H, d, 0, grad_dtype);
+    if (st != LA_OK) return st;
+    if (B < 0 || N < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (B == 0) return LA_OK;
+    const long long T = (long long)B * N;
+    if (T > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return LA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[10] = {q, k, v, dout, dq, dk, dv, state_in, dstate_out, dstate_in};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+    const size_t esz = grad_dtype == LA_FP32 ? 4 : 2;
+    const size_t n_in = (size_t)T * H * la::D * 2, n_g = (size_t)T * H * la::D * esz;
+    const size_t n_state = (size_t)B * H * la::D * la::D * 4;
+    const void *ins[4] = {q, k, v, dout};
+    void *gs[3] = {dq, dk, dv};
+    for (int i = 0; i < 3; ++i) {
+        void *g = gs[i];
+        for (const void *p : ins)
+            if (ranges_overlap(g, n_g, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+        for (int j = i + 1; j < 3; ++j)
+            if (ranges_overlap(g, n_g, gs[j], n_g)) return LA_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(g, n_g, dstate_in, n_state) || ranges_overlap(g, n_g, state_in, n_state) ||
+            ranges_overlap(g, n_g, dstate_out, n_state))
+            return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (ranges_overlap(dstate_in, n_state, state_in, n_state) || ranges_overlap(dstate_in, n_state, dstate_out, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+    const BwdLayout w = bwd_layout(B, N, H);
+    if (!workspace || ws_bytes < w.total) return LA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return LA_ERR_INVALID_ARGUMENT;
+    for (const void *p : ptrs)
+        if (p && ranges_overlap(workspace, w.total, p, p == q || p == k || p == v || p == dout ? n_in
+                                                       : (p == dq || p == dk || p == dv ? n_g : n_state)))
+            return LA_ERR_INVALID_ARGUMENT;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *ws_pre = ws + w.prefill;
+    const size_t pre_bytes = w.agg - w.prefill;
+    void *ws_agg = ws + w.agg;
+    const size_t agg_bytes = w.st0 - w.agg;
+    float *A = reinterpret_cast<float *>(ws + w.st0);
+    float *Bs = reinterpret_cast<float *>(ws + w.st1);
+    float *C = reinterpret_cast<float *>(ws + w.st2);
+    const long long nstates = (long long)B * H;
+
+    // dQ: a forward scan of (q, k, v) = (dO, V, K) from S_in^T
+    //     dq_t = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T
+    if (state_in && (st = launch_transpose(state_in, A, nstates, stream)) != LA_OK) return st;
+    st = prefill_impl(dout, v, k, nullptr, N, B, T, N, H, d, 0, state_in ? A : nullptr, dq, grad_dtype, nullptr,
+                      ws_pre, pre_bytes, stream);
+    if (st != LA_OK) return st;
+    // dK: an ANTI scan of (q, k, v) = (V, dO, Q) from W_k = sum_t g_t^T q_t + G^T
+    //     dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
+    if ((st = la_kv_aggregate(dout, q, B, N, H, d, Bs, ws_agg, agg_bytes, stream)) != LA_OK) return st;
+    const float *s0k = Bs;
+    if (dstate_out) {
+        if ((st = launch_transpose(dstate_out, A, nstates, stream)) != LA_OK) return st;
+        if ((st = la_state_prefix(Bs, 1, A, A, (int)nstates, d, stream)) != LA_OK) return st;
+        s0k = A;
+    }
+    st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, s0k, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
+                      stream, nullptr, 0, true);
+    if (st != LA_OK) return st;
+    // dV: an ANTI scan of (q, k, v) = (K, Q, dO) from W_v = sum_t q_t^T g_t + G
+    //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t = sum_{t >= s} (q_t . k_s) g_t + k_s G
+    //     and dS_in = W_v
+    if ((st = la_kv_aggregate(q, dout, B, N, H, d, C, ws_agg, agg_bytes, stream)) != LA_OK) return st;
+    const float *s0v = C;
+    if (dstate_out) {
+        if ((st = la_state_prefix(C, 1, dstate_out, Bs, (int)nstates, d, stream)) != LA_OK) return st;
+        s0v = Bs;
+    }
+    st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
+                      stream, nullptr, 0, true);
+    if (st != LA_OK) return st;
+    if (dstate_in) return la_state_prefix(nullptr, 0, s0v, dstate_in, (int)nstates, d, stream);
+    return LA_OK;
+}
+
 la_status la_state_prefix(const float *parts, int count, const float *state_in, float *out, int nstates, int d,
                           cudaStream_t stream) {
     if (d <= 0 || nstates < 0 || count < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -660,12 +786,12 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.inject = g_inject.load();
     pp.seg_len = L;
     pp.status = status;
-    if (cudaFuncSetAttribute(la::la_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(la::la_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              la::PREFILL_SMEM) != cudaSuccess)
         return LA_ERR_CUDA;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    la::la_prefill_kernel<false><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;

@@ -21,6 +21,17 @@
 //       out = O (bf16 or fp32)             a7
 //   and, for the last segment, the final state S goes to state_out.
 //
+// The kernel is a template on ANTI.  ANTI = false is the operation above.
+// ANTI = true computes, from a state S_0 passed as state_in,
+//       o_t = q_t (S_0 - sum_{s < t} k_s^T v_s)
+//           = q_t S_0 - sum_{s < t} (q_t . k_s) v_s
+// -- an exclusive mask (s < t) and the V operand negated in a4, a6 and
+// phase A (bit 14 of the MMA instruction descriptor) -- which is how the
+// gradients dK and dV, sums over later tokens, are formed in one forward
+// sweep: with S_0 the sum over all tokens, S_0 minus the earlier tokens
+// leaves the later ones.  ANTI always uses the hi + lo split of S for a5,
+// since S starts at its largest.
+//
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
 //               loads Q
@@ -306,6 +317,7 @@ __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane
     return item[IT_VALID] != 0;
 }
 
+template <bool ANTI>
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
@@ -389,7 +401,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     item[IT_J] = seg.w & (SEG_LAST - 1);
                     const int jj = seg.w & (SEG_LAST - 1);
                     const long long seg_end = (long long)jj * p.seg_len + (seg.z - seg.y);
-                    item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) | (seg_end > LA_LO_SPLIT_FROM ? ITF_LO : 0);
+                    item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) |
+                                     ((ANTI || seg_end > LA_LO_SPLIT_FROM) ? ITF_LO : 0);
                 }
                 mbar_arrive(&cb->item_full[islot]);
                 ++it;
@@ -475,8 +488,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         constexpr uint32_t ID_QK = idesc_bf16_f32(BLK, BLK, 0, 0);    // Q (K-major) x K (K-major)
         constexpr uint32_t ID_QS = idesc_bf16_f32(BLK, D / 2, 0, 1);  // Q (K-major) x S half (MN-major)
         constexpr uint32_t ID_QF = idesc_bf16_f32(BLK, D, 0, 1);      // Q (K-major) x S (MN-major)
-        constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1);        // K^T (MN) x V (MN)
-        constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1);      // P (TMEM) x V (MN)
+        constexpr uint32_t NEG_V = ANTI ? IDESC_NEGATE_B : 0u;        // ANTI: the V operand negated
+        constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1) | NEG_V;  // K^T (MN) x V (MN)
+        constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1) | NEG_V;  // P (TMEM) x V (MN)
         // The whole warp runs this loop in step: every lane holds the same
         // counters, barrier probes are combined with __all_sync, and each MMA or
         // commit is issued by the lane that elect.sync picks.
@@ -657,14 +671,15 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int q4 = warp & 3;               // TMEM lane quarter this warp may access
         const int r = q4 * 32 + lane;          // tile row = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+        constexpr int EXCL = ANTI ? 1 : 0;     // key s kept iff s + EXCL <= t
         uint32_t it = 0, blk_n = 0;
         bool ok = true;
         int item[8];
         while (ok && next_item(it, item, lane, p, cb)) {
             const int nblk = (item[IT_TOK1] - item[IT_TOK0] + BLK - 1) / BLK;
             for (int b = 0; b < nblk; ++b) {
-                // P = bf16(Sc ⊙ M), inclusive mask, packed two per 32-bit column
-                // over the first 64 score columns
+                // P = bf16(Sc ⊙ M), inclusive mask (exclusive under ANTI), packed
+                // two per 32-bit column over the first 64 score columns
                 const uint32_t bn = blk_n + b, tsc = trow + TM_SC;
                 if (!warp_wait(&cb->sc_full, bn & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
@@ -681,7 +696,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                         for (int w = 0; w < 32; ++w) {
                             const int c = hf * 64 + 2 * w;
-                            x[w] = bf16x2_round(c <= r ? x[2 * w] : 0u, c + 1 <= r ? x[2 * w + 1] : 0u);
+                            x[w] = bf16x2_round(c + EXCL <= r ? x[2 * w] : 0u, c + 1 + EXCL <= r ? x[2 * w + 1] : 0u);
                         }
                     }
                     tmem_st32(tsc + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));

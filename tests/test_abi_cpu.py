@@ -185,3 +185,32 @@ def test_sequence_parallel_argument_errors(L):
     assert L.la_state_prefix(fake, 2, None, V((1 << 30) + 4), 4, 128, None) == bad            # misaligned
     assert L.la_state_prefix(fake, 2, V((1 << 30) + 1024), V(1 << 30), 4, 128, None) == bad   # partial overlap
     assert L.la_state_prefix(fake, 2, None, fake, 0, 128, None) == la.LA_OK
+
+
+def test_backward_argument_errors(L):
+    """la_prefill_backward rejects bad arguments before launching."""
+    V = ctypes.c_void_p
+    bad = la.LA_ERR_INVALID_ARGUMENT
+    base = 1 << 32
+    B, N, H = 1, 100, 2
+    n = B * N * H * 128 * 2                      # bytes of one bf16 tensor
+    q, k, v, g = (V(base + i * n) for i in range(4))
+    dq, dk, dv = (V(base + (4 + i) * n) for i in range(3))
+    ws_size = L.la_prefill_backward_workspace_size(B, N, H, 128)
+    assert ws_size >= L.la_prefill_workspace_size(B, N, H, 128, 0) + 3 * B * H * 128 * 128 * 4
+    ws = V(base + 64 * n)
+    args = lambda **kw: dict(dict(q=q, k=k, v=v, g=g, B=B, N=N, H=H, d=128, sin=None, dsout=None, dq=dq, dk=dk,
+                                  dv=dv, gd=0, dsin=None, ws=ws, wsb=ws_size, s=None), **kw)
+    call = lambda a: L.la_prefill_backward(*a.values())
+    assert call(args(d=64)) == la.LA_ERR_UNSUPPORTED
+    assert call(args(gd=7)) == bad                               # unknown gradient dtype
+    assert call(args(N=-1)) == bad
+    assert call(args(g=None)) == bad                             # no dout
+    assert call(args(dk=dq)) == bad                              # two gradients in one buffer
+    assert call(args(dv=q)) == bad                               # a gradient over an input
+    assert call(args(dq=V(base + 4 * n + 8))) == bad             # misaligned
+    assert call(args(ws=None)) == la.LA_ERR_WORKSPACE
+    assert call(args(wsb=ws_size - 1)) == la.LA_ERR_WORKSPACE
+    assert call(args(ws=V(base + 64 * n + 16))) == bad           # workspace not 256-byte aligned
+    assert call(args(ws=V(base + 5 * n))) == bad                 # workspace over a gradient
+    assert call(args(B=0)) == la.LA_OK                           # nothing to do
