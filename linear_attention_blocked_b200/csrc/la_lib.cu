@@ -212,6 +212,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.incl = reinterpret_cast<float *>(ws + w.incl);
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
+    pp.anti_lo = anti && max_seqlen > LA_LO_SPLIT_FROM;
     pp.seg_len = L;
     pp.status = status;
 
@@ -596,27 +597,22 @@ la_status la_prefill_backward(const void *q, const void *k, const void *v, const
     st = prefill_impl(dout, v, k, nullptr, N, B, T, N, H, d, 0, state_in ? A : nullptr, dq, grad_dtype, nullptr,
                       ws_pre, pre_bytes, stream);
     if (st != LA_OK) return st;
-    // dK: an ANTI scan of (q, k, v) = (V, dO, Q) from W_k = sum_t g_t^T q_t + G^T
-    //     dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
-    if ((st = la_kv_aggregate(dout, q, B, N, H, d, Bs, ws_agg, agg_bytes, stream)) != LA_OK) return st;
-    const float *s0k = Bs;
-    if (dstate_out) {
-        if ((st = launch_transpose(dstate_out, A, nstates, stream)) != LA_OK) return st;
-        if ((st = la_state_prefix(Bs, 1, A, A, (int)nstates, d, stream)) != LA_OK) return st;
-        s0k = A;
-    }
-    st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, s0k, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
-                      stream, nullptr, 0, true);
-    if (st != LA_OK) return st;
-    // dV: an ANTI scan of (q, k, v) = (K, Q, dO) from W_v = sum_t q_t^T g_t + G
-    //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t = sum_{t >= s} (q_t . k_s) g_t + k_s G
-    //     and dS_in = W_v
+    // the two starting states: W_v = sum_t q_t^T g_t + G (= dS_in) and
+    // W_k = sum_t g_t^T q_t + G^T = W_v^T -- one sum over (q, dout) serves both
     if ((st = la_kv_aggregate(q, dout, B, N, H, d, C, ws_agg, agg_bytes, stream)) != LA_OK) return st;
     const float *s0v = C;
     if (dstate_out) {
         if ((st = la_state_prefix(C, 1, dstate_out, Bs, (int)nstates, d, stream)) != LA_OK) return st;
         s0v = Bs;
     }
+    if ((st = launch_transpose(s0v, A, nstates, stream)) != LA_OK) return st;
+    // dK: an ANTI scan of (q, k, v) = (V, dO, Q) from W_k
+    //     dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
+    st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, A, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
+                      stream, nullptr, 0, true);
+    if (st != LA_OK) return st;
+    // dV: an ANTI scan of (q, k, v) = (K, Q, dO) from W_v
+    //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t = sum_{t >= s} (q_t . k_s) g_t + k_s G
     st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
                       stream, nullptr, 0, true);
     if (st != LA_OK) return st;
@@ -784,6 +780,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.incl = reinterpret_cast<float *>(ws + w.incl);
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
+    pp.anti_lo = 0;
     pp.seg_len = L;
     pp.status = status;
     if (cudaFuncSetAttribute(la::la_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,

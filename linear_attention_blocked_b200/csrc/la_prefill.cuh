@@ -29,8 +29,10 @@
 // phase A (bit 14 of the MMA instruction descriptor) -- which is how the
 // gradients dK and dV, sums over later tokens, are formed in one forward
 // sweep: with S_0 the sum over all tokens, S_0 minus the earlier tokens
-// leaves the later ones.  ANTI always uses the hi + lo split of S for a5,
-// since S starts at its largest.
+// leaves the later ones.  S starts at the sum over the whole sequence, as
+// large as the forward's state at its end, so ANTI hands S to a5 as hi + lo
+// exactly when the forward would need it somewhere in the sequence: when the
+// host sets p.anti_lo (sequences longer than LA_LO_SPLIT_FROM tokens).
 //
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
@@ -126,6 +128,7 @@ struct PrefillParams {
     int seg_len;            // tokens per segment (the last one of a sequence may be shorter)
     unsigned long long wait_limit_ns;
     int inject;
+    int anti_lo;            // ANTI: hand S to a5 as hi + lo (the sequences are long)
     int *status;            // sticky device status word
 };
 
@@ -402,7 +405,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const int jj = seg.w & (SEG_LAST - 1);
                     const long long seg_end = (long long)jj * p.seg_len + (seg.z - seg.y);
                     item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) |
-                                     ((ANTI || seg_end > LA_LO_SPLIT_FROM) ? ITF_LO : 0);
+                                     ((ANTI ? p.anti_lo != 0 : seg_end > LA_LO_SPLIT_FROM) ? ITF_LO : 0);
                 }
                 mbar_arrive(&cb->item_full[islot]);
                 ++it;
