@@ -2,8 +2,9 @@
 the fp64 oracle's gradients, element by element, on seeded inputs: ragged
 tails, several cross-SM segments, carried-in states and state gradients, bf16
 and fp32 gradients, sampled heads at 4096 tokens, and at the single-sequence
-prefill workload (B=1, H=64, N=32768) the first and last 4096 rows of two
-heads, with the rest of the sequence summarised by the oracle's forward."""
+prefill workload (B=1, H=64, N=32768) and at 131072 tokens the first and
+last rows of sampled heads, with the rest of the sequence summarised by the
+oracle's forward."""
 import numpy as np
 import pytest
 import torch
@@ -74,22 +75,23 @@ def test_backward_bf16_sampled_heads(oracle_mod):
     _check_all(got, ref, B, N, len(heads), True, "bf16 sampled heads")
 
 
-def test_backward_full_size_sampled_rows(oracle_mod):
-    """B=1, H=64, N=32768 (the single-sequence prefill workload), bf16
-    gradients, two heads, the first and the last 4096 rows against the
-    oracle.  The rows' gradients depend on the rest of the sequence only
-    through d x d sums, which the oracle's forward supplies:
-      first rows: dk_s, dv_s also see the later tokens t >= 4096, whose share
-        is v_s G^T and k_s G with G = sum_{t >= 4096} q_t^T g_t -- the
-        oracle's state from zero over those tokens with (k, v) = (q, g) --
-        passed to the oracle's backward of the first rows as dS_out;
-      last rows: dq_t also sees the earlier tokens through S_in = their
-        k^T v sum, the oracle's final state over them.
+@pytest.mark.parametrize("N,H,heads,R", [(32768, 64, [0, 37], 4096), (131072, 2, [0, 1], 2048)])
+def test_backward_long_sequence_sampled_rows(oracle_mod, N, H, heads, R):
+    """B=1 and N=32768, H=64 (the single-sequence prefill workload) or
+    N=131072, H=2 (past the length where the scans split their state into
+    bf16 hi + lo): bf16 gradients of the sampled heads on the first and the
+    last R rows against the oracle.  The rows' gradients depend on the rest
+    of the sequence only through d x d sums, which the oracle's forward
+    supplies:
+      first rows: dk_s, dv_s also see the later tokens t >= R, whose share is
+        v_s G^T and k_s G with G = sum_{t >= R} q_t^T g_t -- the oracle's
+        state from zero over those tokens with (k, v) = (q, g) -- passed to
+        the oracle's backward of the first rows as dS_out;
+      last rows: dq_t also sees the earlier tokens through S_in = their k^T v
+        sum, the oracle's final state over them.
     dS_in equals la_kv_aggregate(q, dout) bit for bit."""
-    B, N, H = 1, 32768, 64
-    R = 4096
-    heads = [0, 37]
-    q, k, v, g = _inputs(B, N, H, seed=960)
+    B = 1
+    q, k, v, g = _inputs(B, N, H, seed=960 + H)
     dq, dk, dv, dsin = la.prefill_backward(q, k, v, g)
     assert la.get_device_status() == la.LA_OK
     assert torch.equal(dsin, la.kv_aggregate(q, g))
@@ -100,10 +102,10 @@ def test_backward_full_size_sampled_rows(oracle_mod):
     ref = oracle_mod.backward(bits(q, 0, R), bits(k, 0, R), bits(v, 0, R), bits(g, 0, R), cu(R), heads=heads,
                               dstate_out=G)
     for name, x, y in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
-        check_out(to_np(x[0, :R, heads]), y, bf16_out=True, what=f"first rows {name}")
+        check_out(to_np(x[0, :R, heads]), y, bf16_out=True, what=f"N={N} first rows {name}")
     # last rows
     _, S = oracle_mod.recurrent(bits(q, 0, N - R), bits(k, 0, N - R), bits(v, 0, N - R), cu(N - R), heads=heads)
     ref = oracle_mod.backward(bits(q, N - R, N), bits(k, N - R, N), bits(v, N - R, N), bits(g, N - R, N), cu(R),
                               heads=heads, state_in=S)
     for name, x, y in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
-        check_out(to_np(x[0, N - R:, heads]), y, bf16_out=True, what=f"last rows {name}")
+        check_out(to_np(x[0, N - R:, heads]), y, bf16_out=True, what=f"N={N} last rows {name}")
