@@ -453,7 +453,7 @@ def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
     return {"workload": "prefill backward B=1 H=64 N=32768 d=128, bf16 dq/dk/dv + fp32 dS_in",
             "ms_per_call": ms, "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (three scans) + la_kv_aggregate_kernel (two sums)",
+                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (three scans) + la_kv_aggregate_kernel (one sum)",
                          "traffic": None, "bytes_per_launch": byts,
                          "duration": "CUDA events around each la_prefill_backward call (about ten kernels)"}}
 
