@@ -15,6 +15,7 @@ ABI (include/lightning_attn.h).  Entry points:
   state_prefix(parts, count, state_in)       la_state_prefix: state_in + parts[0] + ... + parts[count-1]
   lasp_prefill(q, k, v, group=...)           sequence parallelism across ranks (seqpar.py)
   lasp_prefill_varlen(q, k, v, cu, bounds)   the same for a packed batch cut at any token
+  lasp_prefill_backward(q, k, v, dout, ...)  gradients of lasp_prefill across ranks
   prefill_backward(q, k, v, dout, ...)       la_prefill_backward: dq, dk, dv, dS_in
   get_device_status()                        la_get_device_status
 """
@@ -26,5 +27,6 @@ from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, prefill_backwa
                        prefill, prefill_varlen, prefill_varlen_slots,
                        set_segment_len, set_wait_limit_ns, state_prefix, status_string,
                        varlen_workspace_size, workspace_size)
-from .seqpar import lasp_prefill, lasp_prefill_varlen, plan_varlen_rank, split_tokens  # noqa: F401,E402
+from .seqpar import (lasp_prefill, lasp_prefill_backward, lasp_prefill_varlen, plan_varlen_rank,  # noqa: F401,E402
+                     split_tokens)
 from .serving import BatchPlan, plan_batch  # noqa: F401,E402

@@ -24,8 +24,15 @@ carried-in state.  The planning is plain host arithmetic on cu_seqlens
 (plan_varlen_rank); the device steps are la_kv_aggregate, la_state_prefix
 and la_prefill_varlen.
 
+Gradients across ranks (lasp_prefill_backward): a rank's tokens see the
+earlier ranks only through the state they hand on and the later ranks only
+through that state's gradient, so each rank gathers two d x d sums per
+(sequence, head) from every rank and runs la_prefill_backward on its own
+tokens from the two.
+
 The device steps run in the CUDA library (la_kv_aggregate, la_state_prefix,
-la_prefill, la_prefill_varlen); the collective is torch.distributed's.
+la_prefill, la_prefill_varlen, la_prefill_backward); the collective is
+torch.distributed's.
 """
 from __future__ import annotations
 
@@ -53,6 +60,11 @@ class DeviceOps:
     def prefill(q, k, v, state_in, out_dtype):
         out, _ = _binding.prefill(q, k, v, state_in=state_in, out_dtype=out_dtype, want_state=False)
         return out
+
+    @staticmethod
+    def prefill_backward(q, k, v, dout, state_in, dstate_out, grad_dtype):
+        return _binding.prefill_backward(q, k, v, dout, state_in=state_in, dstate_out=dstate_out,
+                                         grad_dtype=grad_dtype, want_dstate_in=False)[:3]
 
     @staticmethod
     def prefill_varlen(q, k, v, cu_seqlens, max_seqlen, state_in, out_dtype):
@@ -85,6 +97,53 @@ def lasp_prefill(q, k, v, group=None, state_in=None, out_dtype=torch.bfloat16, w
     out = ops.prefill(q, k, v, prefix, out_dtype)
     final = ops.state_prefix(parts, world, state_in) if want_state else None
     return out, final
+
+
+# --------------------------------------------------------------------------- gradients
+def backward_local_sums(q, k, v, dout, ops=DeviceOps):
+    """Step 1 of lasp_prefill_backward on one rank: the rank's sums
+    A_r = sum k_t^T v_t (for the forward prefix of later ranks) and
+    B_r = sum q_t^T g_t (for the state gradient of earlier ranks)."""
+    return ops.kv_aggregate(k, v), ops.kv_aggregate(q, dout)
+
+
+def backward_local_grads(rank, world, a_parts, b_parts, q, k, v, dout, state_in=None, dstate_out=None,
+                         grad_dtype=torch.bfloat16, ops=DeviceOps):
+    """Step 3 on one rank, given every rank's sums (a_parts, b_parts: [W, B,
+    H, d, d], rank order).  The rank's tokens see the earlier ranks only
+    through their state, S_in + A_0 + ... + A_{r-1}, and the later ranks only
+    through the gradient of the state they hand on, G + B_{r+1} + ... +
+    B_{W-1}; so its gradients are la_prefill_backward of its own tokens with
+    those two.  Returns (dq, dk, dv, dS_in of the whole sequences)."""
+    prefix = ops.state_prefix(a_parts[:rank], rank, state_in)
+    later = b_parts[rank + 1:]
+    suffix = ops.state_prefix(later, world - rank - 1, dstate_out)
+    dq, dk, dv = ops.prefill_backward(q, k, v, dout, prefix, suffix, grad_dtype)
+    dstate_in = ops.state_prefix(b_parts, world, dstate_out)  # sum over all tokens of q^T g, + G
+    return dq, dk, dv, dstate_in
+
+
+def lasp_prefill_backward(q, k, v, dout, group=None, state_in=None, dstate_out=None, grad_dtype=torch.bfloat16,
+                          ops=DeviceOps):
+    """Gradients of lasp_prefill on this rank's part [B, n_r, H, d] of every
+    sequence, for dL/dout (this rank's rows) and dL/dS_out of the final
+    state of the whole sequences (dstate_out, the same on every rank, or
+    None).  Returns (dq, dk, dv for this rank's tokens, dS_in of the whole
+    sequences, the same on every rank).  One AllGather of each rank's two
+    d x d sums per (sequence, head)."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if q.dim() != 4:
+        raise ValueError("q must be [B, n_r, H, d]")
+    B, _, H, d = q.shape
+    a, b = backward_local_sums(q, k, v, dout, ops)
+    parts = []
+    for local in (a, b):
+        gathered = local.new_empty((world * B, H, d, d))  # rank-major
+        dist.all_gather_into_tensor(gathered, local.contiguous(), group=group)
+        parts.append(gathered.view(world, B, H, d, d))
+    return backward_local_grads(rank, world, parts[0], parts[1], q, k, v, dout, state_in, dstate_out, grad_dtype,
+                                ops)
 
 
 # --------------------------------------------------------------------------- packed batches

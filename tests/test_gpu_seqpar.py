@@ -151,6 +151,41 @@ def test_emulated_ranks_on_a_packed_batch(oracle_mod, lens, world):
     check_state(to_np(final), rst, what="final states")
 
 
+def test_emulated_ranks_gradients(oracle_mod):
+    """Gradients across three ranks (parts of 700, 1500 and 829 tokens), run
+    one after the other on this GPU through the same two steps
+    lasp_prefill_backward runs on each rank, with stacks of the ranks' sums
+    standing in for the AllGathers; fp32 gradients against the oracle's
+    gradients of the whole sequences, with a carried-in state and a state
+    gradient."""
+    from linear_attention_blocked_b200 import seqpar
+    B, H = 2, 3
+    lens = [700, 1500, 829]
+    N = sum(lens)
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=331, device="cuda")
+    g, _, _ = la_inputs.qkv((B, N, H, D), seed=332, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(333)
+    sin = torch.randn((B, H, D, D), generator=gen, device="cuda") * 0.1
+    gs = torch.randn((B, H, D, D), generator=gen, device="cuda") * 0.05
+    bounds = np.concatenate([[0], np.cumsum(lens)])
+    shard = lambda t, r: t[:, bounds[r]:bounds[r + 1]].contiguous()  # noqa: E731
+    W = len(lens)
+    sums = [seqpar.backward_local_sums(shard(q, r), shard(k, r), shard(v, r), shard(g, r)) for r in range(W)]
+    a_parts = torch.stack([a for a, _ in sums])
+    b_parts = torch.stack([b for _, b in sums])
+    grads = [seqpar.backward_local_grads(r, W, a_parts, b_parts, shard(q, r), shard(k, r), shard(v, r), shard(g, r),
+                                         sin, gs, torch.float32) for r in range(W)]
+    assert la.get_device_status() == la.LA_OK
+    flat = lambda t: la_inputs.bits(t.reshape(B * N, H, D))  # noqa: E731
+    ref = oracle_mod.backward(flat(q), flat(k), flat(v), flat(g), _cu(B, N), state_in=to_np(sin),
+                              dstate_out=to_np(gs))
+    for i, name in enumerate(("dq", "dk", "dv")):
+        got = torch.cat([gr[i] for gr in grads], dim=1).reshape(B * N, H, D)
+        check_out(to_np(got), ref[i], bf16_out=False, what=f"ranks {name}")
+    for gr in grads:
+        check_state(to_np(gr[3]), ref[3], what="dS_in")
+
+
 _ONE_RANK = r"""
 import os, sys
 sys.path.insert(0, os.environ["LA_ROOT"])
@@ -174,6 +209,11 @@ sinp = torch.randn((3, H, D, D), device="cuda") * 0.1
 outp, stp, plan = la.seqpar.lasp_prefill_varlen(qp, kp, vp, cu, np.array([0, 2000]), state_in=sinp)
 refp, rstp = la.prefill_varlen(qp, kp, vp, torch.from_numpy(cu).cuda(), 1300, state_in=sinp)
 same = same and torch.equal(outp, refp) and torch.equal(stp, rstp) and bool(plan.ends_here.all())
+g = torch.randn_like(q.float()).mul(0.1).bfloat16()
+gs = torch.randn((B, H, D, D), device="cuda") * 0.05
+bw = la.lasp_prefill_backward(q, k, v, g, state_in=sin, dstate_out=gs)
+bref = la.prefill_backward(q, k, v, g, state_in=sin, dstate_out=gs)
+same = same and all(torch.equal(x, y) for x, y in zip(bw, bref))
 dist.destroy_process_group()
 print("RESULT", int(same), rel, la.get_device_status())
 """
@@ -182,8 +222,9 @@ print("RESULT", int(same), rel, la.get_device_status())
 def test_lasp_prefill_under_one_rank_nccl_group():
     """With one rank the global prefix is the carried-in state itself, so the
     output must equal la_prefill's bit for bit (and the packed form's outputs
-    and states those of la_prefill_varlen); the final state of the
-    equal-length form differs from la_prefill's only in summation order."""
+    and states those of la_prefill_varlen, the gradients those of
+    la_prefill_backward); the final state of the equal-length form differs
+    from la_prefill's only in summation order."""
     import socket
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
@@ -192,6 +233,6 @@ def test_lasp_prefill_under_one_rank_nccl_group():
     res = subprocess.run([sys.executable, "-c", _ONE_RANK], env=env, capture_output=True, text=True, timeout=300)
     assert res.returncode == 0, res.stderr[-2000:]
     line = [x for x in res.stdout.splitlines() if x.startswith("RESULT")][-1].split()
-    assert line[1] == "1", "output differs from la_prefill / la_prefill_varlen"
+    assert line[1] == "1", "output differs from la_prefill / la_prefill_varlen / la_prefill_backward"
     assert float(line[2]) <= 1e-5
     assert int(line[3]) == la.LA_OK

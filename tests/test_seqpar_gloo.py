@@ -3,7 +3,9 @@
 order, the global prefix of the ranks before this one, the local scan seeded
 with it -- reproduces the oracle's result for the whole sequences, and so
 does lasp_prefill_varlen on packed batches cut at arbitrary token positions
-(sequences spanning several ranks, empty sequences, empty ranks).  The device
+(sequences spanning several ranks, empty sequences, empty ranks), and
+lasp_prefill_backward reproduces the oracle's gradients of the whole
+sequences.  The device
 steps are host stand-ins built from the oracle (fp64), so what is checked
 here is the rank logic; the CUDA steps are checked on the GPU."""
 import os
@@ -62,6 +64,14 @@ class _HostOps:
         V, _ = _HostOps._packed(v)
         out, _ = oracle.recurrent(Q, K, V, cu, state_in=state_in.numpy())
         return torch.from_numpy(out).reshape(B, n, H, d)
+
+    @staticmethod
+    def prefill_backward(q, k, v, dout, state_in, dstate_out, grad_dtype):
+        import oracle
+        B, n, H, d = q.shape
+        (Q, cu), (K, _), (V, _), (G, _) = (_HostOps._packed(t) for t in (q, k, v, dout))
+        dq, dk, dv, _ = oracle.backward(Q, K, V, G, cu, state_in=state_in.numpy(), dstate_out=dstate_out.numpy())
+        return tuple(torch.from_numpy(x).reshape(B, n, H, d) for x in (dq, dk, dv))
 
     @staticmethod
     def prefill_varlen(q, k, v, cu_seqlens, max_seqlen, state_in, out_dtype):
@@ -159,5 +169,47 @@ def test_varlen_ranks_reproduce_the_packed_batch(tmp_path, oracle_mod, lens, bou
     bounds = np.asarray(bounds if bounds is not None else seqpar.split_tokens(T, world))
     result = tmp_path / "result.txt"
     mp.start_processes(_varlen_worker, args=(world, _free_port(), lens, bounds, str(result)), nprocs=world,
+                       join=True, start_method="spawn")
+    assert result.read_text() == "ok"
+
+
+def _backward_worker(rank, world, port, lens, result_path):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from linear_attention_blocked_b200 import seqpar
+        B, H = 2, 2
+        N = sum(lens)
+        q, k, v = la_inputs.qkv((B, N, H, D), seed=71, scale=0.5)
+        g, _, _ = la_inputs.qkv((B, N, H, D), seed=72, scale=0.5)
+        rng = np.random.default_rng(73)
+        sin = torch.from_numpy(rng.standard_normal((B, H, D, D)) * 0.3)
+        gs = torch.from_numpy(rng.standard_normal((B, H, D, D)) * 0.3)
+        a = sum(lens[:rank])
+        part = lambda t: t[:, a:a + lens[rank]].contiguous()  # noqa: E731
+        dq, dk, dv, dsin = seqpar.lasp_prefill_backward(part(q), part(k), part(v), part(g), state_in=sin,
+                                                        dstate_out=gs, ops=_HostOps)
+        shares = [None] * world
+        dist.all_gather_object(shares, tuple(x.numpy() for x in (dq, dk, dv, dsin)))
+        if rank == 0:
+            (Q, cu), (K, _), (V, _), (G, _) = (_HostOps._packed(t) for t in (q, k, v, g))
+            ref = oracle.backward(Q, K, V, G, cu, state_in=sin.numpy(), dstate_out=gs.numpy())
+            ok = True
+            for i in range(3):
+                got = np.concatenate([sh[i] for sh in shares], axis=1).reshape(B * N, H, D)
+                ok &= bool(np.abs(got - ref[i]).max() <= 1e-10 * np.abs(ref[i]).max())
+            for sh in shares:
+                ok &= bool(np.abs(sh[3] - ref[3]).max() <= 1e-10 * np.abs(ref[3]).max())
+            with open(result_path, "w") as fh:
+                fh.write("ok" if ok else "mismatch")
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("lens", [[40, 77], [130, 1, 59]])
+def test_backward_ranks_reproduce_the_whole_sequence(tmp_path, oracle_mod, lens):
+    result = tmp_path / "result.txt"
+    mp.start_processes(_backward_worker, args=(len(lens), _free_port(), lens, str(result)), nprocs=len(lens),
                        join=True, start_method="spawn")
     assert result.read_text() == "ok"
