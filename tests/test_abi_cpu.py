@@ -126,10 +126,21 @@ def test_segment_len_control(L):
 
 
 def test_binding_rejects_cpu_tensors():
+    """Every entry point refuses host tensors before calling the library (no
+    CPU fallback exists)."""
     import torch
     q = torch.zeros(1, 128, 1, 128, dtype=torch.bfloat16)
+    s = torch.zeros(1, 1, 128, 128)
     with pytest.raises(ValueError):
         la.prefill(q, q, q)
+    with pytest.raises(ValueError):
+        la.kv_aggregate(q, q)
+    with pytest.raises(ValueError):
+        la.prefill_backward(q, q, q, q)
+    with pytest.raises(ValueError):
+        la.state_prefix(s[None], 1)
+    with pytest.raises(ValueError):
+        la.decode_step(q[:, 0], q[:, 0], q[:, 0], s)
 
 
 def test_slot_and_mixed_argument_errors(L):
