@@ -101,7 +101,8 @@ def lasp_prefill(q, k, v, group=None, state_in=None, out_dtype=torch.bfloat16, w
 
 # --------------------------------------------------------------------------- gradients
 def backward_local_sums(q, k, v, dout, ops=DeviceOps):
-    """Step 1 of lasp_prefill_backward on one rank: the rank's sums
+    """Step 1 of lasp_prefill_backward on one rank (step 2 gathers the
+    results of every rank): the rank's sums
     A_r = sum k_t^T v_t (for the forward prefix of later ranks) and
     B_r = sum q_t^T g_t (for the state gradient of earlier ranks)."""
     return ops.kv_aggregate(k, v), ops.kv_aggregate(q, dout)
@@ -129,8 +130,9 @@ def lasp_prefill_backward(q, k, v, dout, group=None, state_in=None, dstate_out=N
     sequence, for dL/dout (this rank's rows) and dL/dS_out of the final
     state of the whole sequences (dstate_out, the same on every rank, or
     None).  Returns (dq, dk, dv for this rank's tokens, dS_in of the whole
-    sequences, the same on every rank).  One AllGather of each rank's two
-    d x d sums per (sequence, head)."""
+    sequences, the same on every rank).  Two AllGathers, one for each of the
+    rank's two d x d sums per (sequence, head); step 2 between
+    backward_local_sums and backward_local_grads."""
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     if q.dim() != 4:
