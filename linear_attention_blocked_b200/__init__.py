@@ -17,6 +17,8 @@ ABI (include/lightning_attn.h).  Entry points:
   lasp_prefill_varlen(q, k, v, cu, bounds)   the same for a packed batch cut at any token
   lasp_prefill_backward(q, k, v, dout, ...)  gradients of lasp_prefill across ranks
   prefill_backward(q, k, v, dout, ...)       la_prefill_backward: dq, dk, dv, dS_in
+  prefill_from_host(q, k, v, ...)            la_prefill of pinned host tensors, chunks pipelined
+                                             over copy-in / scan / copy-out streams
   get_device_status()                        la_get_device_status
 """
 from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, prefill_backward, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
@@ -30,3 +32,4 @@ from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, prefill_backwa
 from .seqpar import (lasp_prefill, lasp_prefill_backward, lasp_prefill_varlen, plan_varlen_rank,  # noqa: F401,E402
                      split_tokens)
 from .serving import BatchPlan, plan_batch  # noqa: F401,E402
+from .streaming import make_buffers, prefill_from_host  # noqa: F401,E402
