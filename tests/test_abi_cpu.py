@@ -225,3 +225,13 @@ def test_backward_argument_errors(L):
     assert call(args(ws=V(base + 64 * n + 16))) == bad           # workspace not 256-byte aligned
     assert call(args(ws=V(base + 5 * n))) == bad                 # workspace over a gradient
     assert call(args(B=0)) == la.LA_OK                           # nothing to do
+
+
+def test_host_memory_entry_point_validates_before_any_copy():
+    """prefill_from_host refuses unpinned, non-bf16 or non-contiguous host
+    inputs before touching a device."""
+    import torch
+    q = torch.zeros(1, 16, 1, 128, dtype=torch.bfloat16)
+    for bad in (q, q.float(), q[:, ::2]):
+        with pytest.raises(ValueError):
+            la.prefill_from_host(bad, bad, bad)
