@@ -13,6 +13,7 @@ from linear_attention_blocked_b200 import _build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "lightning_attn.h")
+HEADER_DIR = os.path.dirname(HEADER)
 
 
 @pytest.fixture(scope="module")
@@ -235,3 +236,38 @@ def test_host_memory_entry_point_validates_before_any_copy():
     for bad in (q, q.float(), q[:, ::2]):
         with pytest.raises(ValueError):
             la.prefill_from_host(bad, bad, bad)
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    """The boundary as a C user sees it: a C99 translation unit that includes
+    include/lightning_attn.h, takes the address of every entry point, links
+    against the built library and calls its host-only functions (status
+    strings, workspace sizes); no GPU is touched."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    _build.build()
+    lib_dir = os.path.dirname(la.library_path())
+    cuda_inc = "/usr/local/cuda/include"
+    names = declared_functions()
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"lightning_attn.h\"\n"
+        "int main(void) {\n"
+        "    const void *fns[] = {" + ", ".join(f"(const void *)&{n}" for n in names) + "};\n"
+        "    size_t ws = la_kv_aggregate_workspace_size(1, 32768, 64, 128);\n"
+        "    printf(\"%d %s %zu\\n\", (int)(sizeof fns / sizeof fns[0]), la_status_string(LA_ERR_WORKSPACE), ws);\n"
+        "    return la_prefill_workspace_size(1, 1024, 2, 128, 0) > 0 ? 0 : 1;\n"
+        "}\n")
+    exe = tmp_path / "use_abi"
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-I", HEADER_DIR, "-I", cuda_inc, str(src), "-o", str(exe),
+           "-L", lib_dir, "-llightning_attn", f"-Wl,-rpath,{lib_dir}"]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    count, rest = run.stdout.split(" ", 1)
+    assert int(count) == len(names)
+    assert "workspace" in rest and rest.strip().endswith(str(2 * 148 * 128 * 128 * 4))
