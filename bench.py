@@ -337,7 +337,7 @@ def run_cuda(args, world, rank, local):
     def e2e_step():
         # the public host-memory entry point: chunks of tokens copied in, scanned
         # and copied out on three streams, the state carried between chunks
-        la.prefill_from_host(qh, kh, vh, chunk_tokens=E2E_CHUNK, out=oh, state_out=sh, buffers=bufs)
+        la.prefill_from_host(qh, kh, vh, chunk_tokens=E2E_CHUNK, out=oh, state_out=sh, buffers=bufs, device=dev)
 
     e2e_step()
     torch.cuda.synchronize(dev)

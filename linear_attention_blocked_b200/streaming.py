@@ -44,7 +44,12 @@ def prefill_from_host(q, k, v, chunk_tokens: int = 4096, state_in=None, out=None
             raise ValueError(f"{name} must be in pinned host memory")
     if chunk_tokens <= 0:
         raise ValueError("chunk_tokens must be positive")
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if buffers is not None:
+        device = buffers["state"].device
+    elif device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    else:
+        device = torch.device(device)
     if out is None:
         out = torch.empty((B, N, H, d), dtype=out_dtype, pin_memory=True)
     if out.is_cuda or tuple(out.shape) != (B, N, H, d) or not out.is_contiguous():
