@@ -236,7 +236,11 @@ LA_API la_status la_prefill_noalloc(const void *q, const void *k, const void *v,
  *   contiguous (NULL when count == 0); state_in: fp32 [nstates][d][d] or
  *   NULL; out: fp32 [nstates][d][d], may equal state_in, must not overlap
  *   parts or partially overlap state_in.  nstates = B * H.  Asynchronous on
- *   `stream`.
+ *   `stream`.  With count == 0 it copies state_in into out (or zeroes out).
+ * Errors of both, returned before any launch: d != 128 -> LA_ERR_UNSUPPORTED;
+ * a negative size or count, a needed pointer that is NULL or not 16-byte
+ * aligned, or overlapping buffers -> LA_ERR_INVALID_ARGUMENT; a missing or
+ * short workspace -> LA_ERR_WORKSPACE.
  * ------------------------------------------------------------------------- */
 LA_API size_t la_kv_aggregate_workspace_size(int B, int N, int H, int d);
 
