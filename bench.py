@@ -8,6 +8,8 @@ iid N(0,1)*128^-0.5, fp32 accumulation, bf16 output plus the final fp32
 cross-SM segment hand-off + epilogue).  In the same run the fused batched
 decode step is timed on its own workload (256 sequences x 64 heads, fp32
 states initialised by a 4096-token prefill) and reported under "decode", and
+the packed variable-length batch (8 sequences of 1024-65536 tokens, 64
+heads) under "varlen", the 1M-token prefill (8 heads) under "long_context",
 the local-prefix step of sequence parallelism (la_kv_aggregate) on the
 prefill's k and v under "kv_aggregate", and the gradients of the prefill
 (la_prefill_backward) under "backward".
@@ -53,18 +55,47 @@ def prefill_bytes(tok_heads: int, heads: int, seqs: int) -> int:
     return tok_heads * D * 2 * 4 + seqs * heads * D * D * 4
 
 
-def prefill_flops(tok_heads: int, block: int, frac_phase_a: float):
-    """(algorithmic, executed) FLOPs, 2 FLOP per multiply-add.
-    algorithmic per token-head: 2*(Bk+1)*d for the causal triangle of the
-    block including its diagonal (scores and P V) + 4*d^2 (inter term Q S and
-    state update K^T V).
-    executed per token-head, what the tensor pipe runs in this kernel:
-    Q K^T and P V over full 128x128 blocks (4*Bk*d), Q S_hi + Q S_lo (4*d^2),
-    K^T V in the scan (2*d^2) and again in the segment-sum pass for the
-    fraction of tokens whose segment has a successor (2*d^2*frac_phase_a)."""
-    alg = 2 * (block + 1) * D + 4 * D * D
-    exe = 4 * block * D + 6 * D * D + 2 * D * D * frac_phase_a
-    return tok_heads * alg, tok_heads * exe
+LO_SPLIT_FROM = 65536  # segments ending past this token use S as bf16 hi + lo in Q S
+
+
+def prefill_alg_flops(tok_heads: int, block: int) -> int:
+    """Algorithmic FLOPs (2 per multiply-add) per the blocked definition:
+    2*(Bk+1)*d per token-head for the causal triangle of its block including
+    the diagonal, plus 4*d^2 for the inter-block term Q S and the update K^T V."""
+    return tok_heads * (2 * (block + 1) * D + 4 * D * D)
+
+
+def prefill_survey_exec_flops(tok_heads: int, block: int) -> int:
+    """The dense count 4*Bk*d + 4*d^2 per token-head (full score and P V tiles,
+    one Q S and one K^T V), independent of how the kernel splits the work."""
+    return tok_heads * (4 * block * D + 4 * D * D)
+
+
+def prefill_mma_flops(lengths, heads: int, seg_len: int, want_state: bool = True) -> int:
+    """FLOPs the tensor pipe executes in la_prefill_kernel, counted MMA by MMA
+    the way the kernel issues them (one unit = a 128 x 128 x 128 product,
+    2 * 128^3 FLOPs), per segment of seg_len tokens of every sequence:
+      Q K^T and P V: one unit each per 128-row block (full tiles, masked or not);
+      Q S: one unit per block, two when the segment ends past LO_SPLIT_FROM
+           tokens into its sequence (S handed over as bf16 hi + lo);
+      K^T V in the scan: one unit per block except the segment's last block,
+           which also gets one in the final segment when the state is wanted;
+      K^T V in the segment-sum pass: one unit per block of every segment that
+           has a successor in its sequence."""
+    unit = 2 * 128 ** 3
+    units = 0
+    for n in lengths:
+        n = int(n)
+        nseg = -(-n // seg_len) if n > 0 else 0
+        for j in range(nseg):
+            t0, t1 = j * seg_len, min(n, (j + 1) * seg_len)
+            nblk = -(-(t1 - t0) // 128)
+            last = j == nseg - 1
+            units += 2 * nblk                                   # Q K^T, P V
+            units += nblk * (2 if t1 > LO_SPLIT_FROM else 1)    # Q S (hi [+ lo])
+            units += nblk - 1 + (1 if (last and want_state) else 0)  # K^T V, scan
+            units += 0 if last else nblk                        # K^T V, segment sums
+    return units * unit * heads
 
 
 def aggregate_bytes(tok_heads: int, pairs: int) -> int:
@@ -174,6 +205,60 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML every `period`
+    seconds from a background thread (a finer grid than nvidia-smi's 200 ms,
+    so that a timed region of a few tens of milliseconds still gets samples).
+    The GPU is found by its PCI bus id, so CUDA and NVML numbering may differ."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, dev: torch.device, period: float = 0.002):
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml as nv
+            self.nv = nv
+            nv.nvmlInit()
+            pr = torch.cuda.get_device_properties(dev)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            self.period = period
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.time(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+
+    def summary(self, t0: float, t1: float):
+        rows = [(m, r) for (t, m, r) in self.samples if t0 <= t <= t1]
+        if not rows:
+            return None
+        reasons = sorted({name for (_, r) in rows for (name, mask) in self.masks if r & mask})
+        return {"sm_mhz": float(np.median([m for m, _ in rows])), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(rows), "source": "NVML, 2 ms period"}
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -219,12 +304,12 @@ def oracle_sample_rate(budget_s: float, seed: int):
     while heads_done < H and elapsed < budget_s:
         hs = list(range(heads_done, min(H, heads_done + step)))
         t = time.perf_counter()
-        oracle.recurrent(Q, K, V, cu, heads=hs)
+        oracle.recurrent(Q, K, V, cu, heads=hs, threads=threads)
         elapsed += time.perf_counter() - t
         heads_done += len(hs)
     rate = N * heads_done / H / elapsed
-    desc = (f"fp64 recurrent oracle, {heads_done} of {H} heads x {N} tokens in {elapsed:.1f} s; "
-            f"tok/s scaled by {heads_done}/{H}")
+    desc = (f"fp64 recurrent oracle, {heads_done} of {H} heads x {N} tokens in {elapsed:.1f} s on "
+            f"{threads} OpenMP threads; tok/s scaled by {heads_done}/{H}")
     return rate, threads, desc
 
 
@@ -247,14 +332,17 @@ def run_reference(args, world, rank):
     ntok = int(max(64, min(N, per_step_s / per_tok * 0.8)))
     cu = np.array([0, ntok], np.int32)
     hs = list(range(nh))
+    # every call names its thread count: the 1-thread probe above must not
+    # leave the oracle on one thread
     for _ in range(args.warmup):
-        oracle.recurrent(Q[:ntok], K[:ntok], V[:ntok], cu, heads=hs)
+        oracle.recurrent(Q[:ntok], K[:ntok], V[:ntok], cu, heads=hs, threads=threads)
     t = time.perf_counter()
     for _ in range(args.steps):
-        oracle.recurrent(Q[:ntok], K[:ntok], V[:ntok], cu, heads=hs)
+        oracle.recurrent(Q[:ntok], K[:ntok], V[:ntok], cu, heads=hs, threads=threads)
     dt = time.perf_counter() - t
     value = ntok * nh / H * args.steps / dt       # tok/s of the 64-head workload
-    sample = f"each step: fp64 recurrent oracle on the first {ntok} tokens of {nh} of {H} heads; tok/s scaled by {nh}/{H}"
+    sample = (f"each step: fp64 recurrent oracle on the first {ntok} tokens of {nh} of {H} heads, "
+              f"{threads} OpenMP threads (one (sequence, head) pair each); tok/s scaled by {nh}/{H}")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -297,6 +385,7 @@ def run_cuda(args, world, rank, local):
         raise RuntimeError("device status not OK after warm-up")
 
     sampler = ClockSampler(local if world > 1 else 0) if rank == 0 else None
+    fast = NvmlClockSampler(dev) if rank == 0 else None
     time.sleep(0.3 if sampler else 0)
     launches0 = la.kernel_launches()
     barrier(world)
@@ -314,8 +403,16 @@ def run_cuda(args, world, rank, local):
     ms = ev0.elapsed_time(ev1) / args.steps
     ms_max = max_over_ranks(ms, world)
     status = la.get_device_status()
-    clocks = sampler.summary(t_host0, t_host1) if sampler else None
+    clocks = None
+    if fast is not None:
+        clocks = fast.summary(t_host0, t_host1)
+        fast.stop()
     if sampler:
+        smi = sampler.summary(t_host0, t_host1)
+        if clocks is None:
+            clocks = smi
+        else:
+            clocks["nvidia_smi"] = smi
         sampler.stop()
 
     tok_heads = B * N * H
@@ -323,8 +420,9 @@ def run_cuda(args, world, rank, local):
     value = tokens_all / (ms_max * 1e-3)
     byts = prefill_bytes(tok_heads, H, B)
     L = la.last_segment_len()
-    nseg = -(-N // L)
-    f_alg, f_exe = prefill_flops(tok_heads, BLOCK, (nseg - 1) * L / N)
+    f_alg = prefill_alg_flops(tok_heads, BLOCK)
+    f_mma = prefill_mma_flops([N] * B, H, L, want_state=True)
+    f_dense = prefill_survey_exec_flops(tok_heads, BLOCK)
     achieved_gbs = byts / (ms * 1e-3) / 1e9
 
     # ---------------- end to end through the public API with host buffers
@@ -356,6 +454,10 @@ def run_cuda(args, world, rank, local):
     if rank == 0 or world > 1:
         dec = bench_decode(la, dev, stream, args, hbm_peak, world)
 
+    # ---------------- the packed varlen batch and the 1M-token prefill
+    varlen = bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank)
+    longc = bench_long_context(la, dev, stream, args, hbm_peak, tc_peak, world, rank)
+
     # ---------------- local prefix of sequence parallelism on the same k, v
     agg = bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world)
     # ---------------- gradients of the prefill on the same q, k, v
@@ -375,8 +477,15 @@ def run_cuda(args, world, rank, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(world),
         "segment_len": L,
-        "tflops_alg": f_alg / (ms * 1e-3) / 1e12, "tflops_exec": f_exe / (ms * 1e-3) / 1e12,
-        "tensor_frac_exec": f_exe / (ms * 1e-3) / 1e12 / tc_peak,
+        "tflops_alg": f_alg / (ms * 1e-3) / 1e12,
+        "tflops_mma": f_mma / (ms * 1e-3) / 1e12,
+        "tensor_frac_mma": f_mma / (ms * 1e-3) / 1e12 / tc_peak,
+        "tensor_frac_alg": f_alg / (ms * 1e-3) / 1e12 / tc_peak,
+        "tensor_frac_dense_count": f_dense / (ms * 1e-3) / 1e12 / tc_peak,
+        "tensor_note": ("tflops_mma counts every tcgen05 MMA the kernel issues (full 128-row tiles, Q S once "
+                        "per block below 65536 tokens, K^T V in the scan and in the segment-sum pass); "
+                        "tflops_alg the blocked definition 2(Bk+1)d + 4d^2 per token-head; dense_count "
+                        "4 Bk d + 4 d^2; fractions of the measured cuBLAS bf16 burst peak"),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                      "kernel": "la_prefill_kernel", "bytes_per_launch": byts,
@@ -389,6 +498,8 @@ def run_cuda(args, world, rank, local):
         "gpu_launches": int(launches),
         "clocks": clocks,
         "decode": dec,
+        "varlen": varlen,
+        "long_context": longc,
         "kv_aggregate": agg,
         "backward": bwd,
         "cpu_baseline": cpu,
@@ -459,9 +570,14 @@ def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
                          "duration": "CUDA events around each la_prefill_backward call (about ten kernels)"}}
 
 
+DATASHEET_HBM_GBS = 7700.0  # HGX B200 HBM3e datasheet figure (8000 on DGX), context only
+
+
 def bench_decode(la, dev, stream, args, hbm_peak, world):
     """Decode workload: 256 sequences x 64 heads, states from a 4096-token
-    prefill (run in chunks of sequences), then timed decode steps."""
+    prefill (run in chunks of sequences), then timed decode steps, each on its
+    own freshly drawn q, k, v (one seeded set per step, generated before the
+    timed region and read from HBM once)."""
     state = torch.empty((DEC_SEQS, H, D, D), dtype=torch.float32, device=dev)
     chunk = 16
     for s0 in range(0, DEC_SEQS, chunk):
@@ -469,28 +585,129 @@ def bench_decode(la, dev, stream, args, hbm_peak, world):
         la.prefill(qp, kp, vp, block=BLOCK, state_out=state[s0:s0 + chunk])
         del qp, kp, vp
     steps = max(16, min(args.steps, 1024))
-    qs = [la_inputs.qkv((DEC_SEQS, H, D), la_inputs.decode_seed(SEED, s), device=dev) for s in range(8)]
+    warm = 3
+    qkv = torch.empty((warm + steps, 3, DEC_SEQS, H, D), dtype=torch.bfloat16, device=dev)
+    for i in range(warm + steps):
+        for j, t in enumerate(la_inputs.qkv((DEC_SEQS, H, D), la_inputs.decode_seed(SEED, i), device=dev)):
+            qkv[i, j] = t
     o = torch.empty((DEC_SEQS, H, D), dtype=torch.bfloat16, device=dev)
-    for i in range(3):
-        la.decode_step(*qs[i % 8], state, out=o)
+    for i in range(warm):
+        la.decode_step(qkv[i, 0], qkv[i, 1], qkv[i, 2], state, out=o)
     torch.cuda.synchronize(dev)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(steps):
-        la.decode_step(*qs[i % 8], state, out=o)
+    for i in range(warm, warm + steps):
+        la.decode_step(qkv[i, 0], qkv[i, 1], qkv[i, 2], state, out=o)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     pairs = DEC_SEQS * H
-    gbs = decode_bytes(pairs) / (ms * 1e-3) / 1e9
-    del state
-    return {"workload": "decode 256 seqs x H=64 x d=128, fp32 state (1 GiB) from a 4096-token prefill",
-            "tok_s": DEC_SEQS * world / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
+    byts = decode_bytes(pairs)
+    gbs = byts / (ms * 1e-3) / 1e9
+    traffic = recorded_traffic("la_decode_kernel", "decode_S256_H64")
+    del state, qkv
+    roof = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+            "frac": gbs / hbm_peak, "kernel": "la_decode_kernel", "traffic": traffic,
+            "bytes_per_launch": byts,
+            "datasheet_peak": DATASHEET_HBM_GBS, "frac_of_datasheet": gbs / DATASHEET_HBM_GBS}
+    if traffic is not None:
+        roof["achieved_dram"] = traffic / (ms * 1e-3) / 1e9
+        roof["frac_dram"] = roof["achieved_dram"] / hbm_peak
+    if roof["frac"] > 1.0:
+        roof["frac_above_1"] = ("algorithmic bytes / time exceed the measured copy bandwidth: part of the "
+                                "state is served from L2 between steps (ncu DRAM bytes below the "
+                                "algorithmic bytes), so this is not a DRAM roofline fraction; frac_dram "
+                                "and frac_of_datasheet bound it")
+    return {"workload": "decode 256 seqs x H=64 x d=128, fp32 state (1 GiB) from a 4096-token prefill, "
+                        "fresh q/k/v every step",
+            "tok_s": DEC_SEQS * world / (ms * 1e-3), "ms_per_step": ms, "steps": steps, "roofline": roof}
+
+
+def bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank):
+    """Packed variable-length prefill: 8 sequences with lengths drawn uniform in
+    [1024, 65536] from a seed, concatenated (cu_seqlens on the device), H=64,
+    bf16 out + fp32 final states.  About 266K tokens, 17 GB of algorithmic
+    traffic per call (inputs far larger than L2)."""
+    lens = la_inputs.varlen_lengths(8, 1024, 65536, seed=3)
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    T = int(cu[-1])
+    q, k, v = la_inputs.qkv((T, H, D), seed=303 + rank, device=dev)
+    cu_d = torch.from_numpy(cu).to(dev)
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    st = torch.empty((len(lens), H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(la.varlen_workspace_size(len(lens), T, int(lens.max()), H, D, BLOCK), dtype=torch.uint8,
+                     device=dev)
+
+    def call():
+        la.prefill_varlen(q, k, v, cu_d, int(lens.max()), block=BLOCK, out=out, state_out=st, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(5, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    L = la.last_segment_len()
+    byts = prefill_bytes(T * H, H, len(lens))
+    gbs = byts / (ms * 1e-3) / 1e9
+    f_mma = prefill_mma_flops(lens, H, L, want_state=True)
+    del q, k, v, out, st, ws
+    return {"workload": f"packed varlen prefill, 8 seqs U[1024, 65536] (seed 3): lengths {lens.tolist()}, "
+                        f"{T} tokens, H=64, d=128, bf16 in/out + fp32 final states",
+            "tok_s": T * world / (ms * 1e-3), "ms_per_call": ms, "steps": steps, "segment_len": L,
+            "tflops_alg": prefill_alg_flops(T * H, BLOCK) / (ms * 1e-3) / 1e12,
+            "tflops_mma": f_mma / (ms * 1e-3) / 1e12, "tensor_frac_mma": f_mma / (ms * 1e-3) / 1e12 / tc_peak,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": gbs / hbm_peak, "kernel": "la_decode_kernel",
-                         "traffic": recorded_traffic("la_decode_kernel", "decode_S256_H64"),
-                         "bytes_per_launch": decode_bytes(pairs)}}
+                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel", "bytes_per_launch": byts,
+                         "traffic": recorded_traffic("la_prefill_kernel", "varlen_S8_H64"),
+                         "duration": "CUDA events around each la_prefill_varlen call (scheduler + prefill)"}}
+
+
+def bench_long_context(la, dev, stream, args, hbm_peak, tc_peak, world, rank):
+    """Long-context prefill: B=1, H=8, N=1048576, bf16 out + fp32 final states
+    (8.6 GB of algorithmic traffic per call).  Segments past 65536 tokens hand
+    S to the inter-block product as bf16 hi + lo."""
+    NL, HL = 1048576, 8
+    q, k, v = la_inputs.qkv((1, NL, HL, D), seed=404 + rank, device=dev)
+    out = torch.empty((1, NL, HL, D), dtype=torch.bfloat16, device=dev)
+    st = torch.empty((1, HL, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(la.workspace_size(1, NL, HL, D, BLOCK), dtype=torch.uint8, device=dev)
+
+    def call():
+        la.prefill(q, k, v, block=BLOCK, out=out, state_out=st, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(5, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    L = la.last_segment_len()
+    byts = prefill_bytes(NL * HL, HL, 1)
+    gbs = byts / (ms * 1e-3) / 1e9
+    f_mma = prefill_mma_flops([NL], HL, L, want_state=True)
+    del q, k, v, out, st, ws
+    return {"workload": "long-context prefill B=1 H=8 N=1048576 d=128, bf16 in/out + fp32 final states",
+            "tok_s": NL * world / (ms * 1e-3), "ms_per_call": ms, "steps": steps, "segment_len": L,
+            "tflops_alg": prefill_alg_flops(NL * HL, BLOCK) / (ms * 1e-3) / 1e12,
+            "tflops_mma": f_mma / (ms * 1e-3) / 1e12, "tensor_frac_mma": f_mma / (ms * 1e-3) / 1e12 / tc_peak,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel", "bytes_per_launch": byts,
+                         "traffic": recorded_traffic("la_prefill_kernel", "prefill_B1_H8_N1048576"),
+                         "duration": "CUDA events around each la_prefill call (scheduler + prefill)"}}
 
 
 def main():

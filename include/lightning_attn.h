@@ -189,9 +189,8 @@ LA_API la_status la_mixed_step(const void *q, const void *k, const void *v,
  * the process uses from library load until exit; the call allocates and frees
  * nothing.  To fit, it may use longer cross-SM segments than la_prefill
  * (changing only speed and rounding).  A problem whose scratch needs exceed
- * 32 MiB even with one segment per sequence -- more than about 500
- * (sequence, head) pairs -- is rejected with LA_ERR_WORKSPACE before any
- * launch.  The first call on a device looks up the array's device address
+ * 32 MiB even with one segment per sequence -- B * H above 511 (sequence,
+ * head) pairs -- is rejected with LA_ERR_WORKSPACE before any launch.  The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
  * any stream capture.  Every call uses the same array and the kernels reset
  * the parts that must start at zero, so leftover contents do not matter, but

@@ -110,7 +110,40 @@ WsLayout ws_layout(long long gmax, int H) {
     return w;
 }
 
+// Upper bound of the number of segments of a packed batch: every sequence
+// boundary can add one partial segment.
 long long gmax_for(int nseq, long long T, int L) { return (T + L - 1) / L + nseq; }
+
+// Exact number of segments of B equal-length sequences of N tokens.
+long long gmax_fixed(int B, long long N, int L) { return (long long)B * ((N + L - 1) / L); }
+
+// Dynamic shared-memory limits are a property of each device's context, so the
+// attribute is set once per device (and again on a device that has not seen it).
+constexpr int kMaxDevices = 64;
+
+struct SmemAttr {
+    std::mutex mu;
+    bool done[kMaxDevices] = {};
+};
+
+template <typename Kernel>
+la_status ensure_smem_attr(SmemAttr &a, Kernel *kernel, int bytes) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return LA_ERR_CUDA;
+    if (dev >= kMaxDevices) {  // not cached: set it on every call
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess
+                   ? LA_OK : LA_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(a.mu);
+    if (!a.done[dev]) {
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+            return LA_ERR_CUDA;
+        a.done[dev] = true;
+    }
+    return LA_OK;
+}
+
+SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_agg;
 
 bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
     if (!a || !b || na == 0 || nb == 0) return false;
@@ -158,7 +191,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
 
     const int L = choose_seg_len(nseq, T, H);
     if (L <= 0 || L % la::BLK) return LA_ERR_INVALID_ARGUMENT;
-    const long long gmax = gmax_for(nseq, T, L);
+    const long long gmax = cu ? gmax_for(nseq, T, L) : gmax_fixed(nseq, fixed_len, L);
     const WsLayout w = ws_layout(gmax, H);
     if (!workspace || ws_bytes < w.total) return LA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return LA_ERR_INVALID_ARGUMENT;
@@ -216,16 +249,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.seg_len = L;
     pp.status = status;
 
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(la::la_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        la::PREFILL_SMEM);
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(la::la_prefill_kernel<true>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, la::PREFILL_SMEM);
-    });
-    if (attr_err != cudaSuccess) return LA_ERR_CUDA;
+    st = anti ? ensure_smem_attr(g_attr_prefill_anti, la::la_prefill_kernel<true>, la::PREFILL_SMEM)
+              : ensure_smem_attr(g_attr_prefill, la::la_prefill_kernel<false>, la::PREFILL_SMEM);
+    if (st != LA_OK) return st;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
     if (anti)
@@ -308,7 +334,7 @@ BwdLayout bwd_layout(int B, int N, int H) {
     BwdLayout w;
     const long long T = (long long)B * N;
     const int L = choose_seg_len(B, T, H);
-    const size_t pre = ws_layout(gmax_for(B, T, L), H).total;
+    const size_t pre = ws_layout(gmax_fixed(B, N, L), H).total;
     const size_t agg = agg_ws_bytes(agg_plan((long long)B * H, N));
     const size_t st = (size_t)B * H * la::D * la::D * sizeof(float);
     w.prefill = 0;
@@ -330,7 +356,7 @@ size_t la_prefill_workspace_size(int B, int N, int H, int d, int block) {
     if (B <= 0 || N < 0 || H <= 0) return la::HDR_BYTES;
     const long long T = (long long)B * N;
     const int L = choose_seg_len(B, T, H);
-    return ws_layout(gmax_for(B, T, L), H).total;
+    return ws_layout(gmax_fixed(B, N, L), H).total;
 }
 
 size_t la_prefill_varlen_workspace_size(int nseq, int total_tokens, int max_seqlen, int H, int d,
@@ -518,13 +544,8 @@ la_status la_kv_aggregate(const void *k, const void *v, int B, int N, int H, int
         p.per_cta = a.per_cta;
         p.wait_limit_ns = g_wait_limit_ns.load();
         p.status = status;
-        static std::once_flag attr_once;
-        static cudaError_t attr_err = cudaSuccess;
-        std::call_once(attr_once, [] {
-            attr_err = cudaFuncSetAttribute(la::la_kv_aggregate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            la::AGG_SMEM);
-        });
-        if (attr_err != cudaSuccess) return LA_ERR_CUDA;
+        st = ensure_smem_attr(g_attr_agg, la::la_kv_aggregate_kernel, la::AGG_SMEM);
+        if (st != LA_OK) return st;
         la::la_kv_aggregate_kernel<<<a.ctas, la::AGG_THREADS, la::AGG_SMEM, stream>>>(mk, mv, p);
         if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
         ++g_launches;
@@ -725,9 +746,9 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     // longest useful segment: one per sequence
     const int max_len = (int)(((long long)(N > 0 ? N : 1) + la::BLK - 1) / la::BLK * la::BLK);
     int L = choose_seg_len(B, T, H);
-    while (ws_layout(gmax_for(B, T, L), H).total > LA_NOALLOC_SCRATCH_BYTES && L < max_len)
+    while (ws_layout(gmax_fixed(B, N, L), H).total > LA_NOALLOC_SCRATCH_BYTES && L < max_len)
         L = (2 * L < max_len) ? 2 * L : max_len;
-    const long long gmax = gmax_for(B, T, L);
+    const long long gmax = gmax_fixed(B, N, L);
     const WsLayout w = ws_layout(gmax, H);
     if (w.total > LA_NOALLOC_SCRATCH_BYTES) return LA_ERR_WORKSPACE;  // beyond the built-in scratch
 
@@ -783,9 +804,8 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.anti_lo = 0;
     pp.seg_len = L;
     pp.status = status;
-    if (cudaFuncSetAttribute(la::la_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             la::PREFILL_SMEM) != cudaSuccess)
-        return LA_ERR_CUDA;
+    st = ensure_smem_attr(g_attr_prefill, la::la_prefill_kernel<false>, la::PREFILL_SMEM);
+    if (st != LA_OK) return st;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
     la::la_prefill_kernel<false><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);

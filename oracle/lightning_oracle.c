@@ -75,10 +75,25 @@ static int check_common(const int32_t *cu, int nseq, int H, int d,
     return 0;
 }
 
+/* The host's default thread count, captured before any call changes it, so
+ * that a call with nthreads = 0 runs on the default again after a call that
+ * asked for a specific count (omp_set_num_threads persists in the calling
+ * thread). */
+static int default_threads(void)
+{
+#ifdef _OPENMP
+    static int def = 0;
+    if (def <= 0) def = omp_get_max_threads();
+    return def;
+#else
+    return 1;
+#endif
+}
+
 static void set_threads(int nthreads)
 {
 #ifdef _OPENMP
-    if (nthreads > 0) omp_set_num_threads(nthreads);
+    omp_set_num_threads(nthreads > 0 ? nthreads : default_threads());
 #else
     (void)nthreads;
 #endif
@@ -86,11 +101,7 @@ static void set_threads(int nthreads)
 
 int lao_max_threads(void)
 {
-#ifdef _OPENMP
-    return omp_get_max_threads();
-#else
-    return 1;
-#endif
+    return default_threads();
 }
 
 /* Pointer to the d-vector of token t, head h in a [T][H][d] array. */
