@@ -45,6 +45,7 @@
  * closed forms, exact-integer library routines and brute force (see the
  * test files); none is "parity unpinned".
  */
+#include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -476,4 +477,324 @@ int lao_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const 
         free(Q); free(K); free(V); free(G);
     }
     return bad ? -1 : 0;
+}
+
+/* ===========================================================================
+ * Per-head decay.  [P5] §3.3 item 1 names a "decay value computation" fused
+ * into the prefill and [P2]/[P5] §2.3 describe the attention as the
+ * "transnormer" block, but no page gives the formula.  Reading (stated, not
+ * printed on the pages): the decayed recurrence of the TransNormer /
+ * Lightning Attention line, one constant lambda_h in (0, 1] per head h,
+ *
+ *   S_t = lambda S_{t-1} + k_t^T v_t,   o_t = q_t S_t,   S_{-1} = S_in,
+ *
+ * with t counted from the start of the sequence, equivalently
+ *
+ *   o_t = sum_{s <= t} lambda^{t-s} (q_t . k_s) v_s + lambda^{t+1} q_t S_in.
+ *
+ * lambda = 1 is the undecayed operation above (each decayed form below then
+ * reproduces its undecayed counterpart bit for bit: every extra factor is an
+ * exact 1.0).  `decay` is double [H], indexed by the head number h (not by the
+ * position in `heads`).  Powers lambda^n use the C library's pow().
+ * ======================================================================== */
+static int check_decay(const double *decay, int H)
+{
+    if (!decay) return -1;
+    for (int h = 0; h < H; ++h)
+        if (!(decay[h] >= 0.0 && decay[h] <= 1.0)) return -1;
+    return 0;
+}
+
+/* Decayed recurrent form: S_t = lambda S_{t-1} + k_t^T v_t, o_t = q_t S_t. */
+int lao_recurrent_decay(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *cu_seqlens, int nseq, int H, int d,
+                        const int32_t *heads, int nh, const double *decay,
+                        const double *state_in, double *out, double *state_out,
+                        int nthreads)
+{
+    if (!q || !k || !v || !out) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh) || check_decay(decay, H)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        const double lam = decay[h];
+        double *S = (double *)calloc((size_t)d * d, sizeof(double));
+        double *kt = (double *)malloc((size_t)d * sizeof(double));
+        double *vt = (double *)malloc((size_t)d * sizeof(double));
+        double *qt = (double *)malloc((size_t)d * sizeof(double));
+        if (!S || !kt || !vt || !qt) {
+            bad = 1;
+            free(S); free(kt); free(vt); free(qt);
+            continue;
+        }
+        if (state_in)
+            memcpy(S, state_in + (size_t)p * d * d, (size_t)d * d * sizeof(double));
+        for (int t = cu_seqlens[i]; t < cu_seqlens[i + 1]; ++t) {
+            for (int a = 0; a < d; ++a) {
+                qt[a] = widen_bf16(ROW(q, t, h)[a]);
+                kt[a] = widen_bf16(ROW(k, t, h)[a]);
+                vt[a] = widen_bf16(ROW(v, t, h)[a]);
+            }
+            /* S_t = lambda S_{t-1} + k_t^T v_t */
+            for (int a = 0; a < d; ++a)
+                for (int b = 0; b < d; ++b)
+                    S[(size_t)a * d + b] = lam * S[(size_t)a * d + b] + kt[a] * vt[b];
+            /* o_t = q_t S_t */
+            double *o = out + ((size_t)t * nh + j) * d;
+            for (int b = 0; b < d; ++b) o[b] = 0.0;
+            for (int a = 0; a < d; ++a)
+                for (int b = 0; b < d; ++b)
+                    o[b] += qt[a] * S[(size_t)a * d + b];
+        }
+        if (state_out)
+            memcpy(state_out + (size_t)p * d * d, S, (size_t)d * d * sizeof(double));
+        free(S); free(kt); free(vt); free(qt);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Decayed quadratic form, the closed form of the recurrence:
+ *   o_t   = sum_{s <= t} lambda^{t-s} (q_t . k_s) v_s + lambda^{t-t0+1} q_t S_in
+ *   S_out = lambda^{n} S_in + sum_s lambda^{t1-1-s} k_s^T v_s
+ * (t0, t1 = the sequence's first and one-past-last token, n = t1 - t0).
+ */
+int lao_quadratic_decay(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *cu_seqlens, int nseq, int H, int d,
+                        const int32_t *heads, int nh, const double *decay,
+                        const double *state_in, double *out, double *state_out,
+                        int nthreads)
+{
+    if (!q || !k || !v || !out) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh) || check_decay(decay, H)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        const double lam = decay[h];
+        const int t0 = cu_seqlens[i], t1 = cu_seqlens[i + 1];
+        const double *Sin = state_in ? state_in + (size_t)p * d * d : NULL;
+        for (int t = t0; t < t1; ++t) {
+            double *o = out + ((size_t)t * nh + j) * d;
+            for (int b = 0; b < d; ++b) o[b] = 0.0;
+            for (int s = t0; s <= t; ++s) {
+                double score = 0.0;                  /* (Q K^T)[t][s] */
+                for (int a = 0; a < d; ++a)
+                    score += widen_bf16(ROW(q, t, h)[a]) * widen_bf16(ROW(k, s, h)[a]);
+                const double w = score * pow(lam, (double)(t - s));
+                for (int b = 0; b < d; ++b)
+                    o[b] += w * widen_bf16(ROW(v, s, h)[b]);
+            }
+            if (Sin) {
+                const double f = pow(lam, (double)(t - t0 + 1));
+                for (int a = 0; a < d; ++a) {
+                    const double qa = widen_bf16(ROW(q, t, h)[a]) * f;
+                    for (int b = 0; b < d; ++b) o[b] += qa * Sin[(size_t)a * d + b];
+                }
+            }
+        }
+        if (state_out) {
+            double *S = state_out + (size_t)p * d * d;
+            const double f = pow(lam, (double)(t1 - t0));
+            for (size_t e = 0; e < (size_t)d * d; ++e) S[e] = Sin ? f * Sin[e] : 0.0;
+            for (int s = t0; s < t1; ++s) {
+                const double w = pow(lam, (double)(t1 - 1 - s));
+                for (int a = 0; a < d; ++a) {
+                    const double ka = widen_bf16(ROW(k, s, h)[a]) * w;
+                    for (int b = 0; b < d; ++b)
+                        S[(size_t)a * d + b] += ka * widen_bf16(ROW(v, s, h)[b]);
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Decayed blocked form (the blocked algorithm of [P2]/[P5] §2.2 with the
+ * decay of the reading above).  Rows b0 <= t < b1 of one block, local index
+ * r = t - b0, block length nb = b1 - b0:
+ *   O_b     = ((Q_b K_b^T) ⊙ D_b) V_b + diag(lambda^{r+1}) Q_b S_{<b},
+ *             D_b[r][c] = lambda^{r-c} for c <= r, else 0
+ *   S_{<=b} = lambda^{nb} S_{<b} + sum_{c} lambda^{nb-1-c} k_{b0+c}^T v_{b0+c}
+ */
+static void blocked_decay_one(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              int H, int d, int h, int j, int nh, int t0, int t1,
+                              int block, double lam, double *S, double *out)
+{
+    for (int b0 = t0; b0 < t1; b0 += block) {
+        const int b1 = (b0 + block < t1) ? b0 + block : t1;
+        for (int t = b0; t < b1; ++t) {
+            double *o = out + ((size_t)t * nh + j) * d;
+            for (int b = 0; b < d; ++b) o[b] = 0.0;
+            /* intra-block left product ((Q_b K_b^T) ⊙ D_b) V_b */
+            for (int s = b0; s <= t; ++s) {
+                double score = 0.0;
+                for (int a = 0; a < d; ++a)
+                    score += widen_bf16(ROW(q, t, h)[a]) * widen_bf16(ROW(k, s, h)[a]);
+                const double w = score * pow(lam, (double)(t - s));
+                for (int b = 0; b < d; ++b)
+                    o[b] += w * widen_bf16(ROW(v, s, h)[b]);
+            }
+            /* inter-block right product lambda^{r+1} q_t S_{<b} */
+            const double f = pow(lam, (double)(t - b0 + 1));
+            for (int a = 0; a < d; ++a) {
+                const double qa = widen_bf16(ROW(q, t, h)[a]) * f;
+                for (int b = 0; b < d; ++b) o[b] += qa * S[(size_t)a * d + b];
+            }
+        }
+        /* S_{<=b} = lambda^{nb} S_{<b} + sum_c lambda^{nb-1-c} k^T v */
+        const double f = pow(lam, (double)(b1 - b0));
+        for (size_t e = 0; e < (size_t)d * d; ++e) S[e] *= f;
+        for (int s = b0; s < b1; ++s) {
+            const double w = pow(lam, (double)(b1 - 1 - s));
+            for (int a = 0; a < d; ++a) {
+                const double ka = widen_bf16(ROW(k, s, h)[a]) * w;
+                for (int b = 0; b < d; ++b)
+                    S[(size_t)a * d + b] += ka * widen_bf16(ROW(v, s, h)[b]);
+            }
+        }
+    }
+}
+
+int lao_blocked_decay(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                      const int32_t *cu_seqlens, int nseq, int H, int d,
+                      const int32_t *heads, int nh, int block, const double *decay,
+                      const double *state_in, double *out, double *state_out, int nthreads)
+{
+    if (!q || !k || !v || !out || block <= 0) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh) || check_decay(decay, H)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        double *S = (double *)calloc((size_t)d * d, sizeof(double));
+        if (!S) { bad = 1; continue; }
+        if (state_in)
+            memcpy(S, state_in + (size_t)p * d * d, (size_t)d * d * sizeof(double));
+        blocked_decay_one(q, k, v, H, d, h, j, nh, cu_seqlens[i], cu_seqlens[i + 1],
+                          block, decay[h], S, out);
+        if (state_out)
+            memcpy(state_out + (size_t)p * d * d, S, (size_t)d * d * sizeof(double));
+        free(S);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * Decayed segmented form (the LASP+ recipe of [P5] §3.2 item 3 over the
+ * segments of one sequence, with the decay of the reading above):
+ *   1. local sums   A_r = sum_{s in r} lambda^{e_r-1-s} k_s^T v_s
+ *      (segment r = tokens [s_r, e_r));
+ *   2. the local sums are gathered;
+ *   3. global prefix G_r = lambda^{s_r-t0} S_in + sum_{r' < r} lambda^{s_r-e_r'} A_r',
+ *      then the decayed blocked form over segment r starting from G_r.
+ * The final state is lambda^{n} S_in + sum_r lambda^{t1-e_r} A_r.
+ */
+int lao_segmented_decay(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const int32_t *cu_seqlens, int nseq, int H, int d,
+                        const int32_t *heads, int nh, int seg_len, int block,
+                        const double *decay, const double *state_in, double *out,
+                        double *state_out, int nthreads)
+{
+    if (!q || !k || !v || !out || block <= 0 || seg_len <= 0) return -1;
+    if (check_common(cu_seqlens, nseq, H, d, heads, nh) || check_decay(decay, H)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)nseq * nh;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long p = 0; p < npairs; ++p) {
+        const int i = (int)(p / nh), j = (int)(p % nh);
+        const int h = heads ? heads[j] : j;
+        const double lam = decay[h];
+        const int t0 = cu_seqlens[i], t1 = cu_seqlens[i + 1];
+        const int nseg = (t1 - t0 + seg_len - 1) / seg_len;
+        const size_t dd = (size_t)d * d;
+        double *local = (double *)calloc((size_t)(nseg > 0 ? nseg : 1) * dd, sizeof(double));
+        double *G = (double *)malloc(dd * sizeof(double));
+        if (!local || !G) { bad = 1; free(local); free(G); continue; }
+        /* step 1: local sums */
+        for (int r = 0; r < nseg; ++r) {
+            const int s0 = t0 + r * seg_len;
+            const int s1 = (s0 + seg_len < t1) ? s0 + seg_len : t1;
+            double *L = local + (size_t)r * dd;
+            for (int s = s0; s < s1; ++s) {
+                const double w = pow(lam, (double)(s1 - 1 - s));
+                for (int a = 0; a < d; ++a) {
+                    const double ka = widen_bf16(ROW(k, s, h)[a]) * w;
+                    for (int b = 0; b < d; ++b)
+                        L[(size_t)a * d + b] += ka * widen_bf16(ROW(v, s, h)[b]);
+                }
+            }
+        }
+        /* step 3: global prefix of each segment, then its blocked scan */
+        for (int r = 0; r < nseg; ++r) {
+            const int s0 = t0 + r * seg_len;
+            const int s1 = (s0 + seg_len < t1) ? s0 + seg_len : t1;
+            const double fin = pow(lam, (double)(s0 - t0));
+            for (size_t e = 0; e < dd; ++e)
+                G[e] = state_in ? fin * state_in[(size_t)p * dd + e] : 0.0;
+            for (int r2 = 0; r2 < r; ++r2) {
+                const int e2 = t0 + (r2 + 1) * seg_len;     /* end of segment r2 (< t1) */
+                const double f = pow(lam, (double)(s0 - e2));
+                for (size_t e = 0; e < dd; ++e) G[e] += f * local[(size_t)r2 * dd + e];
+            }
+            blocked_decay_one(q, k, v, H, d, h, j, nh, s0, s1, block, lam, G, out);
+        }
+        if (state_out) {
+            double *So = state_out + (size_t)p * dd;
+            const double fin = pow(lam, (double)(t1 - t0));
+            for (size_t e = 0; e < dd; ++e)
+                So[e] = state_in ? fin * state_in[(size_t)p * dd + e] : 0.0;
+            for (int r = 0; r < nseg; ++r) {
+                const int e_r = (t0 + (r + 1) * seg_len < t1) ? t0 + (r + 1) * seg_len : t1;
+                const double f = pow(lam, (double)(t1 - e_r));
+                for (size_t e = 0; e < dd; ++e) So[e] += f * local[(size_t)r * dd + e];
+            }
+        }
+        free(local); free(G);
+    }
+    return bad ? -1 : 0;
+}
+
+/*
+ * One decayed decode step (the decode step of [P5] §3.3 items 1-2 under the
+ * decay reading above).  For every (b, h):
+ *   S <- lambda_h S + k^T v,   o = q S.
+ */
+int lao_decode_step_decay(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          int B, int H, int d, const double *decay, double *state,
+                          double *out, int nthreads)
+{
+    if (!q || !k || !v || !state || !out || B < 0 || H <= 0 || d <= 0) return -1;
+    if (check_decay(decay, H)) return -1;
+    set_threads(nthreads);
+    const long npairs = (long)B * H;
+#pragma omp parallel for schedule(static)
+    for (long p = 0; p < npairs; ++p) {
+        const double lam = decay[p % H];
+        double *S = state + (size_t)p * d * d;
+        const uint16_t *qp = q + (size_t)p * d, *kp = k + (size_t)p * d, *vp = v + (size_t)p * d;
+        for (int a = 0; a < d; ++a) {
+            const double ka = widen_bf16(kp[a]);
+            for (int b = 0; b < d; ++b)
+                S[(size_t)a * d + b] = lam * S[(size_t)a * d + b] + ka * widen_bf16(vp[b]);
+        }
+        double *o = out + (size_t)p * d;
+        for (int b = 0; b < d; ++b) o[b] = 0.0;
+        for (int a = 0; a < d; ++a) {
+            const double qa = widen_bf16(qp[a]);
+            for (int b = 0; b < d; ++b) o[b] += qa * S[(size_t)a * d + b];
+        }
+    }
+    return 0;
 }

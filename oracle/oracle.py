@@ -15,6 +15,8 @@ Forms (see the C file for the cited passages):
   blocked(...)     intra-block left product + inter-block right product
   segmented(...)   LASP+ recipe: local sums, gather, global prefix, blocked scan
   decode_step(...) one recurrent step on a persistent state
+  *_decay(...)     the same forms with a per-head decay lambda_h (a reading:
+                   S_t = lambda S_{t-1} + k_t^T v_t; see the C file)
 """
 from __future__ import annotations
 
@@ -37,7 +39,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
         tmp = _SO + f".tmp{os.getpid()}"
         cmd = ["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
-               "-ffp-contract=off", "-std=c11", _SRC, "-o", tmp]
+               "-ffp-contract=off", "-std=c11", _SRC, "-o", tmp, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _SO)
     return _SO
@@ -49,8 +51,8 @@ def build_variant(source_text: str, so_path: str):
     c_path = so_path[:-3] + ".c"
     with open(c_path, "w") as f:
         f.write(source_text)
-    subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-fopenmp", "-std=c11", c_path,
-                    "-o", so_path], check=True)
+    subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-std=c11", c_path,
+                    "-o", so_path, "-lm"], check=True)
     return _bind(so_path)
 
 
@@ -80,6 +82,17 @@ def _bind(path: str):
     lib.lao_backward.argtypes = [u16p, u16p, u16p, u16p, i32p, c_int, c_int, c_int, i32p, c_int,
                                  f64p, f64p, f64p, f64p, f64p, f64p, c_int]
     lib.lao_backward.restype = c_int
+    f64c = ctypes.POINTER(ctypes.c_double)
+    for name in ("lao_recurrent_decay", "lao_quadratic_decay"):
+        fn = getattr(lib, name)
+        fn.argtypes = common + [f64c, f64p, f64p, f64p, c_int]
+        fn.restype = c_int
+    lib.lao_blocked_decay.argtypes = common + [c_int, f64c, f64p, f64p, f64p, c_int]
+    lib.lao_blocked_decay.restype = c_int
+    lib.lao_segmented_decay.argtypes = common + [c_int, c_int, f64c, f64p, f64p, f64p, c_int]
+    lib.lao_segmented_decay.restype = c_int
+    lib.lao_decode_step_decay.argtypes = [u16p, u16p, u16p, c_int, c_int, c_int, f64c, f64p, f64p, c_int]
+    lib.lao_decode_step_decay.restype = c_int
     lib.lao_max_threads.argtypes = []
     lib.lao_max_threads.restype = c_int
     return lib
@@ -156,6 +169,74 @@ def segmented(q, k, v, cu_seqlens, seg_len, block, heads=None, state_in=None, th
     """LASP+ recipe over segments of ``seg_len`` tokens, each scanned in blocks."""
     return _run("lao_segmented", q, k, v, cu_seqlens, heads, state_in, threads,
                 (int(seg_len), int(block)), lib=lib)
+
+
+def _decay_arr(decay, H):
+    lam = np.ascontiguousarray(decay, dtype=np.float64)
+    if lam.shape != (H,):
+        raise ValueError(f"decay must hold one value per head, shape ({H},)")
+    return lam
+
+
+def _run_decay(name, q, k, v, cu_seqlens, decay, heads, state_in, threads, extra=(), lib=None):
+    q, k, v, cu, nseq, T, H, d, hs, nh, state_in = _prep(q, k, v, cu_seqlens, heads, state_in)
+    lam = _decay_arr(decay, H)
+    out = np.zeros((T, nh, d), dtype=np.float64)
+    state_out = np.zeros((nseq, nh, d, d), dtype=np.float64)
+    fn = getattr(lib or _load(), name)
+    rc = fn(_ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16), _ptr(v, ctypes.c_uint16),
+            _ptr(cu, ctypes.c_int32), nseq, H, d, _ptr(hs, ctypes.c_int32), nh, *extra,
+            _ptr(lam, ctypes.c_double), _ptr(state_in, ctypes.c_double), _ptr(out, ctypes.c_double),
+            _ptr(state_out, ctypes.c_double), int(threads or 0))
+    if rc != 0:
+        raise ValueError(f"{name} rejected its arguments")
+    return out, state_out
+
+
+def recurrent_decay(q, k, v, cu_seqlens, decay, heads=None, state_in=None, threads=None, lib=None):
+    """Decayed recurrent form S_t = lambda_h S_{t-1} + k_t^T v_t, o_t = q_t S_t;
+    decay: one value per head (length H, indexed by head number)."""
+    return _run_decay("lao_recurrent_decay", q, k, v, cu_seqlens, decay, heads, state_in, threads, lib=lib)
+
+
+def quadratic_decay(q, k, v, cu_seqlens, decay, heads=None, state_in=None, threads=None, lib=None):
+    """Decayed closed form o_t = sum_{s<=t} lambda^{t-s} (q_t . k_s) v_s + lambda^{t+1} q_t S_in."""
+    return _run_decay("lao_quadratic_decay", q, k, v, cu_seqlens, decay, heads, state_in, threads, lib=lib)
+
+
+def blocked_decay(q, k, v, cu_seqlens, block, decay, heads=None, state_in=None, threads=None, lib=None):
+    """Decayed blocked form (intra-block decay mask, row-scaled inter term, decayed state update)."""
+    return _run_decay("lao_blocked_decay", q, k, v, cu_seqlens, decay, heads, state_in, threads,
+                      (int(block),), lib=lib)
+
+
+def segmented_decay(q, k, v, cu_seqlens, seg_len, block, decay, heads=None, state_in=None, threads=None,
+                    lib=None):
+    """Decayed LASP+ recipe over segments of ``seg_len`` tokens."""
+    return _run_decay("lao_segmented_decay", q, k, v, cu_seqlens, decay, heads, state_in, threads,
+                      (int(seg_len), int(block)), lib=lib)
+
+
+def decode_step_decay(q, k, v, state, decay, threads=None, lib=None):
+    """One decayed decode step S <- lambda_h S + k^T v, o = q S (copies the state)."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    if q.ndim != 3 or q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v must be [B, H, d] bf16 bit arrays of one shape")
+    B, H, d = q.shape
+    lam = _decay_arr(decay, H)
+    st = np.array(state, dtype=np.float64, copy=True, order="C")
+    if st.shape != (B, H, d, d):
+        raise ValueError("state must be [B, H, d, d]")
+    out = np.zeros((B, H, d), dtype=np.float64)
+    rc = (lib or _load()).lao_decode_step_decay(_ptr(q, ctypes.c_uint16), _ptr(k, ctypes.c_uint16),
+                                                _ptr(v, ctypes.c_uint16), B, H, d, _ptr(lam, ctypes.c_double),
+                                                _ptr(st, ctypes.c_double), _ptr(out, ctypes.c_double),
+                                                int(threads or 0))
+    if rc != 0:
+        raise ValueError("lao_decode_step_decay rejected its arguments")
+    return out, st
 
 
 def decode_step(q, k, v, state, threads=None, lib=None):

@@ -385,7 +385,172 @@ def pin_backward_homogeneity(orc, lib=None):
     assert np.allclose(s_out - Sin, kv, rtol=0, atol=1e-12)
 
 
+# -------------------------------------------------------------------------- per-head decay
+def _decays(H, seed):
+    """Per-head decays in (0, 1], one exactly 1 and one small."""
+    lam = np.random.default_rng(seed).uniform(0.55, 0.999, H)
+    lam[0] = 1.0
+    if H > 2:
+        lam[-1] = 0.2
+    return lam
+
+
+def pin_decay_one_is_undecayed(orc, lib=None):
+    """lambda = 1 on every head: each decayed form equals its undecayed
+    counterpart bit for bit (every extra factor is an exact 1.0)."""
+    lens = [11, 0, 23, 6]
+    T, H, d = sum(lens), 3, 5
+    Q, K, V = _rand_bits(T, H, d, seed=40)
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    sin = np.random.default_rng(41).normal(size=(len(lens), H, d, d))
+    one = np.ones(H)
+    pairs = [
+        (orc.recurrent_decay(Q, K, V, cu, one, state_in=sin, lib=lib), orc.recurrent(Q, K, V, cu, state_in=sin, lib=lib)),
+        (orc.quadratic_decay(Q, K, V, cu, one, state_in=sin, lib=lib), orc.quadratic(Q, K, V, cu, state_in=sin, lib=lib)),
+        (orc.blocked_decay(Q, K, V, cu, 4, one, state_in=sin, lib=lib),
+         orc.blocked(Q, K, V, cu, 4, state_in=sin, lib=lib)),
+        (orc.segmented_decay(Q, K, V, cu, 8, 3, one, state_in=sin, lib=lib),
+         orc.segmented(Q, K, V, cu, 8, 3, state_in=sin, lib=lib)),
+    ]
+    for i, ((o1, s1), (o2, s2)) in enumerate(pairs):
+        assert np.array_equal(o1, o2) and np.array_equal(s1, s2), i
+    Qd, Kd, Vd = _rand_bits(2 * H, 1, d, seed=42)
+    sd = np.random.default_rng(43).normal(size=(2, H, d, d))
+    shp = lambda x: x.reshape(2, H, d)  # noqa: E731
+    o1, s1 = orc.decode_step_decay(shp(Qd), shp(Kd), shp(Vd), sd, one, lib=lib)
+    o2, s2 = orc.decode_step(shp(Qd), shp(Kd), shp(Vd), sd, lib=lib)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+
+
+def pin_decay_brute_force(orc, lib=None):
+    """Pure-Python sums o_t[b] = sum_{s<=t} lam^(t-s) sum_a q_t[a] k_s[a] v_s[b]
+    + lam^(t+1) sum_a q_t[a] S_in[a][b] and the final state, tiny inputs."""
+    for seed, (T, d, lam) in enumerate([(1, 1, 0.5), (6, 2, 0.9), (9, 3, 0.3), (7, 4, 0.77)]):
+        Q, K, V = _rand_bits(T, 1, d, seed=110 + seed)
+        sin = np.random.default_rng(120 + seed).normal(size=(1, 1, d, d))
+        q, k, v, S = _f(Q)[:, 0].tolist(), _f(K)[:, 0].tolist(), _f(V)[:, 0].tolist(), sin[0, 0].tolist()
+        exp = [[sum(lam ** (t - s) * sum(q[t][a] * k[s][a] for a in range(d)) * v[s][b] for s in range(t + 1))
+                + lam ** (t + 1) * sum(q[t][a] * S[a][b] for a in range(d))
+                for b in range(d)] for t in range(T)]
+        st = [[lam ** T * S[a][b] + sum(lam ** (T - 1 - s) * k[s][a] * v[s][b] for s in range(T))
+               for b in range(d)] for a in range(d)]
+        cu = np.array([0, T], np.int32)
+        for form in ("recurrent_decay", "quadratic_decay"):
+            out, so = getattr(orc, form)(Q, K, V, cu, [lam], state_in=sin, lib=lib)
+            assert np.allclose(out[:, 0], np.array(exp), rtol=1e-12, atol=1e-15), (form, T, d)
+            assert np.allclose(so[0, 0], np.array(st), rtol=1e-12, atol=1e-15), (form, T, d)
+
+
+def pin_decay_constant_kv(orc, lib=None):
+    """k_t = k, v_t = v: S_t = lam^(t+1) S_in + (1 - lam^(t+1)) / (1 - lam) k^T v
+    (a geometric series), o_t = q_t S_t."""
+    T, d, H = 41, 6, 2
+    Q, K, V = _rand_bits(T, H, d, seed=44)
+    K[:] = K[0]
+    V[:] = V[0]
+    lam = np.array([0.93, 0.6])
+    sin = np.random.default_rng(45).normal(size=(1, H, d, d))
+    cu = np.array([0, T], np.int32)
+    q, k, v = _f(Q), _f(K), _f(V)
+    for form in ("recurrent_decay", "quadratic_decay"):
+        out, st = getattr(orc, form)(Q, K, V, cu, lam, state_in=sin, lib=lib)
+        for h in range(H):
+            kv = np.outer(k[0, h], v[0, h])
+            for t in range(T):
+                S_t = lam[h] ** (t + 1) * sin[0, h] + (1 - lam[h] ** (t + 1)) / (1 - lam[h]) * kv
+                assert np.allclose(out[t, h], q[t, h] @ S_t, rtol=1e-11, atol=1e-13), (form, h, t)
+            S_T = lam[h] ** T * sin[0, h] + (1 - lam[h] ** T) / (1 - lam[h]) * kv
+            assert np.allclose(st[0, h], S_T, rtol=1e-11, atol=1e-13), (form, h)
+
+
+def pin_decay_exact_half(orc, lib=None):
+    """lam = 1/2 (an exact power of two) and small-integer inputs: every term
+    is exact, so the oracle must equal numpy's ((Q K^T) ⊙ D) V + diag(2^-(t+1)) Q S_in
+    with D[t][s] = 2^-(t-s) for s <= t, and the matching final state, bit for bit."""
+    rng = np.random.default_rng(46)
+    lens = [12, 9]
+    T, H, d = sum(lens), 2, 4
+    qf = rng.integers(-3, 4, (T, H, d)).astype(np.float64)
+    kf = rng.integers(-3, 4, (T, H, d)).astype(np.float64)
+    vf = rng.integers(-3, 4, (T, H, d)).astype(np.float64)
+    sin = rng.integers(-2, 3, (2, H, d, d)).astype(np.float64)
+    Q, K, V = la_inputs.bf16_exact(qf), la_inputs.bf16_exact(kf), la_inputs.bf16_exact(vf)
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    lam = np.array([0.5, 1.0])
+    exp_out = np.zeros((T, H, d))
+    exp_st = np.zeros((2, H, d, d))
+    for i in range(2):
+        a, b = cu[i], cu[i + 1]
+        n = b - a
+        for h in range(H):
+            tt = np.arange(n)
+            D = np.tril(lam[h] ** (tt[:, None] - tt[None, :]).clip(min=0))
+            qs, ks, vs = qf[a:b, h], kf[a:b, h], vf[a:b, h]
+            exp_out[a:b, h] = ((qs @ ks.T) * D) @ vs + (lam[h] ** (tt + 1))[:, None] * (qs @ sin[i, h])
+            exp_st[i, h] = lam[h] ** n * sin[i, h] + (ks * (lam[h] ** (n - 1 - tt))[:, None]).T @ vs
+    runs = {
+        "recurrent": orc.recurrent_decay(Q, K, V, cu, lam, state_in=sin, lib=lib),
+        "quadratic": orc.quadratic_decay(Q, K, V, cu, lam, state_in=sin, lib=lib),
+        "blocked5": orc.blocked_decay(Q, K, V, cu, 5, lam, state_in=sin, lib=lib),
+        "segmented": orc.segmented_decay(Q, K, V, cu, 7, 3, lam, state_in=sin, lib=lib),
+    }
+    for name, (out, st) in runs.items():
+        assert np.array_equal(out, exp_out), name
+        assert np.array_equal(st, exp_st), name
+
+
+def pin_decay_forms_agree(orc, lib=None):
+    """recurrent == quadratic == blocked (every block size) == segmented under
+    decay, with packed sequences and a carried-in state; lam -> 0 leaves only
+    the diagonal term (q_t . k_t) v_t."""
+    lens = [37, 27]
+    T, H, d = sum(lens), 3, 6
+    Q, K, V = _rand_bits(T, H, d, seed=47)
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    lam = _decays(H, 48)
+    sin = np.random.default_rng(49).normal(size=(2, H, d, d))
+    ref, rst = orc.quadratic_decay(Q, K, V, cu, lam, state_in=sin, lib=lib)
+    out, st = orc.recurrent_decay(Q, K, V, cu, lam, state_in=sin, lib=lib)
+    assert _rel(out, ref) < 1e-12 and _rel(st, rst) < 1e-12
+    for blk in range(1, max(lens) + 1):
+        out, st = orc.blocked_decay(Q, K, V, cu, blk, lam, state_in=sin, lib=lib)
+        assert _rel(out, ref) < 1e-12 and _rel(st, rst) < 1e-12, blk
+    for seg, blk in [(1, 1), (8, 4), (10, 3), (37, 37), (50, 6)]:
+        out, st = orc.segmented_decay(Q, K, V, cu, seg, blk, lam, state_in=sin, lib=lib)
+        assert _rel(out, ref) < 1e-12 and _rel(st, rst) < 1e-12, (seg, blk)
+    zero = np.zeros(H)
+    q, k, v = _f(Q), _f(K), _f(V)
+    exp = np.einsum("tha,tha->th", q, k)[:, :, None] * v
+    for form in ("recurrent_decay", "quadratic_decay"):
+        out, st = getattr(orc, form)(Q, K, V, cu, zero, state_in=sin, lib=lib)
+        assert np.allclose(out, exp, rtol=1e-14, atol=1e-300), form
+        for i in range(2):
+            last = cu[i + 1] - 1
+            assert np.allclose(st[i], np.einsum("ha,hb->hab", k[last], v[last]), rtol=1e-14, atol=1e-300)
+
+
+def pin_decay_carry_and_decode(orc, lib=None):
+    """prefill(A) then prefill(B, S_A) == prefill(A ++ B) and prefill(N) then m
+    decayed decode steps == prefill(N + m), with per-head decays."""
+    N, m, H, d = 30, 5, 3, 6
+    Q, K, V = _rand_bits(N + m, H, d, seed=50)
+    lam = _decays(H, 51)
+    full, fst = orc.recurrent_decay(Q, K, V, np.array([0, N + m], np.int32), lam, lib=lib)
+    _, sA = orc.quadratic_decay(Q[:N], K[:N], V[:N], np.array([0, N], np.int32), lam, lib=lib)
+    outB, sB = orc.blocked_decay(Q[N:], K[N:], V[N:], np.array([0, m], np.int32), 2, lam, state_in=sA, lib=lib)
+    assert _rel(outB, full[N:]) < 1e-12 and _rel(sB, fst) < 1e-12
+    state = sA[0][None]
+    for t in range(N, N + m):
+        o, state = orc.decode_step_decay(Q[t][None], K[t][None], V[t][None], state, lam, lib=lib)
+        assert _rel(o[0], full[t]) < 1e-12, t
+    assert _rel(state[0], fst[0]) < 1e-12
+    # a subset of heads, in another order, reads the decay of its own head number
+    out, st = orc.recurrent_decay(Q, K, V, np.array([0, N + m], np.int32), lam, heads=[2, 0], lib=lib)
+    assert np.array_equal(out, full[:, [2, 0]]) and np.array_equal(st, fst[:, [2, 0]])
+
+
 ALL_PINS = [pin_golden, pin_single_token, pin_constant_kv, pin_one_hot_q, pin_exact_integers,
             pin_brute_force, pin_forms_agree, pin_causality_and_packing,
             pin_state_carry_and_decode, pin_linearity, pin_backward_golden, pin_backward_autograd,
-            pin_backward_homogeneity]
+            pin_backward_homogeneity, pin_decay_one_is_undecayed, pin_decay_brute_force,
+            pin_decay_constant_kv, pin_decay_exact_half, pin_decay_forms_agree, pin_decay_carry_and_decode]

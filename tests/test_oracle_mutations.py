@@ -53,6 +53,29 @@ MUTANTS = [
     ("backward_dsin_drops_state_grad", "D[e] = GS ? GS[e] : 0.0;", "D[e] = 0.0;", 0),
     ("backward_dsin_transposed", "D[(size_t)a * d + b] += Q[(size_t)t * d + a] * G[(size_t)t * d + b];",
      "D[(size_t)b * d + a] += Q[(size_t)t * d + a] * G[(size_t)t * d + b];", 0),
+    # per-head decay
+    ("decay_recurrent_decays_new_token", "S[(size_t)a * d + b] = lam * S[(size_t)a * d + b] + kt[a] * vt[b];",
+     "S[(size_t)a * d + b] = lam * (S[(size_t)a * d + b] + kt[a] * vt[b]);", 0),
+    ("decay_recurrent_position_not_head", "const double lam = decay[h];", "const double lam = decay[j];", 0),
+    ("decay_quadratic_exponent_plus_one", "const double w = score * pow(lam, (double)(t - s));",
+     "const double w = score * pow(lam, (double)(t - s + 1));", 0),
+    ("decay_quadratic_state_in_factor", "const double f = pow(lam, (double)(t - t0 + 1));",
+     "const double f = pow(lam, (double)(t - t0));", 0),
+    ("decay_quadratic_final_state_exponent", "const double w = pow(lam, (double)(t1 - 1 - s));",
+     "const double w = pow(lam, (double)(t1 - s));", 0),
+    ("decay_blocked_intra_exponent", "const double w = score * pow(lam, (double)(t - s));",
+     "const double w = score * pow(lam, (double)(s - t));", 1),
+    ("decay_blocked_inter_factor", "const double f = pow(lam, (double)(t - b0 + 1));",
+     "const double f = pow(lam, (double)(t - b0));", 0),
+    ("decay_blocked_state_factor", "const double f = pow(lam, (double)(b1 - b0));",
+     "const double f = pow(lam, (double)(b1 - b0 - 1));", 0),
+    ("decay_segmented_local_exponent", "const double w = pow(lam, (double)(s1 - 1 - s));",
+     "const double w = pow(lam, (double)(s1 - s));", 0),
+    ("decay_segmented_prefix_factor", "const double f = pow(lam, (double)(s0 - e2));",
+     "const double f = pow(lam, (double)(s0 - e2 + 1));", 0),
+    ("decay_decode_decays_new_token",
+     "S[(size_t)a * d + b] = lam * S[(size_t)a * d + b] + ka * widen_bf16(vp[b]);",
+     "S[(size_t)a * d + b] = lam * (S[(size_t)a * d + b] + ka * widen_bf16(vp[b]));", 0),
 ]
 
 

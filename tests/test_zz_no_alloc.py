@@ -10,8 +10,9 @@ the fp64 oracle under the tolerances of the other parity tests, for both
 output dtypes, with and without a carried-in state; the shapes include one
 just under the scratch limit and one where the segments are lengthened past
 65536 tokens (the state then reaches the inter-block product as bf16 hi + lo).
-A second comparison against la_prefill on the same inputs checks that the two
-entry points compute the same thing.  This file is collected last on purpose."""
+A second comparison against la_prefill on the same inputs, run with the
+segment length the scratch-bound call chose, checks that the two entry points
+compute the same thing.  This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -84,8 +85,13 @@ def test_noalloc_matches_oracle_twice(oracle_mod, case, out_dtype, with_state):
         what = f"{B}x{N}x{H} {out_dtype} state={with_state} call {call}"
         check_out(to_np(out[:, :, hsel]), ref, bf16_out=bf16, what=what)
         check_state(to_np(st[:, hsel]), rst, what=what)
-        # the workspace entry point on the same inputs agrees too
-        ref_out, ref_st = la.prefill(q, k, v, state_in=s_in, out_dtype=out_dtype)
+        # the workspace entry point on the same inputs, with the segment length
+        # the scratch-bound call chose, computes the same outputs and states
+        la.set_segment_len(la.last_segment_len())
+        try:
+            ref_out, ref_st = la.prefill(q, k, v, state_in=s_in, out_dtype=out_dtype)
+        finally:
+            la.set_segment_len(0)
         assert la.get_device_status() == la.LA_OK
         check_out(to_np(out[:, :, hsel]), to_np(ref_out[:, :, hsel]), bf16_out=bf16, what=what + " vs la_prefill")
         check_state(to_np(st), to_np(ref_st), what=what + " vs la_prefill")
