@@ -12,8 +12,9 @@
  * updated by S += K_b^T V_b ("MiniMax-01技术报告解读", §2.2 线性注意力: the
  * right-product kernel trick, the recursively updated KV product, intra-block
  * left product and inter-block right product over row blocks of Q/K/V).
- * No scale, feature map, normalisation or decay is applied inside the
- * operation: callers pass q/k/v already scaled.
+ * No scale, feature map or normalisation is applied inside the operation:
+ * callers pass q/k/v already scaled.  A per-head decay is applied only by the
+ * *_decay entry points below.
  *
  * Conventions shared by every entry point
  *   - Ownership: the caller allocates and owns every buffer (inputs, outputs,
@@ -130,6 +131,49 @@ LA_API la_status la_prefill_varlen(const void *q, const void *k, const void *v,
 LA_API la_status la_decode_step(const void *q, const void *k, const void *v, float *state,
                          void *out, la_dtype out_dtype, int B, int H, int d,
                          cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Per-head decay.  "MiniMax-01技术报告解读" §3.3 item 1 names a decay value
+ * computation fused into the prefill but gives no formula; these entry points
+ * take the reading of the TransNormer / Lightning Attention line: one constant
+ * lambda_h in (0, 1] per head h and the decayed recurrence
+ *
+ *     S_t = lambda_h S_{t-1} + k_t^T v_t,   o_t = q_t S_t,   S_{-1} = S_in
+ *   i.e.
+ *     o_t = sum_{s <= t} lambda^{t-s} (q_t . k_s) v_s + lambda^{t+1} q_t S_in
+ *     S   = lambda^{n} S_in + sum_s lambda^{n-1-s} k_s^T v_s     (n tokens)
+ *
+ * with t counted from the start of each sequence.  lambda_h = 1 on every head
+ * is the undecayed operation (to rounding).  The blocked form keeps the
+ * decayed keys of the state update exact to ~2^-16 (a bf16 hi + lo pair), so
+ * the fp32 state meets the same error bound as without decay.
+ *
+ *   decay   DEVICE fp32 [H], 4-byte aligned, read only.  Checked on the device:
+ *           a value outside (0, 1] (or NaN) computes nothing and records
+ *           LA_ERR_INVALID_ARGUMENT in the sticky word (la_prefill_*_decay:
+ *           the whole call; la_decode_step_decay: the rows of that head).
+ *   block   0 or 128.  Other arguments, layouts, workspace sizes (those of
+ *           la_prefill / la_prefill_varlen) and errors as without decay;
+ *           decay = NULL is LA_ERR_INVALID_ARGUMENT.
+ * ------------------------------------------------------------------------- */
+LA_API la_status la_prefill_decay(const void *q, const void *k, const void *v,
+                                  int B, int N, int H, int d, int block, const float *decay,
+                                  const float *state_in, void *out, la_dtype out_dtype,
+                                  float *state_out, void *workspace, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+LA_API la_status la_prefill_varlen_decay(const void *q, const void *k, const void *v,
+                                         const int *cu_seqlens, int nseq, int total_tokens,
+                                         int max_seqlen, int H, int d, int block,
+                                         const float *decay, const float *state_in, void *out,
+                                         la_dtype out_dtype, float *state_out, void *workspace,
+                                         size_t ws_bytes, cudaStream_t stream);
+
+/* S <- lambda_h S + k^T v, o = q S for every (b, h); as la_decode_step otherwise. */
+LA_API la_status la_decode_step_decay(const void *q, const void *k, const void *v,
+                                      const float *decay, float *state, void *out,
+                                      la_dtype out_dtype, int B, int H, int d,
+                                      cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * State slots and the mixed prefill/decode step ("MiniMax-01技术报告解读",

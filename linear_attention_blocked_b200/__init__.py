@@ -7,6 +7,8 @@ ABI (include/lightning_attn.h).  Entry points:
   prefill(q, k, v, ...)                      la_prefill          [B, N, H, 128]
   prefill_varlen(q, k, v, cu_seqlens, ...)   la_prefill_varlen   [T, H, 128] packed
   decode_step(q, k, v, state, ...)           la_decode_step      [B, H, 128]
+                                             (each of the three with decay=<fp32 [H] on the
+                                             device>: la_*_decay, per-head decay lambda_h)
   prefill_varlen_slots / decode_step_slots   the same on a pool of per-request states
   mixed_step(q, k, v, cu_seqlens, ...)       la_mixed_step: prefill chunks and decode tokens
                                              of one batch on two streams (plan with

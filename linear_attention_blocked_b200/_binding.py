@@ -26,7 +26,8 @@ EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_worksp
             "la_last_segment_len", "la_kernel_launches", "la_prefill_noalloc",
             "la_prefill_varlen_slots", "la_decode_step_slots", "la_mixed_step",
             "la_kv_aggregate_workspace_size", "la_kv_aggregate", "la_state_prefix",
-            "la_prefill_backward_workspace_size", "la_prefill_backward")
+            "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_decay",
+            "la_prefill_varlen_decay", "la_decode_step_decay")
 
 
 class LAError(RuntimeError):
@@ -67,6 +68,14 @@ def lib():
         L.la_prefill_noalloc.restype = c_int
         L.la_decode_step.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
         L.la_decode_step.restype = c_int
+        L.la_prefill_decay.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, vp, c_int, vp, vp,
+                                       sz, vp]
+        L.la_prefill_decay.restype = c_int
+        L.la_prefill_varlen_decay.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int, vp,
+                                              vp, vp, c_int, vp, vp, sz, vp]
+        L.la_prefill_varlen_decay.restype = c_int
+        L.la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
+        L.la_decode_step_decay.restype = c_int
         L.la_prefill_varlen_slots.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
                                               vp, c_int, vp, c_int, vp, sz, vp]
         L.la_prefill_varlen_slots.restype = c_int
@@ -157,9 +166,20 @@ def _alloc_workspace(nbytes, device):
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
+def _need_decay(decay, H, device):
+    if decay is None:
+        return None
+    _need(decay, "decay", torch.float32, (H,))
+    if decay.device != device:
+        raise ValueError("decay must be on the device of q")
+    return decay
+
+
 def prefill(q, k, v, block: int = 0, state_in=None, out=None, out_dtype=torch.bfloat16,
-            state_out=None, want_state: bool = True, workspace=None, stream=None):
-    """la_prefill on [B, N, H, d] bf16 tensors. Returns (out, state_out or None)."""
+            state_out=None, want_state: bool = True, workspace=None, stream=None, decay=None):
+    """la_prefill on [B, N, H, d] bf16 tensors (la_prefill_decay when `decay`,
+    a device fp32 [H] tensor of per-head decays in (0, 1], is given).
+    Returns (out, state_out or None)."""
     if q.dim() != 4:
         raise ValueError("q must be [B, N, H, d]")
     B, N, H, d = q.shape
@@ -174,20 +194,28 @@ def prefill(q, k, v, block: int = 0, state_in=None, out=None, out_dtype=torch.bf
         state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
     if state_out is not None:
         _need(state_out, "state_out", torch.float32, (B, H, d, d))
+    decay = _need_decay(decay, H, q.device)
     ws_bytes = workspace_size(B, N, H, d, block)
     if workspace is None:
         workspace = _alloc_workspace(ws_bytes, q.device)
-    st = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), B, N, H, d, block, _ptr(state_in), _ptr(out),
-                          _out_code(out.dtype), _ptr(state_out), _ptr(workspace),
-                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
-    _check(st, "la_prefill")
+    if decay is None:
+        st = lib().la_prefill(_ptr(q), _ptr(k), _ptr(v), B, N, H, d, block, _ptr(state_in), _ptr(out),
+                              _out_code(out.dtype), _ptr(state_out), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream_handle(stream))
+        _check(st, "la_prefill")
+    else:
+        st = lib().la_prefill_decay(_ptr(q), _ptr(k), _ptr(v), B, N, H, d, block, _ptr(decay), _ptr(state_in),
+                                    _ptr(out), _out_code(out.dtype), _ptr(state_out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream_handle(stream))
+        _check(st, "la_prefill_decay")
     return out, state_out
 
 
 def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, block: int = 0, state_in=None, out=None,
                    out_dtype=torch.bfloat16, state_out=None, want_state: bool = True, workspace=None,
-                   stream=None):
-    """la_prefill_varlen on packed [T, H, d] tensors with device int32 cu_seqlens."""
+                   stream=None, decay=None):
+    """la_prefill_varlen on packed [T, H, d] tensors with device int32 cu_seqlens
+    (la_prefill_varlen_decay when `decay`, device fp32 [H], is given)."""
     if q.dim() != 3:
         raise ValueError("q must be [T, H, d]")
     T, H, d = q.shape
@@ -206,19 +234,28 @@ def prefill_varlen(q, k, v, cu_seqlens, max_seqlen: int, block: int = 0, state_i
         state_out = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device)
     if state_out is not None:
         _need(state_out, "state_out", torch.float32, (nseq, H, d, d))
+    decay = _need_decay(decay, H, q.device)
     ws_bytes = varlen_workspace_size(nseq, T, max_seqlen, H, d, block)
     if workspace is None:
         workspace = _alloc_workspace(ws_bytes, q.device)
-    st = lib().la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, int(max_seqlen),
-                                 H, d, block, _ptr(state_in), _ptr(out), _out_code(out.dtype),
-                                 _ptr(state_out), _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream_handle(stream))
-    _check(st, "la_prefill_varlen")
+    if decay is None:
+        st = lib().la_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, int(max_seqlen),
+                                     H, d, block, _ptr(state_in), _ptr(out), _out_code(out.dtype),
+                                     _ptr(state_out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream_handle(stream))
+        _check(st, "la_prefill_varlen")
+    else:
+        st = lib().la_prefill_varlen_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), nseq, T, int(max_seqlen),
+                                           H, d, block, _ptr(decay), _ptr(state_in), _ptr(out),
+                                           _out_code(out.dtype), _ptr(state_out), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size(), _stream_handle(stream))
+        _check(st, "la_prefill_varlen_decay")
     return out, state_out
 
 
-def decode_step(q, k, v, state, out=None, out_dtype=torch.bfloat16, stream=None):
-    """la_decode_step on [B, H, d] bf16 tensors; `state` [B, H, d, d] fp32 is updated in place."""
+def decode_step(q, k, v, state, out=None, out_dtype=torch.bfloat16, stream=None, decay=None):
+    """la_decode_step on [B, H, d] bf16 tensors; `state` [B, H, d, d] fp32 is updated in place
+    (la_decode_step_decay when `decay`, device fp32 [H], is given)."""
     if q.dim() != 3:
         raise ValueError("q must be [B, H, d]")
     B, H, d = q.shape
@@ -228,9 +265,15 @@ def decode_step(q, k, v, state, out=None, out_dtype=torch.bfloat16, stream=None)
     if out is None:
         out = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
     _need(out, "out", out.dtype, (B, H, d))
-    st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), _out_code(out.dtype),
-                              B, H, d, _stream_handle(stream))
-    _check(st, "la_decode_step")
+    decay = _need_decay(decay, H, q.device)
+    if decay is None:
+        st = lib().la_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(state), _ptr(out), _out_code(out.dtype),
+                                  B, H, d, _stream_handle(stream))
+        _check(st, "la_decode_step")
+    else:
+        st = lib().la_decode_step_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(decay), _ptr(state), _ptr(out),
+                                        _out_code(out.dtype), B, H, d, _stream_handle(stream))
+        _check(st, "la_decode_step_decay")
     return out
 
 

@@ -2,7 +2,9 @@
 //
 // "MiniMax-01技术报告解读", §3.3 items 1-2: length-1 tokens run in a kernel of
 // their own whose KV computation is fused with the update of the prefix-KV
-// cache.  For every (b, h):  S <- S + k^T v  (in place),  o = q S  (inclusive).
+// cache.  For every (b, h):  S <- S + k^T v  (in place),  o = q S  (inclusive);
+// with a per-head decay lambda_h (the decayed recurrence, read from §3.3
+// item 1's decay computation):  S <- lambda_h S + k^T v.
 //
 // The step is a pure stream over the state (read 64 KiB, write 64 KiB per
 // (b, h) at d = 128), so the kernel is built for HBM bandwidth: one CTA of
@@ -40,7 +42,7 @@ __global__ void __launch_bounds__(DEC_THREADS)
 la_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                  const __nv_bfloat16 *__restrict__ v, float *__restrict__ state, void *__restrict__ out,
                  int out_fp32, long long npairs, int H, const int *__restrict__ slots, int n_slots,
-                 int *status) {
+                 const float *__restrict__ decay, int *status) {
     constexpr int Dd = 128;
     __shared__ float red[8][Dd];
     __shared__ float qs[Dd], ks[Dd];
@@ -57,6 +59,15 @@ la_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
                 continue;
             }
             spair = (long long)slot * H + (pair - b * H);
+        }
+        // per-head decay lambda (1 without decay): S <- lambda S + k^T v
+        float lam = 1.f;
+        if (decay) {
+            lam = decay[pair % H];
+            if (!(lam > 0.f && lam <= 1.f)) {  // uniform across the block; also rejects NaN
+                if (tid == 0) atomicCAS(status, 0, 1);
+                continue;
+            }
         }
         float *S = state + (size_t)spair * Dd * Dd;
         float4 s[DEC_ROWS_PER_THREAD];
@@ -76,10 +87,10 @@ la_decode_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__res
             const int i = g + 8 * m;
             const float ki = ks[i], qi = qs[i];
             float4 x = s[m];
-            x.x = fmaf(ki, va.x, x.x);  // S[i][j] += k_i v_j
-            x.y = fmaf(ki, va.y, x.y);
-            x.z = fmaf(ki, vb.x, x.z);
-            x.w = fmaf(ki, vb.y, x.w);
+            x.x = fmaf(ki, va.x, lam * x.x);  // S[i][j] = lambda S[i][j] + k_i v_j
+            x.y = fmaf(ki, va.y, lam * x.y);
+            x.z = fmaf(ki, vb.x, lam * x.z);
+            x.w = fmaf(ki, vb.y, lam * x.w);
             st_stream_f4(S + (size_t)i * Dd + 4 * c, x);
             acc.x = fmaf(qi, x.x, acc.x);  // o_j += q_i S'[i][j]
             acc.y = fmaf(qi, x.y, acc.y);

@@ -83,7 +83,10 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int choose_seg_len(int nseq, long long T, int H) {
     const int ov = g_seg_len_override.load();
     if (ov > 0) return ov;
-    int L = (H <= 16) ? 2048 : 1024;
+    // Longer segments for few heads: each (sequence, head) scan then has fewer
+    // cross-SM hand-offs in its chain (measured at H = 8, N = 1M: 6.2 / 3.3 /
+    // 2.5 / 2.5 / 2.7 ms for 1024 / 2048 / 4096 / 8192 / 16384 tokens).
+    int L = (H <= 16) ? 4096 : 1024;
     const long long target = 2 * 148;  // want at least ~2 items per SM of a B200
     while (L > la::BLK) {
         const long long segs = (T + L - 1) / L + 0;  // lower bound of segments over all sequences
@@ -143,7 +146,7 @@ la_status ensure_smem_attr(SmemAttr &a, Kernel *kernel, int bytes) {
     return LA_OK;
 }
 
-SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_agg;
+SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_prefill_decay, g_attr_prefill_b64, g_attr_agg;
 
 bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
     if (!a || !b || na == 0 || nb == 0) return false;
@@ -155,16 +158,22 @@ la_status check_common(int H, int d, int block, la_dtype out_dtype) {
     if (H <= 0 || d <= 0 || block < 0) return LA_ERR_INVALID_ARGUMENT;
     if (out_dtype != LA_BF16 && out_dtype != LA_FP32) return LA_ERR_INVALID_ARGUMENT;
     if (d != la::D) return LA_ERR_UNSUPPORTED;
-    if (block != 0 && block != la::BLK) return LA_ERR_UNSUPPORTED;
+    if (block != 0 && block != 64 && block != la::BLK) return LA_ERR_UNSUPPORTED;
     return LA_OK;
 }
+
+// The prefill kernel instantiation for a row-block length (0 = 128).
+template <bool ANTI, bool DECAY>
+la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                         const la::PrefillParams &pp, cudaStream_t stream);
 
 // Shared body of la_prefill / la_prefill_varlen.
 la_status prefill_impl(const void *q, const void *k, const void *v, const int *cu, int fixed_len,
                        int nseq, long long T, int max_seqlen, int H, int d, int block,
                        const float *state_in, void *out, la_dtype out_dtype, float *state_out,
                        void *workspace, size_t ws_bytes, cudaStream_t stream,
-                       const int *slots = nullptr, int n_slots = 0, bool anti = false) {
+                       const int *slots = nullptr, int n_slots = 0, bool anti = false,
+                       const float *decay = nullptr) {
     la_status st = check_common(H, d, block, out_dtype);
     if (st != LA_OK) return st;
     if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -178,6 +187,8 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     const size_t n_in = (size_t)T * H * la::D * 2, n_out = (size_t)T * H * la::D * esz;
     if (slots && (n_slots <= 0 || !aligned(slots, 4) || state_in != state_out || !state_out))
         return LA_ERR_INVALID_ARGUMENT;
+    if (decay && (anti || !aligned(decay, 4))) return LA_ERR_INVALID_ARGUMENT;
+    if (block == 64 && (anti || decay)) return LA_ERR_UNSUPPORTED;
     const size_t n_state = (size_t)(slots ? n_slots : nseq) * H * la::D * la::D * 4;
     if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
@@ -220,6 +231,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     sp.state_out = state_out;
     sp.slots = slots;
     sp.n_slots = n_slots;
+    sp.decay = decay;
     sp.status = status;
     la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
@@ -246,26 +258,42 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
     pp.anti_lo = anti && max_seqlen > LA_LO_SPLIT_FROM;
+    pp.decay = decay;
     pp.seg_len = L;
     pp.status = status;
 
-    st = anti ? ensure_smem_attr(g_attr_prefill_anti, la::la_prefill_kernel<true>, la::PREFILL_SMEM)
-              : ensure_smem_attr(g_attr_prefill, la::la_prefill_kernel<false>, la::PREFILL_SMEM);
-    if (st != LA_OK) return st;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    if (anti)
-        la::la_prefill_kernel<true><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
-    else
-        la::la_prefill_kernel<false><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
-    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    st = anti ? launch_prefill<true, false>(block, grid, mq, mk, mv, pp, stream)
+         : decay ? launch_prefill<false, true>(block, grid, mq, mk, mv, pp, stream)
+                 : launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream);
+    if (st != LA_OK) return st;
     ++g_launches;
     return LA_OK;
 }
 
+template <bool ANTI, bool DECAY, int BK>
+la_status launch_prefill_bk(SmemAttr &attr, int grid, const CUtensorMap &mq, const CUtensorMap &mk,
+                            const CUtensorMap &mv, const la::PrefillParams &pp, cudaStream_t stream) {
+    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<ANTI, DECAY, BK>, la::PREFILL_SMEM);
+    if (st != LA_OK) return st;
+    la::la_prefill_kernel<ANTI, DECAY, BK><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+template <bool ANTI, bool DECAY>
+la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                         const la::PrefillParams &pp, cudaStream_t stream) {
+    if (ANTI) return launch_prefill_bk<true, false, 128>(g_attr_prefill_anti, grid, mq, mk, mv, pp, stream);
+    if (DECAY) return launch_prefill_bk<false, true, 128>(g_attr_prefill_decay, grid, mq, mk, mv, pp, stream);
+    if (block == 64) return launch_prefill_bk<false, false, 64>(g_attr_prefill_b64, grid, mq, mk, mv, pp, stream);
+    return launch_prefill_bk<false, false, 128>(g_attr_prefill, grid, mq, mk, mv, pp, stream);
+}
+
 // Shared body of la_decode_step / la_decode_step_slots.
 la_status decode_impl(const void *q, const void *k, const void *v, float *state, const int *slots, int n_slots,
-                      void *out, la_dtype out_dtype, int B, int H, int d, cudaStream_t stream) {
+                      void *out, la_dtype out_dtype, int B, int H, int d, cudaStream_t stream,
+                      const float *decay = nullptr) {
     la_status st = check_common(H, d, 0, out_dtype);
     if (st != LA_OK) return st;
     if (B < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -275,6 +303,7 @@ la_status decode_impl(const void *q, const void *k, const void *v, float *state,
     for (const void *p : ptrs)
         if (!aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
     if (slots && (n_slots <= 0 || !aligned(slots, 4))) return LA_ERR_INVALID_ARGUMENT;
+    if (decay && !aligned(decay, 4)) return LA_ERR_INVALID_ARGUMENT;
     const long long npairs = (long long)B * H;
     const long long nstates = (slots ? (long long)n_slots : (long long)B) * H;
     const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
@@ -287,7 +316,7 @@ la_status decode_impl(const void *q, const void *k, const void *v, float *state,
     la::la_decode_kernel<<<(unsigned)grid, la::DEC_THREADS, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
         static_cast<const __nv_bfloat16 *>(v), state, out, out_dtype == LA_FP32, npairs, H, slots, n_slots,
-        status);
+        decay, status);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
     ++g_launches;
     return LA_OK;
@@ -412,6 +441,31 @@ la_status la_decode_step_slots(const void *q, const void *k, const void *v, floa
     return decode_impl(q, k, v, state_pool, slots, n_slots, out, out_dtype, B, H, d, stream);
 }
 
+la_status la_prefill_decay(const void *q, const void *k, const void *v, int B, int N, int H, int d, int block,
+                           const float *decay, const float *state_in, void *out, la_dtype out_dtype,
+                           float *state_out, void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (B < 0 || N < 0 || !decay) return LA_ERR_INVALID_ARGUMENT;
+    const long long T = (long long)B * N;
+    return prefill_impl(q, k, v, nullptr, N, B, T, N, H, d, block, state_in, out, out_dtype, state_out,
+                        workspace, ws_bytes, stream, nullptr, 0, false, decay);
+}
+
+la_status la_prefill_varlen_decay(const void *q, const void *k, const void *v, const int *cu_seqlens, int nseq,
+                                  int total_tokens, int max_seqlen, int H, int d, int block, const float *decay,
+                                  const float *state_in, void *out, la_dtype out_dtype, float *state_out,
+                                  void *workspace, size_t ws_bytes, cudaStream_t stream) {
+    if (!cu_seqlens || nseq < 0 || total_tokens < 0 || !decay) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARGUMENT;
+    return prefill_impl(q, k, v, cu_seqlens, 0, nseq, total_tokens, max_seqlen, H, d, block, state_in,
+                        out, out_dtype, state_out, workspace, ws_bytes, stream, nullptr, 0, false, decay);
+}
+
+la_status la_decode_step_decay(const void *q, const void *k, const void *v, const float *decay, float *state,
+                               void *out, la_dtype out_dtype, int B, int H, int d, cudaStream_t stream) {
+    if (!decay) return LA_ERR_INVALID_ARGUMENT;
+    return decode_impl(q, k, v, state, nullptr, 0, out, out_dtype, B, H, d, stream, decay);
+}
+
 la_status la_mixed_step(const void *q, const void *k, const void *v, const int *cu_seqlens,
                         const int *prefill_slots, int n_prefill, int prefill_tokens, int max_seqlen,
                         const int *decode_slots, int n_decode, int H, int d, float *state_pool, int n_slots,
@@ -475,7 +529,7 @@ const char *la_status_string(la_status s) {
     switch (s) {
         case LA_OK: return "ok";
         case LA_ERR_INVALID_ARGUMENT: return "invalid argument";
-        case LA_ERR_UNSUPPORTED: return "unsupported (only d = 128 and block 0/128 are built)";
+        case LA_ERR_UNSUPPORTED: return "unsupported (d = 128 only; row blocks 0/64/128, 64 without decay)";
         case LA_ERR_CUDA: return "CUDA error";
         case LA_ERR_TIMEOUT: return "a bounded device-side wait ran out";
         case LA_ERR_WORKSPACE: return "workspace missing or too small";
@@ -777,6 +831,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     sp.state_out = state_out;
     sp.slots = nullptr;
     sp.n_slots = 0;
+    sp.decay = nullptr;
     sp.status = status;
     la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
@@ -802,14 +857,13 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
     pp.anti_lo = 0;
+    pp.decay = nullptr;
     pp.seg_len = L;
     pp.status = status;
-    st = ensure_smem_attr(g_attr_prefill, la::la_prefill_kernel<false>, la::PREFILL_SMEM);
-    if (st != LA_OK) return st;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    la::la_prefill_kernel<false><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
-    if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
+    st = launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream);
+    if (st != LA_OK) return st;
     ++g_launches;
     return LA_OK;
 }

@@ -34,6 +34,26 @@
 // exactly when the forward would need it somewhere in the sequence: when the
 // host sets p.anti_lo (sequences longer than LA_LO_SPLIT_FROM tokens).
 //
+// A second template flag, DECAY, adds a per-head decay lambda_h in (0, 1]
+// (the "decay value computation" of "MiniMax-01技术报告解读" §3.3 item 1, read
+// as the decayed recurrence S_t = lambda S_{t-1} + k_t^T v_t, o_t = q_t S_t).
+// With r the row in a block of nb rows:
+//       P[r][c] = bf16(Sc[r][c] lambda^{r-c})           a3 (decay in the mask)
+//       O       = P V + lambda^{r+1} Q S_{<b}           a4 into O buffer 0, a5 into
+//                                                       buffer 1, combined by the
+//                                                       store warps in fp32
+//       S      <- lambda^{nb} S + (Lambda K)^T V        a6, Lambda = lambda^{nb-1-r}
+//       A_j     = sum_b (Lambda_b K_b)^T V_b            phase A, rows scaled to the
+//                                                       segment end
+//       INCL_j  = lambda^{len_j} E_j + A_j              phase L
+// The row-scaled keys Lambda K are split into a bf16 pair hi + lo (x = hi +
+// lo to within 2^-16 |x|), so the state sees the decayed keys as exactly as
+// the undecayed state sees the raw ones: hi is written over the K tile once
+// the scores have read it, lo into the block's Q slot once a5 has read it (in
+// phase A: into the snapshot buffer, idle there), and a6 is the two products
+// hi^T V + lo^T V.  The state warps rescale S by lambda^{nb} in TMEM when they
+// take each snapshot.  DECAY and ANTI are not combined.
+//
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
 //               loads Q
@@ -129,6 +149,7 @@ struct PrefillParams {
     unsigned long long wait_limit_ns;
     int inject;
     int anti_lo;            // ANTI: hand S to a5 as hi + lo (the sequences are long)
+    const float *decay;     // DECAY: lambda_h per head, [H] (validated by the scheduler)
     int *status;            // sticky device status word
 };
 
@@ -147,10 +168,13 @@ struct CtrlBlock {
     uint64_t snap_empty;          // [1] a5 has read the snapshot
     uint64_t agg_full;            // [1] phase A done: A_j in the first block's O buffer
     uint64_t a_free;              // [4] state warps: A_j read, that O buffer is free
-    uint64_t incl_stored;         // [4] state warps: INCL_j written to the workspace
+    uint64_t incl_stored;         // [4] state warps: their rows of INCL_j are in the workspace
     uint64_t item_full[2];        // [1] producer
     uint64_t item_empty[2];       // [14] Q producer lane + MMA lane 0 + 3 x 4 warps
     uint64_t fin;                 // [1] tear-down: every MMA done
+    uint64_t a5_done;             // [1] DECAY: a5 of a block done (its Q slot may take K lo)
+    uint64_t alo_free;            // [1] DECAY: the phase-A lo tile (snapshot buffer) is free
+    uint64_t alo_ready;           // [4] DECAY: a phase-A K tile is scaled (hi in place, lo)
     int item[2][8];
     uint32_t tmem_base;
     volatile int abort;
@@ -252,13 +276,22 @@ __device__ __forceinline__ void tmem_ld_wait32(uint32_t taddr, uint32_t (&x)[32]
     reg_fence(x);
 }
 
+// Multiply 32 fp32 words (bit patterns) by c in place.
+__device__ __forceinline__ void scale32(uint32_t (&x)[32], float c) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = __float_as_uint(__uint_as_float(x[i]) * c);
+}
+
 // Read S from TMEM and hand it to a5 through the snapshot buffer: either the
 // whole state as bf16 (one arrival; columns 0-63 in `shi`, 64-127 in `slo`),
 // or, when `lo`, as bf16 hi + lo one 64-column half at a time (two arrivals).
 // The last arrival also tells the MMA warp that S has been read, so a6 may
-// overwrite it.
+// overwrite it.  DECAY: S is also written back multiplied by `wb` (the decay
+// lambda^{nb} of the block whose update a6 adds next) before the arrival.
+template <bool DECAY>
 __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint8_t *slo, int r, int lane, bool lo,
-                                            uint32_t &snap_n, const PrefillParams &p, CtrlBlock *cb) {
+                                            uint32_t &snap_n, const PrefillParams &p, CtrlBlock *cb,
+                                            float wb = 1.f) {
     if (!lo) {
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {  // columns [64 hf, 64 hf + 64) -> shi (hf = 0) or slo (hf = 1)
@@ -271,7 +304,15 @@ __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint
                 *reinterpret_cast<uint4 *>(half + r * 128 + ((q ^ (r & 7)) << 4)) =
                     make_uint4(bf16x2_round(x[8 * q], x[8 * q + 1]), bf16x2_round(x[8 * q + 2], x[8 * q + 3]),
                                bf16x2_round(x[8 * q + 4], x[8 * q + 5]), bf16x2_round(x[8 * q + 6], x[8 * q + 7]));
+            if (DECAY) {
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    scale32(*reinterpret_cast<uint32_t(*)[32]>(&x[32 * c2]), wb);
+                    tmem_st32(trow + TM_S + hf * 64 + 32 * c2, *reinterpret_cast<uint32_t(*)[32]>(&x[32 * c2]));
+                }
+            }
         }
+        if (DECAY) tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -297,7 +338,12 @@ __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint
                 *reinterpret_cast<uint4 *>(shi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
                 *reinterpret_cast<uint4 *>(slo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
             }
+            if (DECAY) {
+                scale32(x, wb);
+                tmem_st32(trow + TM_S + hf * 64 + qq * 32, x);
+            }
         }
+        if (DECAY) tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
@@ -305,6 +351,52 @@ __device__ __forceinline__ bool snapshot_state(uint32_t trow, uint8_t *shi, uint
         ++snap_n;
     }
     return true;
+}
+
+// Release the hand-off flag of a segment once all four state warps have
+// stored their rows of its inclusive prefix (incl_stored); `leader` is the one
+// thread that waits and releases.  Its acquire on the barrier orders the other
+// warps' stores before the gpu-scope release of the flag.
+__device__ __forceinline__ bool publish_incl(bool leader, uint32_t pub_n, int *flag, const PrefillParams &p,
+                                          CtrlBlock *cb) {
+    if (!leader) return true;
+    const bool all_in = wait_or_abort(&cb->incl_stored, pub_n & 1, p, cb);
+    if (all_in && p.inject != LA_INJECT_SKIP_PUBLISH) {
+        const int two = 2;
+        asm volatile("fence.acq_rel.gpu;" ::: "memory");
+        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(two) : "memory");
+    }
+    return all_in;
+}
+
+// lambda^n for n >= 0 from log2(lambda) (lambda in (0, 1]: exact 1 for n = 0
+// or lambda = 1; underflows to 0 where the true power is below fp32 range).
+__device__ __forceinline__ float decay_pow(float l2, int n) { return exp2f(l2 * (float)n); }
+
+// DECAY: scale row r of a swizzled [128 x 128] bf16 tile by c and split the
+// fp32 products into bf16 hi (written back in place) and lo (written at the
+// same offsets of `lo_tile`): x = hi + lo with |x - hi - lo| <= 2^-17 |x|.
+// One thread per row; every 16-byte chunk is read once and written twice.
+__device__ __forceinline__ void scale_row_hi_lo(uint8_t *tile, uint8_t *lo_tile, int r, float c) {
+#pragma unroll 4
+    for (int ch = 0; ch < 16; ++ch) {
+        const uint32_t off = sw_off(r, ch);
+        const uint4 x = *reinterpret_cast<const uint4 *>(tile + off);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float a = __uint_as_float(w[i] << 16) * c;           // low bf16 of the pair
+            const float b = __uint_as_float(w[i] & 0xffff0000u) * c;   // high bf16
+            const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+            hi[i] = *reinterpret_cast<const uint32_t *>(&h);
+            lo[i] = *reinterpret_cast<const uint32_t *>(&l);
+        }
+        *reinterpret_cast<uint4 *>(tile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(lo_tile + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
 }
 
 // Every role reads the same item from the two-slot queue the producer fills.
@@ -320,10 +412,13 @@ __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane
     return item[IT_VALID] != 0;
 }
 
-template <bool ANTI>
+template <bool ANTI, bool DECAY, int BK>
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
+    static_assert(BK == 64 || BK == 128, "row blocks of 64 or 128 tokens");
+    static_assert(BK == 128 || (!ANTI && !DECAY), "64-row blocks: the plain forward only");
+    constexpr bool B64 = BK == 64;  // two 64-row blocks per 128-row tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -357,6 +452,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         mbar_init(&cb->a_free, 4);
         mbar_init(&cb->incl_stored, 4);
         mbar_init(&cb->fin, 1);
+        mbar_init(&cb->a5_done, 1);
+        mbar_init(&cb->alo_free, 1);
+        mbar_init(&cb->alo_ready, 4);
         cb->abort = 0;
         fence_mbarrier_init();
         tma_prefetch_desc(&tmq);
@@ -497,12 +595,18 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         // The whole warp runs this loop in step: every lane holds the same
         // counters, barrier probes are combined with __all_sync, and each MMA or
         // commit is issued by the lane that elect.sync picks.
-        uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0, afree_n = 0;
+        uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0, afree_n = 0, a_n = 0;
         bool ok = true;
         int item[8];
         auto ready = [&](uint64_t *bar, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_test(bar, parity)) != 0;
         };
+        // O buffers: block bn accumulates in buffer bn & 1 (double-buffered);
+        // under DECAY a block uses both (P V in buffer 0, Q S in buffer 1), so
+        // one block is in flight and the barrier phase advances every block.
+        auto ob = [&](uint32_t bn) -> uint32_t { return DECAY ? 0u : (bn & 1); };
+        auto obpar = [&](uint32_t bn) -> uint32_t { return DECAY ? (bn & 1) : ((bn >> 1) & 1); };
+        const uint32_t tm_a = DECAY ? TM_O + 128 : 0;  // DECAY: phase A sums in O buffer 1
         while (ok && next_item(it, item, lane, p, cb)) {
             const int tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
@@ -511,21 +615,31 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             if (!last) {
                 // phase A: A_j = sum_b K_b^T V_b, accumulated in the O buffer of this
                 // item's first block once the block two before it has been read out
-                if (!warp_wait(&cb->o_empty[blk_n & 1], ((blk_n >> 1) & 1) ^ 1, p, cb)) break;
+                // (DECAY: in O buffer 1 once the previous block has been read out)
+                if (!warp_wait(&cb->o_empty[ob(blk_n)], obpar(blk_n) ^ 1, p, cb)) break;
                 tc_fence_after();
+                const uint32_t ta = DECAY ? tmem + tm_a : tmem + TM_O + (blk_n & 1) * 128;
                 for (int b = 0; b < nblk; ++b) {
                     if (cb->abort) { ok = false; break; }
                     const int s = kv_n % KV_STAGES;
+                    if (DECAY) tc_commit_w(&cb->alo_free);  // every MMA so far has read the lo tile
                     if (!warp_wait(&cb->kv_full[s], (kv_n / KV_STAGES) & 1, p, cb)) { ok = false; break; }
+                    if (DECAY && !warp_wait(&cb->alo_ready, a_n & 1, p, cb)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
                     const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BLK / 16; ++kk)
-                        mma_ss_w(tmem + TM_O + (blk_n & 1) * 128, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV,
-                                 (b > 0 || kk > 0) ? 1u : 0u);
+                        mma_ss_w(ta, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, (b > 0 || kk > 0) ? 1u : 0u);
+                    if (DECAY) {  // + (Lambda K)_lo^T V, lo tile in the snapshot buffer
+                        const uint32_t kl = sbase + SM_SHI;
+#pragma unroll
+                        for (int kk = 0; kk < BLK / 16; ++kk)
+                            mma_ss_w(ta, desc_mnmajor(kl, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                    }
                     tc_commit_w(&cb->kv_empty[s]);
                     ++kv_n;
+                    ++a_n;
                 }
                 if (!ok) break;
                 tc_commit_w(&cb->agg_full);
@@ -533,12 +647,14 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             // ---------------- phase O: polled three-chain schedule ----------------
             const bool want_final = last && p.state_out != nullptr;
             const uint32_t kv0 = kv_n, q0 = q_n, blk0 = blk_n;
-            int i2 = 0, i4 = 0, i5 = 0, half = 0;  // next block of a2 / a4 / a5; a5 half pending
+            int i2 = 0, i4 = 0, i5 = 0, sub = 0;  // next block of a2 / a4 / a5; a5 sub-step pending
             uint32_t spins = 0;
             uint64_t deadline = 0;
             while (i4 < nblk) {
                 bool prog = false;
                 // O chain, a4(i4): P ready, a5 of the block issued
+                // (DECAY: P ready also means the block's K rows are scaled into
+                // hi + lo, and a6 follows a4)
                 if (i4 < i5) {
                     const uint32_t bn = blk0 + i4;
                     if (ready(&cb->p_full, bn & 1)) {
@@ -546,9 +662,25 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const int s = (kv0 + i4) % KV_STAGES;
                         const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
 #pragma unroll
-                        for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns
-                            mma_ts_w(tmem + TM_O + (bn & 1) * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV, 1u);
-                        tc_commit_w(&cb->o_full[bn & 1]);
+                        for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns; DECAY: P V
+                            mma_ts_w(tmem + TM_O + ob(bn) * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV,
+                                     (DECAY && kk == 0) ? 0u : 1u);  // has buffer 0 to itself and starts it
+                        if (DECAY) {
+                            const uint32_t qn = q0 + i4;
+                            if ((i4 < nblk - 1) || want_final) {  // a6: S += (Lambda K)_hi^T V + (Lambda K)_lo^T V
+                                const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
+                                const uint32_t kl = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
+#pragma unroll
+                                for (int kk = 0; kk < BLK / 16; ++kk)
+                                    mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+#pragma unroll
+                                for (int kk = 0; kk < BLK / 16; ++kk)
+                                    mma_ss_w(tmem + TM_S, desc_mnmajor(kl, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                                tc_commit_w(&cb->s_done);
+                            }
+                            tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // a5 and a6 have read the Q slot
+                        }
+                        tc_commit_w(&cb->o_full[ob(bn)]);
                         tc_commit_w(&cb->kv_empty[s]);  // a2, a6 and a4 of this block are issued
                         ++i4;
                         prog = true;
@@ -558,52 +690,86 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 // the hi + lo pair) then a6(i5): Q landed (a2 issued), snapshot
                 // ready, the block's O buffer free (block i5 - 2 read out; for the
                 // first block of a segment with a successor, A_j read out of it)
+                // DECAY: a5 goes to O buffer 1 and a6 waits for the scaled keys
                 if (i5 < i2) {
                     const uint32_t bn = blk0 + i5;
                     const bool a_read = last || i5 > 0 || ready(&cb->a_free, afree_n & 1);
-                    if (a_read && ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty[bn & 1], ((bn >> 1) & 1) ^ 1)) {
+                    if (a_read && ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty[ob(bn)], obpar(bn) ^ 1)) {
                         tc_fence_after();
                         const int s = (kv0 + i5) % KV_STAGES;
                         const uint32_t qn = q0 + i5;
                         const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
                         const uint32_t sh = sbase + SM_SHI, sl = sbase + SM_SLO;
+                        const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
+                        const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
+                        const uint32_t tq = DECAY ? tmem + TM_O + 128 : tmem + TM_O + ob(bn) * 128;
                         const bool upd = (i5 < nblk - 1) || want_final;
-                        bool block_done = true;
+                        // sub-step: one snapshot arrival = one column half (hi + lo
+                        // mode) of one row half (64-row blocks) of the tile
+                        const int nch = lo ? 2 : 1;
+                        const int rh = B64 ? sub / nch : 0;  // 64-row blocks: rows 64 rh .. 64 rh + 63
+                        const int ch = sub % nch;            // hi + lo: columns 64 ch .. 64 ch + 63
+                        // 64-row blocks: only the lanes (rows) of this block are written
+                        const uint32_t m_lo = (B64 && rh == 1) ? ~0u : 0u, m_hi = (B64 && rh == 0) ? ~0u : 0u;
                         if (!lo) {  // O = Q S, S = the whole [128 x 128] snapshot
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss_w(tmem + TM_O + (bn & 1) * 128, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF,
-                                         kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                if (B64)
+                                    mma_ss_w_lanes(tq, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, kk > 0 ? 1u : 0u,
+                                                   m_lo, m_lo, m_hi, m_hi);
+                                else
+                                    mma_ss_w(tq, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, kk > 0 ? 1u : 0u);
+                            }
                         } else {  // one 64-column half of O = Q (S_hi + S_lo)
-                            const uint32_t to = tmem + TM_O + (bn & 1) * 128 + half * 64;
+                            const uint32_t to = tq + ch * 64;
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                if (B64)
+                                    mma_ss_w_lanes(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u,
+                                                   m_lo, m_lo, m_hi, m_hi);
+                                else
+                                    mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u);
+                            }
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk)
-                                mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
-                            block_done = half == 1;
-                            half ^= 1;
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                if (B64)
+                                    mma_ss_w_lanes(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u,
+                                                   m_lo, m_lo, m_hi, m_hi);
+                                else
+                                    mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
+                            }
                         }
                         tc_commit_w(&cb->snap_empty);
                         ++snap_n;
-                        if (!last && i5 == 0 && block_done) ++afree_n;
-                        if (block_done) {
-                            tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // a2 and a5 have read the Q tile
-                            if (upd) {  // a6: S += K^T V (S_{<b} has been read out)
-                                const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
-                                const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
+                        const bool rh_done = ch == nch - 1;
+                        const bool tile_done = rh_done && (!B64 || rh == 1);
+                        if (!last && i5 == 0 && tile_done) ++afree_n;
+                        if (B64 && rh_done && rh == 0) {
+                            // S += K_lo^T V_lo over rows 0-63: S_{<b1} for the second block
 #pragma unroll
-                                for (int kk = 0; kk < BLK / 16; ++kk)
-                                    mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
-                                tc_commit_w(&cb->s_done);
+                            for (int kk = 0; kk < BLK / 32; ++kk)
+                                mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                            tc_commit_w(&cb->s_done);
+                        }
+                        if (tile_done) {
+                            if (DECAY) {
+                                tc_commit_w(&cb->a5_done);  // the Q slot may now take the block's K lo
+                            } else {
+                                tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // a2 and a5 have read the Q tile
+                                if (upd) {  // a6: S += K^T V (S_{<b} has been read out); 64-row blocks: rows 64-127
+#pragma unroll
+                                    for (int kk = B64 ? BLK / 32 : 0; kk < BLK / 16; ++kk)
+                                        mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                                    tc_commit_w(&cb->s_done);
+                                }
                             }
                             ++i5;
                         }
+                        sub = tile_done ? 0 : sub + 1;
                         prog = true;
                     }
                 }
-                // intra chain, a2(i2): its score buffer free (a4 of block i2 - 2
+                // intra chain, a2(i2): its score buffer free (a4 of block i2 - 1
                 // issued), tiles landed
                 if (i2 < nblk && i2 <= i4) {
                     const int s = (kv0 + i2) % KV_STAGES;
@@ -675,26 +841,63 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int r = q4 * 32 + lane;          // tile row = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
         constexpr int EXCL = ANTI ? 1 : 0;     // key s kept iff s + EXCL <= t
-        uint32_t it = 0, blk_n = 0;
+        uint32_t it = 0, blk_n = 0, kv_n = 0, q_n = 0, a_n = 0;
         bool ok = true;
         int item[8];
         while (ok && next_item(it, item, lane, p, cb)) {
-            const int nblk = (item[IT_TOK1] - item[IT_TOK0] + BLK - 1) / BLK;
+            const int tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
+            const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
+            const bool last = (item[IT_FLAGS] & ITF_LAST) != 0;
+            const float l2 = DECAY ? log2f(__ldg(p.decay + item[IT_H])) : 0.f;
+            const float lam = DECAY ? exp2f(l2) : 1.f;
+            if (DECAY && !last) {
+                // phase A: scale each K tile's rows to the segment end, row r of
+                // block b by lambda^{len-1-128b-r}, hi in place, lo into the
+                // snapshot buffer (free: every MMA that read it has completed)
+                for (int b = 0; b < nblk; ++b) {
+                    const int s = kv_n % KV_STAGES;
+                    if (!warp_wait(&cb->alo_free, a_n & 1, p, cb)) { ok = false; break; }
+                    if (!warp_wait(&cb->kv_full[s], (kv_n / KV_STAGES) & 1, p, cb)) { ok = false; break; }
+                    scale_row_hi_lo(smem + SM_K + s * TILE_BYTES, smem + SM_SHI, r,
+                                    decay_pow(l2, (tok1 - tok0) - 1 - b * BLK - r));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&cb->alo_ready);
+                    ++kv_n;
+                    ++a_n;
+                }
+                if (!ok) break;
+            }
+            const bool want_final = last && p.state_out != nullptr;
             for (int b = 0; b < nblk; ++b) {
                 // P = bf16(Sc ⊙ M), inclusive mask (exclusive under ANTI), packed
                 // two per 32-bit column over the first 64 score columns
+                // (DECAY: P = bf16(Sc lambda^{r-c}) for c <= r)
                 const uint32_t bn = blk_n + b, tsc = trow + TM_SC;
                 if (!warp_wait(&cb->sc_full, bn & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t x[64];
-                    if (hf == 1 && q4 < 2) {
-                        // rows 0-63 see none of the keys 64-127
+                    if ((hf == 1 && q4 < 2) || (B64 && hf == 0 && q4 >= 2)) {
+                        // rows 0-63 see none of the keys 64-127; with 64-row blocks,
+                        // rows 64-127 (the second block) see none of the keys 0-63
 #pragma unroll
                         for (int w = 0; w < 32; ++w) x[w] = 0u;
                     } else {
                         tmem_ld_cols<64>(tsc + hf * 64, x);
+                        if (DECAY) {
+                            // x[i] *= lambda^{r-c}, c = 64 hf + i, from the top column
+                            // down: the factor restarts at 1 on the diagonal and
+                            // gains one factor lambda per column below it
+                            const int ctop = hf * 64 + 63;
+                            float f = r > ctop ? decay_pow(l2, r - ctop - 1) : 0.f;
+#pragma unroll
+                            for (int i = 63; i >= 0; --i) {
+                                f = (hf * 64 + i == r) ? 1.f : f * lam;
+                                x[i] = __float_as_uint(__uint_as_float(x[i]) * f);
+                            }
+                        }
                         // in place: x[w] <- (x[2w], x[2w+1]) only overwrites words already read
 #pragma unroll
                         for (int w = 0; w < 32; ++w) {
@@ -704,12 +907,26 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                     tmem_st32(tsc + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
                 }
+                if (DECAY && ((b < nblk - 1) || want_final)) {
+                    // keys of the state update: row r scaled by lambda^{nb-1-r} (rows past
+                    // the block's end are zero), hi over the K tile, lo into the Q slot
+                    // once a5 has read it
+                    const int valid = min(BLK, tok1 - (tok0 + b * BLK));
+                    const int s = (kv_n + b) % KV_STAGES;
+                    const uint32_t qn = q_n + b;
+                    if (!warp_wait(&cb->a5_done, bn & 1, p, cb)) { ok = false; break; }
+                    scale_row_hi_lo(smem + SM_K + s * TILE_BYTES, smem + SM_Q + (qn % Q_STAGES) * TILE_BYTES, r,
+                                    r < valid ? decay_pow(l2, valid - 1 - r) : 0.f);
+                    fence_proxy_async_smem();
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cb->p_full);
             }
             blk_n += nblk;
+            kv_n += nblk;
+            q_n += nblk;
         }
     } else if (warp < W_STATE) {
         // ====== warps 6-9: output store (a7), publication of inclusive prefixes ======
@@ -720,32 +937,72 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         bool ok = true;
         int item[8];
         while (ok && next_item(it, item, lane, p, cb)) {
-            const int t = item[IT_T], h = item[IT_H], tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
+            const int h = item[IT_H], tok0 = item[IT_TOK0], tok1 = item[IT_TOK1];
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
             if (!(item[IT_FLAGS] & ITF_LAST)) {
                 // the state warps have written INCL_j: release the flag the next
-                // segment's look-back waits for (this thread's acquire on the
-                // barrier orders their stores before its release)
-                if (r == 0) {
-                    const bool all_in = wait_or_abort(&cb->incl_stored, pub_n & 1, p, cb);
-                    if (all_in && p.inject != LA_INJECT_SKIP_PUBLISH) {
-                        const int two = 2;
-                        int *fl = p.flags + t;
-                        asm volatile("fence.acq_rel.gpu;" ::: "memory");
-                        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(fl), "r"(two) : "memory");
-                    }
-                }
+                // segment's look-back waits for
+                publish_incl(r == 0, pub_n, p.flags + item[IT_T], p, cb);
                 ++pub_n;
             }
+            // DECAY: the inter-block term of row r carries lambda^{r+1}
+            const float fq = DECAY ? decay_pow(log2f(__ldg(p.decay + h)), r + 1) : 1.f;
             for (int b = 0; b < nblk && ok; ++b) {
                 const uint32_t bn = blk_n + b;
                 const int row0 = tok0 + b * BLK;
                 const int valid = min(BLK, tok1 - row0);
-                if (!warp_wait(&cb->o_full[bn & 1], (bn >> 1) & 1, p, cb)) { ok = false; break; }
-                const uint32_t tob = trow + TM_O + (bn & 1) * 128;  // this block's O buffer
+                const uint32_t obuf = DECAY ? 0u : (bn & 1), opar = DECAY ? (bn & 1) : ((bn >> 1) & 1);
+                if (!warp_wait(&cb->o_full[obuf], opar, p, cb)) { ok = false; break; }
+                const uint32_t tob = trow + TM_O + obuf * 128;  // this block's O buffer
                 tc_fence_after();
                 const size_t orow = ((size_t)(row0 + r) * H + h) * D;
-                if (!p.out_fp32) {
+                if (DECAY) {
+                    // out = (P V, buffer 0) + lambda^{r+1} (Q S, buffer 1) in fp32, 32
+                    // columns at a time, each chunk stored as soon as it is formed
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t xi[32], xq[32];
+                        tmem_ld32(tob + 32 * c, xi);
+                        tmem_ld32(tob + 128 + 32 * c, xq);
+                        tmem_wait_ld();
+                        reg_fence(xi);
+                        reg_fence(xq);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            xi[i] = __float_as_uint(fmaf(fq, __uint_as_float(xq[i]), __uint_as_float(xi[i])));
+                        if (c == 3) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&cb->o_empty[0]);
+                        }
+                        if (r < valid) {
+                            if (!p.out_fp32) {
+                                uint32_t w[16];
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) w[i] = bf16x2_round(xi[2 * i], xi[2 * i + 1]);
+                                uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow) + 16 * c;
+                                if (p.out_al32) {
+                                    st_global_cs_v8(o, &w[0]);
+                                    st_global_cs_v8(o + 8, &w[8]);
+                                } else {
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q)
+                                        __stcs(reinterpret_cast<uint4 *>(o + 4 * q), make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+                                }
+                            } else {
+                                uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(p.out) + orow) + 32 * c;
+                                if (p.out_al32) {
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) st_global_cs_v8(o + 8 * q, &xi[8 * q]);
+                                } else {
+#pragma unroll
+                                    for (int q = 0; q < 8; ++q)
+                                        __stcs(reinterpret_cast<uint4 *>(o + 4 * q), make_uint4(xi[4 * q], xi[4 * q + 1], xi[4 * q + 2], xi[4 * q + 3]));
+                                }
+                            }
+                        }
+                    }
+                } else if (!p.out_fp32) {
                     // both 64-column rounds into registers (packed to bf16 as they
                     // arrive), release the O buffer, then write the row with 32-byte
                     // stores: full sectors, and no store queued ahead of the TMEM loads
@@ -813,6 +1070,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool lo = (item[IT_FLAGS] & ITF_LO) != 0;
             const int nblk = (tok1 - tok0 + BLK - 1) / BLK;
             bool ok = true;
+            const float l2 = DECAY ? log2f(__ldg(p.decay + h)) : 0.f;
+            // DECAY: lambda^{nb} of block b (its rows), the factor S takes before a6(b)
+            auto block_decay = [&](int b) -> float { return decay_pow(l2, min(BLK, tok1 - (tok0 + b * BLK))); };
 
             // ---------------- phase L: prefix of this segment ----------------
             const float *src_state = nullptr;  // row-major [D][D] (state_in) ...
@@ -873,8 +1133,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                     for (int q = 0; q < 64; ++q) e[q] = 0u;
                 }
-                tmem_st32(trow + TM_S + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&e[0]));
-                tmem_st32(trow + TM_S + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&e[32]));
+                if (!DECAY || !snap_here) {  // (DECAY with a direct snapshot: stored decayed below)
+                    tmem_st32(trow + TM_S + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(&e[0]));
+                    tmem_st32(trow + TM_S + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&e[32]));
+                }
                 if (snap_here) {
                     uint8_t *half = hf ? slo : shi;
 #pragma unroll
@@ -884,25 +1146,50 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                        bf16x2_round(e[8 * q + 4], e[8 * q + 5]), bf16x2_round(e[8 * q + 6], e[8 * q + 7]));
                 }
                 if (!last) {
+                    // A_j: the first block's O buffer (DECAY: O buffer 1);
+                    // DECAY: INCL_j = lambda^{len} E_j + A_j
+                    const uint32_t ta = DECAY ? TM_O + 128 : TM_O + (blk_n & 1) * 128;
+                    const float fl = DECAY ? decay_pow(l2, tok1 - tok0) : 1.f;
 #pragma unroll
                     for (int qq = 0; qq < 2; ++qq) {
                         uint32_t a[32];
-                        tmem_ld_wait32(trow + TM_O + (blk_n & 1) * 128 + hf * 64 + qq * 32, a);  // A_j: first block's O buffer
+                        tmem_ld_wait32(trow + ta + hf * 64 + qq * 32, a);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, hf * 16 + qq * 8 + c)),
-                                   make_float4(__uint_as_float(e[qq * 32 + 4 * c]) + __uint_as_float(a[4 * c]),
-                                               __uint_as_float(e[qq * 32 + 4 * c + 1]) + __uint_as_float(a[4 * c + 1]),
-                                               __uint_as_float(e[qq * 32 + 4 * c + 2]) + __uint_as_float(a[4 * c + 2]),
-                                               __uint_as_float(e[qq * 32 + 4 * c + 3]) + __uint_as_float(a[4 * c + 3])));
+                        for (int c = 0; c < 8; ++c) {
+                            float4 v;
+                            if (DECAY) {
+                                v = make_float4(fmaf(fl, __uint_as_float(e[qq * 32 + 4 * c]), __uint_as_float(a[4 * c])),
+                                                fmaf(fl, __uint_as_float(e[qq * 32 + 4 * c + 1]), __uint_as_float(a[4 * c + 1])),
+                                                fmaf(fl, __uint_as_float(e[qq * 32 + 4 * c + 2]), __uint_as_float(a[4 * c + 2])),
+                                                fmaf(fl, __uint_as_float(e[qq * 32 + 4 * c + 3]), __uint_as_float(a[4 * c + 3])));
+                            } else {
+                                v = make_float4(__uint_as_float(e[qq * 32 + 4 * c]) + __uint_as_float(a[4 * c]),
+                                                __uint_as_float(e[qq * 32 + 4 * c + 1]) + __uint_as_float(a[4 * c + 1]),
+                                                __uint_as_float(e[qq * 32 + 4 * c + 2]) + __uint_as_float(a[4 * c + 2]),
+                                                __uint_as_float(e[qq * 32 + 4 * c + 3]) + __uint_as_float(a[4 * c + 3]));
+                            }
+                            __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, hf * 16 + qq * 8 + c)), v);
+                        }
+                    }
+                }
+                if (DECAY && snap_here) {  // S = lambda^{nb} E_j, ready for a6 of the first block
+                    const float f0 = block_decay(0);
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        scale32(*reinterpret_cast<uint32_t(*)[32]>(&e[32 * c2]), f0);
+                        tmem_st32(trow + TM_S + hf * 64 + 32 * c2, *reinterpret_cast<uint32_t(*)[32]>(&e[32 * c2]));
                     }
                 }
             }
             if (!last) {  // A_j has been read: its O buffer is free for a5 of the first block
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->a_free);
+                if (lane == 0) {
+                    mbar_arrive(&cb->a_free);
+                    mbar_arrive(&cb->incl_stored);  // this warp's rows of INCL_j are stored
+                }
             }
+            // (the store warps release the flag once all four warps have arrived)
             tmem_wait_st();
             if (snap_here) {
                 fence_proxy_async_smem();
@@ -910,25 +1197,31 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cb->snap_full);
                 ++snap_n;
-            } else if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) {
+            } else if (!snapshot_state<DECAY>(trow, shi, slo, r, lane, lo, snap_n, p, cb, DECAY ? block_decay(0) : 1.f)) {
                 ok = false;
-            }
-            if (!last) {  // INCL_j is written: the store warps release the flag
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&cb->incl_stored);
             }
             if (!__all_sync(0xffffffffu, ok && !cb->abort)) break;
 
             // ------------- phase O: state snapshots and the final state -------------
             const bool want_final = last && p.state_out != nullptr;
             for (int b = 0; b < nblk; ++b) {
+                if (B64) {  // S_{<b1} after the update over the tile's first 64 rows
+                    if (!warp_wait(&cb->s_done, upd_n & 1, p, cb)) { ok = false; break; }
+                    ++upd_n;
+                    tc_fence_after();
+                    if (!snapshot_state<DECAY>(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }
+                }
                 const bool update = (b < nblk - 1) || want_final;
                 if (!update) continue;
                 if (!warp_wait(&cb->s_done, upd_n & 1, p, cb)) { ok = false; break; }
                 ++upd_n;
                 tc_fence_after();
                 if (b < nblk - 1) {
-                    if (!snapshot_state(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }  // S_{<b+1}
+                    if (!snapshot_state<DECAY>(trow, shi, slo, r, lane, lo, snap_n, p, cb,
+                                               DECAY ? block_decay(b + 1) : 1.f)) {  // S_{<b+1}
+                        ok = false;
+                        break;
+                    }
                 } else {
                     // final state of the sequence -> state_out (row-major fp32)
                     float *so = p.state_out + ((size_t)(p.slots ? p.slots[seq] : seq) * H + h) * D * D + (size_t)r * D;
@@ -974,6 +1267,7 @@ struct ScheduleParams {
     float *state_out;
     const int *slots;       // null, or [nseq] state slots in a pool of n_slots
     int n_slots;
+    const float *decay;     // null, or [H] per-head decays, each must lie in (0, 1]
     int *status;
 };
 
@@ -997,6 +1291,11 @@ __global__ void __launch_bounds__(SCHED_THREADS, 1) la_schedule_kernel(const Sch
     if (s.slots)
         for (int i = tid; i < s.nseq; i += SCHED_THREADS)
             if (s.slots[i] < 0 || s.slots[i] >= s.n_slots) bad = 1;
+    if (s.decay)
+        for (int h = tid; h < s.H; h += SCHED_THREADS) {
+            const float lam = s.decay[h];
+            if (!(lam > 0.f && lam <= 1.f)) bad = 1;  // also rejects NaN
+        }
     bad = __syncthreads_or(bad);
     if (bad) {
         if (tid == 0) {

@@ -260,6 +260,20 @@ __device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint6
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// mma_ss_w with an output-lane mask: the lanes whose bit is set in the
+// disable-output-lane vector {m0, m1, m2, m3} (bit i of m_w: TMEM lane 32 w + i)
+// keep their contents; the others receive A x B (+ D).
+__device__ __forceinline__ void mma_ss_w_lanes(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                               uint32_t accumulate, uint32_t m0, uint32_t m1, uint32_t m2,
+                                               uint32_t m3) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(m0), "r"(m1), "r"(m2), "r"(m3)
+        : "memory");
+}
 __device__ __forceinline__ void tc_commit_w(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"

@@ -66,8 +66,8 @@ def _prefill(L, B=1, N=128, H=1, d=128, block=0, q=FAKE, out=FAKE, state_in=None
 
 def test_prefill_argument_errors(L):
     assert _prefill(L, d=64) == la.LA_ERR_UNSUPPORTED
-    assert _prefill(L, block=64) == la.LA_ERR_UNSUPPORTED
-    assert _prefill(L, block=256) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(L, block=96) == la.LA_ERR_UNSUPPORTED
+    assert _prefill(L, block=512) == la.LA_ERR_UNSUPPORTED
     assert _prefill(L, block=-1) == la.LA_ERR_INVALID_ARGUMENT
     assert _prefill(L, H=0) == la.LA_ERR_INVALID_ARGUMENT
     assert _prefill(L, B=-1) == la.LA_ERR_INVALID_ARGUMENT
@@ -103,6 +103,31 @@ def test_varlen_and_decode_argument_errors(L):
     assert L.la_decode_step(V(FAKE), V(FAKE), V(FAKE), V(1 << 40), V((1 << 40) + 256), 0, 1, 1, 128,
                             None) == la.LA_ERR_INVALID_ARGUMENT
     assert L.la_decode_step(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 0, 1, 128, None) == la.LA_OK
+
+
+def test_decay_argument_errors(L):
+    """The decay entry points check their arguments like the undecayed ones,
+    and a missing or misaligned decay array is an argument error."""
+    far = 1 << 40
+
+    def pd(decay=FAKE, block=0, d=128, out=far):
+        return L.la_prefill_decay(V(FAKE), V(FAKE), V(FAKE), 1, 128, 1, d, block, V(decay) if decay else None,
+                                  None, V(out), 0, None, V(2 * far), 1 << 30, None)
+    assert pd(decay=0) == la.LA_ERR_INVALID_ARGUMENT
+    assert pd(decay=FAKE + 2) == la.LA_ERR_INVALID_ARGUMENT
+    assert pd(d=64) == la.LA_ERR_UNSUPPORTED
+    assert pd(block=64) == la.LA_ERR_UNSUPPORTED                      # decay: block 128 only
+    assert pd(out=FAKE) == la.LA_ERR_INVALID_ARGUMENT                 # out overlaps q
+    assert L.la_prefill_varlen_decay(V(FAKE), V(FAKE), V(FAKE), V(FAKE), 1, 10, 10, 1, 128, 0, None, None,
+                                     V(far), 0, None, V(2 * far), 1 << 30, None) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_prefill_varlen_decay(V(FAKE), V(FAKE), V(FAKE), None, 1, 10, 10, 1, 128, 0, V(FAKE), None,
+                                     V(far), 0, None, V(2 * far), 1 << 30, None) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_decode_step_decay(V(FAKE), V(FAKE), V(FAKE), None, V(FAKE), V(FAKE), 0, 1, 1, 128, None) == \
+        la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_decode_step_decay(V(FAKE), V(FAKE), V(FAKE), V(FAKE + 1), V(FAKE), V(far), 0, 1, 1, 128,
+                                  None) == la.LA_ERR_INVALID_ARGUMENT
+    assert L.la_decode_step_decay(V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), V(FAKE), 0, 0, 1, 128,
+                                  None) == la.LA_OK
 
 
 def test_workspace_sizes(L):

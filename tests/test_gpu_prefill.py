@@ -38,11 +38,12 @@ def _oracle_prefill(oracle_mod, q, k, v, cu, state_in=None, heads=None, form="re
 
 
 def test_config1_small_prefill_fp32(oracle_mod):
-    """B=1, H=2, N=1024, fp32 out; the oracle's blocked form at block 64 (the
-    block of this configuration) and its quadratic form both serve as reference."""
+    """B=1, H=2, N=1024, fp32 out, row blocks of 64 (the block of this
+    configuration); the oracle's blocked form at block 64 and its quadratic
+    form both serve as reference."""
     B, N, H = 1, 1024, 2
     q, k, v = la_inputs.qkv((B, N, H, D), seed=1, device="cuda")
-    out, st = la.prefill(q, k, v, out_dtype=torch.float32)
+    out, st = la.prefill(q, k, v, block=64, out_dtype=torch.float32)
     assert la.get_device_status() == la.LA_OK
     cu = np.array([0, N], np.int32)
     ref_b, st_b = _oracle_prefill(oracle_mod, q[0], k[0], v[0], cu, form="blocked", block=64)
@@ -247,3 +248,59 @@ def test_output_only_16_byte_aligned(oracle_mod, dtype):
     assert out2.data_ptr() == out.data_ptr()
     ref, _ = _oracle_prefill(oracle_mod, q[0], k[0], v[0], np.array([0, N], np.int32))
     check_out(to_np(out[0]), ref, bf16_out=dtype == torch.bfloat16, what="16-byte aligned out")
+
+
+# ------------------------------------------------------------------ row blocks of 64
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 127, 129, 300, 1000])
+@pytest.mark.parametrize("seg", [0, 128, 256])
+def test_block64_ragged_and_segmented(oracle_mod, N, seg):
+    """block = 64: two 64-row blocks per 128-row tile, each with its own state
+    snapshot; against the oracle's blocked form at 64 and its recurrent form."""
+    B, H = 2, 3
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=200 + N, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(17)
+    state_in = torch.randn((B, H, D, D), generator=gen, device="cuda") * 0.3
+    la.set_segment_len(seg)
+    out, st = la.prefill(q, k, v, block=64, state_in=state_in, out_dtype=torch.float32)
+    assert la.get_device_status() == la.LA_OK
+    cu = la_inputs.cu_seqlens_from_lengths([N] * B)
+    qf, kf, vf = (x.reshape(B * N, H, D) for x in (q, k, v))
+    ref, rst = _oracle_prefill(oracle_mod, qf, kf, vf, cu, state_in=state_in, form="blocked", block=64)
+    check_out(to_np(out.reshape(B * N, H, D)), ref, bf16_out=False, what=f"block64 N={N} seg={seg}")
+    check_state(to_np(st), rst, what=f"block64 N={N} seg={seg}")
+    ref2, _ = _oracle_prefill(oracle_mod, qf, kf, vf, cu, state_in=state_in)
+    check_out(to_np(out.reshape(B * N, H, D)), ref2, bf16_out=False, what=f"block64 vs recurrent N={N}")
+
+
+def test_block64_varlen_bf16(oracle_mod):
+    lens = [0, 1, 64, 65, 1000, 0, 2500, 191]
+    H = 4
+    T = sum(lens)
+    q, k, v = la_inputs.qkv((T, H, D), seed=210, device="cuda")
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    la.set_segment_len(256)
+    out, st = la.prefill_varlen(q, k, v, torch.from_numpy(cu).cuda(), max(lens), block=64,
+                                out_dtype=torch.bfloat16)
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = _oracle_prefill(oracle_mod, q, k, v, cu, form="blocked", block=64)
+    check_out(to_np(out), ref, bf16_out=True, what="block64 varlen")
+    check_state(to_np(st), rst, what="block64 varlen states")
+
+
+def test_block64_long_sequence_hi_lo(oracle_mod):
+    """131072 tokens at block 64: the state reaches the inter-block products as
+    bf16 hi + lo past 65536 tokens, two row halves per tile."""
+    B, N, H = 1, 131072, 2
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=211, device="cuda")
+    out, st = la.prefill(q, k, v, block=64, out_dtype=torch.float32)
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = _oracle_prefill(oracle_mod, q[0], k[0], v[0], np.array([0, N], np.int32))
+    check_out(to_np(out[0]), ref, bf16_out=False, what="block64 131072")
+    check_state(to_np(st[0]), rst[0], what="block64 131072 state")
+
+
+def test_block64_rejected_with_decay():
+    q, k, v = la_inputs.qkv((1, 128, 2, D), seed=212, device="cuda")
+    with pytest.raises(la.LAError) as e:
+        la.prefill(q, k, v, block=64, decay=torch.ones(2, device="cuda"))
+    assert e.value.status == la.LA_ERR_UNSUPPORTED
