@@ -55,7 +55,7 @@ def prefill_bytes(tok_heads: int, heads: int, seqs: int) -> int:
     return tok_heads * D * 2 * 4 + seqs * heads * D * D * 4
 
 
-LO_SPLIT_FROM = 65536  # segments ending past this token use S as bf16 hi + lo in Q S
+LO_SPLIT_FROM = 32768  # segments ending past this token use S as bf16 hi + lo in Q S
 
 
 def prefill_alg_flops(tok_heads: int, block: int) -> int:
@@ -71,19 +71,25 @@ def prefill_survey_exec_flops(tok_heads: int, block: int) -> int:
     return tok_heads * (4 * block * D + 4 * D * D)
 
 
-def prefill_mma_flops(lengths, heads: int, seg_len: int, want_state: bool = True) -> int:
+def prefill_mma_flops(lengths, heads: int, seg_len: int, want_state: bool = True, block: int = 128) -> int:
     """FLOPs the tensor pipe executes in la_prefill_kernel, counted MMA by MMA
     the way the kernel issues them (one unit = a 128 x 128 x 128 product,
-    2 * 128^3 FLOPs), per segment of seg_len tokens of every sequence:
-      Q K^T and P V: one unit each per 128-row block (full tiles, masked or not);
-      Q S: one unit per block, two when the segment ends past LO_SPLIT_FROM
-           tokens into its sequence (S handed over as bf16 hi + lo);
-      K^T V in the scan: one unit per block except the segment's last block,
-           which also gets one in the final segment when the state is wanted;
-      K^T V in the segment-sum pass: one unit per block of every segment that
-           has a successor in its sequence."""
+    2 * 128^3 FLOPs), per segment of seg_len tokens of every sequence, over its
+    128-row tiles:
+      block 128: per tile Q K^T and P V (full tiles, masked or not), Q S (two
+           units when the segment ends past LO_SPLIT_FROM tokens: S as bf16
+           hi + lo), K^T V except for the segment's last tile (which gets it in
+           the final segment when the state is wanted);
+      block 64: per tile Q K^T, P V, Q S twice (once per 64-row block, each a
+           full product writing half the rows; doubled again for hi + lo), K^T V
+           of the first 64 rows always and of the last 64 rows as above;
+      block 256: per pair of tiles Q K^T and P V three times (two diagonal
+           tiles and the second tile against the first), Q S once per tile,
+           K^T V for both tiles unless the pair is the segment's last (as above);
+      and K^T V again in the segment-sum pass, one unit per tile of every
+      segment that has a successor in its sequence."""
     unit = 2 * 128 ** 3
-    units = 0
+    units = 0.0
     for n in lengths:
         n = int(n)
         nseg = -(-n // seg_len) if n > 0 else 0
@@ -91,11 +97,26 @@ def prefill_mma_flops(lengths, heads: int, seg_len: int, want_state: bool = True
             t0, t1 = j * seg_len, min(n, (j + 1) * seg_len)
             nblk = -(-(t1 - t0) // 128)
             last = j == nseg - 1
-            units += 2 * nblk                                   # Q K^T, P V
-            units += nblk * (2 if t1 > LO_SPLIT_FROM else 1)    # Q S (hi [+ lo])
-            units += nblk - 1 + (1 if (last and want_state) else 0)  # K^T V, scan
-            units += 0 if last else nblk                        # K^T V, segment sums
-    return units * unit * heads
+            qs = 2 if t1 > LO_SPLIT_FROM else 1          # Q S, bf16 S or hi + lo
+            if block == 256:
+                npair = (nblk + 1) // 2
+                for m in range(npair):
+                    ntp = 2 if 2 * m + 1 < nblk else 1
+                    upd = m < npair - 1 or (last and want_state)
+                    units += 2 * (ntp + (ntp == 2))         # Q K^T, P V (3 steps per full pair)
+                    units += ntp * qs                       # Q S
+                    units += ntp if upd else 0              # K^T V
+            else:
+                fin = 1 if (last and want_state) else 0
+                units += 2 * nblk                           # Q K^T, P V
+                if block == 64:
+                    units += 2 * nblk * qs                  # Q S once per 64-row block
+                    units += 0.5 * nblk + 0.5 * (nblk - 1 + fin)  # K^T V in two halves
+                else:
+                    units += nblk * qs
+                    units += nblk - 1 + fin
+            units += 0 if last else nblk                    # K^T V, segment sums
+    return int(units * unit * heads)
 
 
 def aggregate_bytes(tok_heads: int, pairs: int) -> int:
@@ -421,7 +442,7 @@ def run_cuda(args, world, rank, local):
     byts = prefill_bytes(tok_heads, H, B)
     L = la.last_segment_len()
     f_alg = prefill_alg_flops(tok_heads, BLOCK)
-    f_mma = prefill_mma_flops([N] * B, H, L, want_state=True)
+    f_mma = prefill_mma_flops([N] * B, H, L, want_state=True, block=BLOCK)
     f_dense = prefill_survey_exec_flops(tok_heads, BLOCK)
     achieved_gbs = byts / (ms * 1e-3) / 1e9
 
@@ -454,6 +475,12 @@ def run_cuda(args, world, rank, local):
     if rank == 0 or world > 1:
         dec = bench_decode(la, dev, stream, args, hbm_peak, world)
 
+    # ---------------- the same workload at row blocks of 64 and 256
+    by_block = {f"block{blk}": bench_prefill_block(la, dev, stream, q, k, v, blk, args, hbm_peak, tc_peak, world)
+                for blk in (64, 256)}
+    # ---------------- the same workload with a per-head decay
+    dec_pref = bench_prefill_decay(la, dev, stream, q, k, v, args, hbm_peak, world)
+
     # ---------------- the packed varlen batch and the 1M-token prefill
     varlen = bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank)
     longc = bench_long_context(la, dev, stream, args, hbm_peak, tc_peak, world, rank)
@@ -483,7 +510,8 @@ def run_cuda(args, world, rank, local):
         "tensor_frac_alg": f_alg / (ms * 1e-3) / 1e12 / tc_peak,
         "tensor_frac_dense_count": f_dense / (ms * 1e-3) / 1e12 / tc_peak,
         "tensor_note": ("tflops_mma counts every tcgen05 MMA the kernel issues (full 128-row tiles, Q S once "
-                        "per block below 65536 tokens, K^T V in the scan and in the segment-sum pass); "
+                        "per block up to 32768 tokens into a sequence, twice beyond, K^T V in the scan and in the "
+                        "segment-sum pass); "
                         "tflops_alg the blocked definition 2(Bk+1)d + 4d^2 per token-head; dense_count "
                         "4 Bk d + 4 d^2; fractions of the measured cuBLAS bf16 burst peak"),
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
@@ -497,6 +525,8 @@ def run_cuda(args, world, rank, local):
                 "d2h_bytes_per_step": out.numel() * out.element_size() + st.numel() * st.element_size()},
         "gpu_launches": int(launches),
         "clocks": clocks,
+        "prefill_by_block": by_block,
+        "prefill_decay": dec_pref,
         "decode": dec,
         "varlen": varlen,
         "long_context": longc,
@@ -624,6 +654,83 @@ def bench_decode(la, dev, stream, args, hbm_peak, world):
             "tok_s": DEC_SEQS * world / (ms * 1e-3), "ms_per_step": ms, "steps": steps, "roofline": roof}
 
 
+def bench_prefill_block(la, dev, stream, q, k, v, block, args, hbm_peak, tc_peak, world):
+    """The bench workload (B=1, H=64, N=32768, bf16 out + states) at another
+    row-block length: 64 (two state snapshots per 128-row tile) or 256 (a
+    snapshot per pair of tiles, plus the second tile's queries against the
+    first tile's keys)."""
+    out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=dev)
+    st = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(la.workspace_size(B, N, H, D, block), dtype=torch.uint8, device=dev)
+
+    def call():
+        la.prefill(q, k, v, block=block, out=out, state_out=st, workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(5, min(args.steps, 100))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    L = la.last_segment_len()
+    byts = prefill_bytes(B * N * H, H, B)
+    gbs = byts / (ms * 1e-3) / 1e9
+    f_mma = prefill_mma_flops([N] * B, H, L, want_state=True, block=block)
+    f_alg = prefill_alg_flops(B * N * H, block)
+    f_dense = prefill_survey_exec_flops(B * N * H, block)
+    del out, st, ws
+    return {"workload": f"causal prefill B=1 H=64 N=32768 d=128 at row blocks of {block}",
+            "ms_per_call": ms, "steps": steps, "segment_len": L,
+            "tflops_mma": f_mma / (ms * 1e-3) / 1e12, "tensor_frac_mma": f_mma / (ms * 1e-3) / 1e12 / tc_peak,
+            "tflops_alg": f_alg / (ms * 1e-3) / 1e12, "tensor_frac_alg": f_alg / (ms * 1e-3) / 1e12 / tc_peak,
+            "tensor_frac_dense_count": f_dense / (ms * 1e-3) / 1e12 / tc_peak,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "kernel": "la_prefill_kernel", "bytes_per_launch": byts,
+                         "traffic": recorded_traffic("la_prefill_kernel", f"prefill_B1_H64_N32768_block{block}"),
+                         "duration": "CUDA events around each la_prefill call (scheduler + prefill)"}}
+
+
+def bench_prefill_decay(la, dev, stream, q, k, v, args, hbm_peak, world):
+    """The bench workload with the per-head decay lambda_h = exp(-2^(-8 (h+1)/H))
+    (la_prefill_decay: decay in the mask, the inter-block term and the state,
+    the decayed keys of the state update as bf16 hi + lo)."""
+    lam = torch.tensor(np.exp(-(2.0 ** (-8.0 * (np.arange(H) + 1) / H))), dtype=torch.float32, device=dev)
+    out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=dev)
+    st = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(la.workspace_size(B, N, H, D, BLOCK), dtype=torch.uint8, device=dev)
+
+    def call():
+        la.prefill(q, k, v, block=BLOCK, out=out, state_out=st, workspace=ws, decay=lam)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(5, min(args.steps, 100))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    byts = prefill_bytes(B * N * H, H, B)
+    gbs = byts / (ms * 1e-3) / 1e9
+    del out, st, ws
+    return {"workload": "causal prefill B=1 H=64 N=32768 d=128 with per-head decay exp(-2^(-8(h+1)/64))",
+            "ms_per_call": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "kernel": "la_prefill_kernel (decay)", "bytes_per_launch": byts,
+                         "traffic": None,
+                         "duration": "CUDA events around each la_prefill_decay call (scheduler + prefill)"}}
+
+
 def bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank):
     """Packed variable-length prefill: 8 sequences with lengths drawn uniform in
     [1024, 65536] from a seed, concatenated (cu_seqlens on the device), H=64,
@@ -672,7 +779,7 @@ def bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank):
 
 def bench_long_context(la, dev, stream, args, hbm_peak, tc_peak, world, rank):
     """Long-context prefill: B=1, H=8, N=1048576, bf16 out + fp32 final states
-    (8.6 GB of algorithmic traffic per call).  Segments past 65536 tokens hand
+    (8.6 GB of algorithmic traffic per call).  Segments past 32768 tokens hand
     S to the inter-block product as bf16 hi + lo."""
     NL, HL = 1048576, 8
     q, k, v = la_inputs.qkv((1, NL, HL, D), seed=404 + rank, device=dev)

@@ -80,9 +80,10 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Segment length of the cross-SM scan.  Depends on the problem only (not on
 // the device) so that the workspace size is a pure function of the shape.
-int choose_seg_len(int nseq, long long T, int H) {
+int choose_seg_len(int nseq, long long T, int H, int block = 0) {
+    // with 256-token row blocks a segment holds whole blocks
     const int ov = g_seg_len_override.load();
-    if (ov > 0) return ov;
+    if (ov > 0) return (block == 256 && ov % 256) ? ov + la::BLK : ov;
     // Longer segments for few heads: each (sequence, head) scan then has fewer
     // cross-SM hand-offs in its chain (measured at H = 8, N = 1M: 6.2 / 3.3 /
     // 2.5 / 2.5 / 2.7 ms for 1024 / 2048 / 4096 / 8192 / 16384 tokens).
@@ -94,7 +95,7 @@ int choose_seg_len(int nseq, long long T, int H) {
         L /= 2;
     }
     (void)nseq;
-    return L;
+    return (block == 256 && L % 256) ? L + la::BLK : L;
 }
 
 struct WsLayout {
@@ -146,7 +147,8 @@ la_status ensure_smem_attr(SmemAttr &a, Kernel *kernel, int bytes) {
     return LA_OK;
 }
 
-SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_prefill_decay, g_attr_prefill_b64, g_attr_agg;
+SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_prefill_decay, g_attr_prefill_b64, g_attr_prefill_b256,
+    g_attr_agg;
 
 bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
     if (!a || !b || na == 0 || nb == 0) return false;
@@ -158,7 +160,7 @@ la_status check_common(int H, int d, int block, la_dtype out_dtype) {
     if (H <= 0 || d <= 0 || block < 0) return LA_ERR_INVALID_ARGUMENT;
     if (out_dtype != LA_BF16 && out_dtype != LA_FP32) return LA_ERR_INVALID_ARGUMENT;
     if (d != la::D) return LA_ERR_UNSUPPORTED;
-    if (block != 0 && block != 64 && block != la::BLK) return LA_ERR_UNSUPPORTED;
+    if (block != 0 && block != 64 && block != la::BLK && block != 256) return LA_ERR_UNSUPPORTED;
     return LA_OK;
 }
 
@@ -188,7 +190,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     if (slots && (n_slots <= 0 || !aligned(slots, 4) || state_in != state_out || !state_out))
         return LA_ERR_INVALID_ARGUMENT;
     if (decay && (anti || !aligned(decay, 4))) return LA_ERR_INVALID_ARGUMENT;
-    if (block == 64 && (anti || decay)) return LA_ERR_UNSUPPORTED;
+    if ((block == 64 || block == 256) && (anti || decay)) return LA_ERR_UNSUPPORTED;
     const size_t n_state = (size_t)(slots ? n_slots : nseq) * H * la::D * la::D * 4;
     if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
@@ -200,7 +202,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     if (ranges_overlap(out, n_out, state_out, n_state) || ranges_overlap(out, n_out, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
 
-    const int L = choose_seg_len(nseq, T, H);
+    const int L = choose_seg_len(nseq, T, H, block);
     if (L <= 0 || L % la::BLK) return LA_ERR_INVALID_ARGUMENT;
     const long long gmax = cu ? gmax_for(nseq, T, L) : gmax_fixed(nseq, fixed_len, L);
     const WsLayout w = ws_layout(gmax, H);
@@ -287,6 +289,7 @@ la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUten
     if (ANTI) return launch_prefill_bk<true, false, 128>(g_attr_prefill_anti, grid, mq, mk, mv, pp, stream);
     if (DECAY) return launch_prefill_bk<false, true, 128>(g_attr_prefill_decay, grid, mq, mk, mv, pp, stream);
     if (block == 64) return launch_prefill_bk<false, false, 64>(g_attr_prefill_b64, grid, mq, mk, mv, pp, stream);
+    if (block == 256) return launch_prefill_bk<false, false, 256>(g_attr_prefill_b256, grid, mq, mk, mv, pp, stream);
     return launch_prefill_bk<false, false, 128>(g_attr_prefill, grid, mq, mk, mv, pp, stream);
 }
 
@@ -381,20 +384,18 @@ extern "C" {
 
 size_t la_prefill_workspace_size(int B, int N, int H, int d, int block) {
     (void)d;
-    (void)block;
     if (B <= 0 || N < 0 || H <= 0) return la::HDR_BYTES;
     const long long T = (long long)B * N;
-    const int L = choose_seg_len(B, T, H);
+    const int L = choose_seg_len(B, T, H, block);
     return ws_layout(gmax_fixed(B, N, L), H).total;
 }
 
 size_t la_prefill_varlen_workspace_size(int nseq, int total_tokens, int max_seqlen, int H, int d,
                                         int block) {
     (void)d;
-    (void)block;
     (void)max_seqlen;
     if (nseq <= 0 || total_tokens < 0 || H <= 0) return la::HDR_BYTES;
-    const int L = choose_seg_len(nseq, total_tokens, H);
+    const int L = choose_seg_len(nseq, total_tokens, H, block);
     return ws_layout(gmax_for(nseq, total_tokens, L), H).total;
 }
 
@@ -529,7 +530,7 @@ const char *la_status_string(la_status s) {
     switch (s) {
         case LA_OK: return "ok";
         case LA_ERR_INVALID_ARGUMENT: return "invalid argument";
-        case LA_ERR_UNSUPPORTED: return "unsupported (d = 128 only; row blocks 0/64/128, 64 without decay)";
+        case LA_ERR_UNSUPPORTED: return "unsupported (d = 128 only; row blocks 0/64/128/256, decay at 128 only)";
         case LA_ERR_CUDA: return "CUDA error";
         case LA_ERR_TIMEOUT: return "a bounded device-side wait ran out";
         case LA_ERR_WORKSPACE: return "workspace missing or too small";
@@ -799,7 +800,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
 
     // longest useful segment: one per sequence
     const int max_len = (int)(((long long)(N > 0 ? N : 1) + la::BLK - 1) / la::BLK * la::BLK);
-    int L = choose_seg_len(B, T, H);
+    int L = choose_seg_len(B, T, H, block);
     while (ws_layout(gmax_fixed(B, N, L), H).total > LA_NOALLOC_SCRATCH_BYTES && L < max_len)
         L = (2 * L < max_len) ? 2 * L : max_len;
     const long long gmax = gmax_fixed(B, N, L);

@@ -188,13 +188,15 @@ constexpr int ITF_LO = 2;    // inter-block product uses S = S_hi + S_lo
 
 // Precision of the inter-block product Q_b S_{<b}.  S is rounded to bf16 for
 // the tensor cores (relative error 2^-9).  S grows like sqrt(position) for the
-// unit-scaled inputs this operation sees, so up to LA_LO_SPLIT_FROM tokens into
-// a sequence a single bf16 term keeps the output error far inside the error
-// budget (max abs ~1e-2 at 64K tokens).  Segments that reach past it use
-// S = S_hi + S_lo, two bf16 terms with ~2^-16 relative error, at twice the
-// tensor-core and shared-memory cost of that product.
+// unit-scaled inputs this operation sees, and so does the error of that
+// rounding: measured on the fp32 output, max abs 1.27e-2 over the first 32768
+// tokens and 2.02e-2 (past the 2e-2 bound) near 64K tokens of one sequence.
+// Up to LA_LO_SPLIT_FROM tokens into a sequence a single bf16 term is used;
+// segments that reach past it use S = S_hi + S_lo, two bf16 terms with
+// ~2^-16 relative error, at twice the tensor-core and shared-memory cost of
+// that product.
 #ifndef LA_LO_SPLIT_FROM
-#define LA_LO_SPLIT_FROM 65536
+#define LA_LO_SPLIT_FROM 32768
 #endif
 
 __device__ __forceinline__ void record_status(int *status, int code) {
@@ -416,9 +418,10 @@ template <bool ANTI, bool DECAY, int BK>
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
-    static_assert(BK == 64 || BK == 128, "row blocks of 64 or 128 tokens");
-    static_assert(BK == 128 || (!ANTI && !DECAY), "64-row blocks: the plain forward only");
+    static_assert(BK == 64 || BK == 128 || BK == 256, "row blocks of 64, 128 or 256 tokens");
+    static_assert(BK == 128 || (!ANTI && !DECAY), "64- and 256-row blocks: the plain forward only");
     constexpr bool B64 = BK == 64;  // two 64-row blocks per 128-row tile
+    // BK == 256: one row block per pair of 128-row tiles (see the MMA warp)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
@@ -595,7 +598,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         // The whole warp runs this loop in step: every lane holds the same
         // counters, barrier probes are combined with __all_sync, and each MMA or
         // commit is issued by the lane that elect.sync picks.
-        uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0, afree_n = 0, a_n = 0;
+        uint32_t it = 0, kv_n = 0, q_n = 0, blk_n = 0, snap_n = 0, afree_n = 0, a_n = 0, stp_n = 0;
         bool ok = true;
         int item[8];
         auto ready = [&](uint64_t *bar, uint32_t parity) -> bool {
@@ -650,6 +653,163 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             int i2 = 0, i4 = 0, i5 = 0, sub = 0;  // next block of a2 / a4 / a5; a5 sub-step pending
             uint32_t spins = 0;
             uint64_t deadline = 0;
+            if constexpr (BK == 256) {
+                // Row blocks of 256 tokens = pairs of 128-row tiles (2m, 2m+1)
+                // sharing one state snapshot.  Score steps, in order: (2m, 2m),
+                // (2m+1, 2m+1) with the causal mask, and (2m+1, 2m) unmasked -- the
+                // second tile's queries against the first tile's keys, inside the
+                // block -- each a2 -> [mask] -> a4 through the one score buffer.
+                // a5 of both tiles reads the pair's snapshot S_{<block}; a6 adds
+                // K^T V of both tiles once per pair.  A pair keeps both K/V stages
+                // until its last score step.
+                const int npair = (nblk + 1) / 2, nsteps = 3 * (nblk / 2) + (nblk & 1);
+                const int nch = lo ? 2 : 1;
+                int u2 = 0, u4 = 0, a6n = 0;  // next score step of a2 / a4; pairs whose a6 is issued
+                while (u4 < nsteps) {
+                    bool prog = false;
+                    // a4(u4): P of the step ready, a5 of its query tile issued
+                    if (u4 < u2) {
+                        const int m = u4 / 3, w = u4 % 3, ti = 2 * m + (w > 0), tj = 2 * m + (w == 1);
+                        const bool pair_last = w == 2 || 2 * m + 1 >= nblk;
+                        // (the pair's last step releases its stages: its a6 must be issued)
+                        if (ti < i5 && (!pair_last || a6n > m) && ready(&cb->p_full, (stp_n + u4) & 1)) {
+                            tc_fence_after();
+                            const uint32_t vt = sbase + SM_V + ((kv0 + tj) % KV_STAGES) * TILE_BYTES;
+                            const uint32_t bn = blk0 + ti;
+#pragma unroll
+                            for (int kk = 0; kk < BLK / 16; ++kk)
+                                mma_ts_w(tmem + TM_O + (bn & 1) * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV, 1u);
+                            const bool pair_full = 2 * m + 1 < nblk;
+                            if (w != 1) tc_commit_w(&cb->o_full[bn & 1]);  // tile 2m (step 0) or 2m+1 (step 2) done
+                            if (w == 2 || !pair_full) {  // the pair's last step: both stages are free
+                                tc_commit_w(&cb->kv_empty[(kv0 + 2 * m) % KV_STAGES]);
+                                if (pair_full) tc_commit_w(&cb->kv_empty[(kv0 + 2 * m + 1) % KV_STAGES]);
+                            }
+                            ++u4;
+                            prog = true;
+                        }
+                    }
+                    // a5 sub-step: one column half (hi + lo) of one tile of the pair
+                    if (i5 < nblk) {
+                        const int m = i5 / 2, ntp = (2 * m + 1 < nblk) ? 2 : 1;
+                        const int tp = sub % ntp, ch = sub / ntp, ti = 2 * m + tp;
+                        const uint32_t bn = blk0 + ti;
+                        const uint32_t qn = q0 + ti;
+                        const bool a_read = last || ti > 0 || ready(&cb->a_free, afree_n & 1);
+                        // the tile's Q landed (checked directly: with hi + lo halves the
+                        // second tile reads the first half of the snapshot before the
+                        // first tile's a5 -- and so the second tile's a2 -- can complete)
+                        if (a_read && ready(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1) &&
+                            ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty[bn & 1], ((bn >> 1) & 1) ^ 1)) {
+                            tc_fence_after();
+                            const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
+                            const uint32_t sh = sbase + SM_SHI, sl = sbase + SM_SLO;
+                            const uint32_t tq = tmem + TM_O + (bn & 1) * 128;
+                            if (!lo) {
+#pragma unroll
+                                for (int kk = 0; kk < D / 16; ++kk)
+                                    mma_ss_w(tq, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QF, kk > 0 ? 1u : 0u);
+                            } else {
+                                const uint32_t to = tq + ch * 64;
+#pragma unroll
+                                for (int kk = 0; kk < D / 16; ++kk)
+                                    mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sh, kk), ID_QS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                                for (int kk = 0; kk < D / 16; ++kk)
+                                    mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
+                            }
+                            if (tp == ntp - 1) {  // every tile of the pair has read this snapshot
+                                tc_commit_w(&cb->snap_empty);
+                                ++snap_n;
+                            }
+                            if (ch == nch - 1) {  // the tile's a5 is complete
+                                if (!last && ti == 0) ++afree_n;
+                                // a first tile's Q is free once its a2 is issued too
+                                if ((ti & 1) == 0 && u2 > 3 * (ti / 2)) tc_commit_w(&cb->q_empty[qn % Q_STAGES]);
+                                ++i5;
+                            }
+                            sub = (tp == ntp - 1 && ch == nch - 1) ? 0 : sub + 1;
+                            prog = true;
+                        }
+                    }
+                    // a6 of pair a6n: S += K^T V over both tiles, once the pair's a5 is
+                    // complete (S has been read out) and its last tile's diagonal a2 is
+                    // issued (rows past the sequence end are zeroed by then)
+                    if (a6n < npair) {
+                        const int m = a6n, ntp = (2 * m + 1 < nblk) ? 2 : 1;
+                        if (i5 >= 2 * m + ntp && u2 > 3 * m + ntp - 1) {
+                            if ((m < npair - 1) || want_final) {
+                                for (int t2 = 0; t2 < ntp; ++t2) {
+                                    const int s2 = (kv0 + 2 * m + t2) % KV_STAGES;
+                                    const uint32_t kt = sbase + SM_K + s2 * TILE_BYTES;
+                                    const uint32_t vt = sbase + SM_V + s2 * TILE_BYTES;
+#pragma unroll
+                                    for (int kk = 0; kk < BLK / 16; ++kk)
+                                        mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
+                                }
+                                tc_commit_w(&cb->s_done);
+                            }
+                            ++a6n;
+                            prog = true;
+                        }
+                    }
+                    // a2(u2): the score buffer free (a4 of the previous step issued),
+                    // query tile and key tile landed
+                    if (u2 < nsteps && u2 <= u4) {
+                        const int m = u2 / 3, w = u2 % 3, ti = 2 * m + (w > 0), tj = 2 * m + (w == 1);
+                        const int sj = (kv0 + tj) % KV_STAGES;
+                        const uint32_t kn = (kv0 + tj) / KV_STAGES, qn = q0 + ti;
+                        if (ready(&cb->kv_full[sj], kn & 1) && ready(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1)) {
+                            if (w < 2) {  // a tile's first use: rows past the sequence end add nothing
+                                const int valid = min(BLK, tok1 - (tok0 + tj * BLK));
+                                if (valid < BLK) {
+                                    uint8_t *kp = smem + SM_K + sj * TILE_BYTES;
+                                    uint8_t *vp = smem + SM_V + sj * TILE_BYTES;
+                                    const int nbytes = (BLK - valid) * 128;
+                                    for (int hh = 0; hh < 2; ++hh)
+                                        for (int o = lane * 16; o < nbytes; o += 32 * 16) {
+                                            *reinterpret_cast<uint4 *>(kp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                                            *reinterpret_cast<uint4 *>(vp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                                        }
+                                    fence_proxy_async_smem();
+                                    __syncwarp();
+                                }
+                            }
+                            tc_fence_after();
+                            const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
+                            const uint32_t kt = sbase + SM_K + sj * TILE_BYTES;
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_ss_w(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK, kk > 0 ? 1u : 0u);
+                            tc_commit_w(&cb->sc_full);
+                            if (w == 2) tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // Q of tile 2m+1: last reader
+                            if (w == 0 && i5 > ti) tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // tile 2m: a5 came first
+                            ++u2;
+                            prog = true;
+                        }
+                    }
+                    if (prog) {
+                        spins = 0;
+                        deadline = 0;
+                    } else if (((++spins) & 255u) == 0u) {
+                        int stop = 0;
+                        if (lane == 0) {
+                            const uint64_t now = globaltimer_ns();
+                            if (deadline == 0) deadline = now + p.wait_limit_ns;
+                            if (now > deadline || cb->abort) {
+                                cb->abort = 1;
+                                record_status(p.status, ST_TIMEOUT);
+                                stop = 1;
+                            }
+                        }
+                        if (__shfl_sync(0xffffffffu, stop, 0)) {
+                            ok = false;
+                            break;
+                        }
+                    }
+                }
+                stp_n += nsteps;
+            } else
             while (i4 < nblk) {
                 bool prog = false;
                 // O chain, a4(i4): P ready, a5 of the block issued
@@ -869,17 +1029,22 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 if (!ok) break;
             }
             const bool want_final = last && p.state_out != nullptr;
-            for (int b = 0; b < nblk; ++b) {
+            // score steps: one per tile, or, with 256-row blocks, three per pair of
+            // tiles (the third, the second tile's queries against the first tile's
+            // keys, is not masked)
+            const int nsteps = BK == 256 ? 3 * (nblk / 2) + (nblk & 1) : nblk;
+            for (int b = 0; b < nsteps; ++b) {
                 // P = bf16(Sc ⊙ M), inclusive mask (exclusive under ANTI), packed
                 // two per 32-bit column over the first 64 score columns
                 // (DECAY: P = bf16(Sc lambda^{r-c}) for c <= r)
                 const uint32_t bn = blk_n + b, tsc = trow + TM_SC;
+                const bool full = BK == 256 && b % 3 == 2;  // every key precedes every query
                 if (!warp_wait(&cb->sc_full, bn & 1, p, cb)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t x[64];
-                    if ((hf == 1 && q4 < 2) || (B64 && hf == 0 && q4 >= 2)) {
+                    if (!full && ((hf == 1 && q4 < 2) || (B64 && hf == 0 && q4 >= 2))) {
                         // rows 0-63 see none of the keys 64-127; with 64-row blocks,
                         // rows 64-127 (the second block) see none of the keys 0-63
 #pragma unroll
@@ -902,7 +1067,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                         for (int w = 0; w < 32; ++w) {
                             const int c = hf * 64 + 2 * w;
-                            x[w] = bf16x2_round(c + EXCL <= r ? x[2 * w] : 0u, c + 1 + EXCL <= r ? x[2 * w + 1] : 0u);
+                            x[w] = bf16x2_round(full || c + EXCL <= r ? x[2 * w] : 0u,
+                                                full || c + 1 + EXCL <= r ? x[2 * w + 1] : 0u);
                         }
                     }
                     tmem_st32(tsc + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -924,7 +1090,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&cb->p_full);
             }
-            blk_n += nblk;
+            blk_n += nsteps;
             kv_n += nblk;
             q_n += nblk;
         }
@@ -1103,15 +1269,20 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 ok = __all_sync(0xffffffffu, ok) != 0;
                 src_incl = p.incl + (size_t)pred * D * D;
             }
-            if (!last) {
+            // E_j -> S (TMEM); INCL_j = E_j + A_j -> workspace straight from registers;
+            // E_j as bf16 -> the snapshot buffer for a5 of the first block (one
+            // bf16 term: written here; hi + lo: through snapshot_state below).
+            // With one bf16 term (and no decay) the prefix and its snapshot go out
+            // while phase A still runs, and INCL_j is formed afterwards from S and
+            // A_j in TMEM, so that only the sum remains between the end of phase A
+            // and the first block's a5.
+            const bool snap_here = !lo;
+            const bool early = snap_here && !DECAY;
+            if (!last && !early) {
                 if (!warp_wait(&cb->agg_full, agg_n & 1, p, cb)) ok = false;
                 ++agg_n;
                 tc_fence_after();
             }
-            // E_j -> S (TMEM); INCL_j = E_j + A_j -> workspace straight from registers;
-            // E_j as bf16 -> the snapshot buffer for a5 of the first block (one
-            // bf16 term: written here; hi + lo: through snapshot_state below)
-            const bool snap_here = !lo;
             if (snap_here && !warp_wait(&cb->snap_empty, (snap_n & 1) ^ 1, p, cb)) ok = false;
             float *dst_incl = p.incl + (size_t)t * D * D;
 #pragma unroll 1
@@ -1145,7 +1316,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                             make_uint4(bf16x2_round(e[8 * q], e[8 * q + 1]), bf16x2_round(e[8 * q + 2], e[8 * q + 3]),
                                        bf16x2_round(e[8 * q + 4], e[8 * q + 5]), bf16x2_round(e[8 * q + 6], e[8 * q + 7]));
                 }
-                if (!last) {
+                if (!last && !early) {
                     // A_j: the first block's O buffer (DECAY: O buffer 1);
                     // DECAY: INCL_j = lambda^{len} E_j + A_j
                     const uint32_t ta = DECAY ? TM_O + 128 : TM_O + (blk_n & 1) * 128;
@@ -1181,7 +1352,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                 }
             }
-            if (!last) {  // A_j has been read: its O buffer is free for a5 of the first block
+            if (!last && !early) {  // A_j has been read: its O buffer is free for a5 of the first block
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -1200,23 +1371,55 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             } else if (!snapshot_state<DECAY>(trow, shi, slo, r, lane, lo, snap_n, p, cb, DECAY ? block_decay(0) : 1.f)) {
                 ok = false;
             }
+            if (!last && early) {
+                // INCL_j = E_j + A_j from TMEM once phase A is done (a5 of the first
+                // block, which overwrites A_j, waits for a_free; a6, which changes S,
+                // follows that a5)
+                if (!warp_wait(&cb->agg_full, agg_n & 1, p, cb)) ok = false;
+                ++agg_n;
+                tc_fence_after();
+                const uint32_t ta = TM_O + (blk_n & 1) * 128;
+#pragma unroll 1
+                for (int qq = 0; qq < 4 && ok; ++qq) {
+                    uint32_t e[32], a[32];
+                    tmem_ld32(trow + TM_S + qq * 32, e);
+                    tmem_ld32(trow + ta + qq * 32, a);
+                    tmem_wait_ld();
+                    reg_fence(e);
+                    reg_fence(a);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        __stcg(reinterpret_cast<float4 *>(dst_incl + incl_off(r, qq * 8 + c)),
+                               make_float4(__uint_as_float(e[4 * c]) + __uint_as_float(a[4 * c]),
+                                           __uint_as_float(e[4 * c + 1]) + __uint_as_float(a[4 * c + 1]),
+                                           __uint_as_float(e[4 * c + 2]) + __uint_as_float(a[4 * c + 2]),
+                                           __uint_as_float(e[4 * c + 3]) + __uint_as_float(a[4 * c + 3])));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&cb->a_free);
+                    mbar_arrive(&cb->incl_stored);
+                }
+            }
             if (!__all_sync(0xffffffffu, ok && !cb->abort)) break;
 
             // ------------- phase O: state snapshots and the final state -------------
             const bool want_final = last && p.state_out != nullptr;
-            for (int b = 0; b < nblk; ++b) {
+            const int nupd = BK == 256 ? (nblk + 1) / 2 : nblk;  // state updates: one per row block
+            for (int b = 0; b < nupd; ++b) {
                 if (B64) {  // S_{<b1} after the update over the tile's first 64 rows
                     if (!warp_wait(&cb->s_done, upd_n & 1, p, cb)) { ok = false; break; }
                     ++upd_n;
                     tc_fence_after();
                     if (!snapshot_state<DECAY>(trow, shi, slo, r, lane, lo, snap_n, p, cb)) { ok = false; break; }
                 }
-                const bool update = (b < nblk - 1) || want_final;
+                const bool update = (b < nupd - 1) || want_final;
                 if (!update) continue;
                 if (!warp_wait(&cb->s_done, upd_n & 1, p, cb)) { ok = false; break; }
                 ++upd_n;
                 tc_fence_after();
-                if (b < nblk - 1) {
+                if (b < nupd - 1) {
                     if (!snapshot_state<DECAY>(trow, shi, slo, r, lane, lo, snap_n, p, cb,
                                                DECAY ? block_decay(b + 1) : 1.f)) {  // S_{<b+1}
                         ok = false;

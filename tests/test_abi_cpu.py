@@ -117,6 +117,7 @@ def test_decay_argument_errors(L):
     assert pd(decay=FAKE + 2) == la.LA_ERR_INVALID_ARGUMENT
     assert pd(d=64) == la.LA_ERR_UNSUPPORTED
     assert pd(block=64) == la.LA_ERR_UNSUPPORTED                      # decay: block 128 only
+    assert pd(block=256) == la.LA_ERR_UNSUPPORTED
     assert pd(out=FAKE) == la.LA_ERR_INVALID_ARGUMENT                 # out overlaps q
     assert L.la_prefill_varlen_decay(V(FAKE), V(FAKE), V(FAKE), V(FAKE), 1, 10, 10, 1, 128, 0, None, None,
                                      V(far), 0, None, V(2 * far), 1 << 30, None) == la.LA_ERR_INVALID_ARGUMENT

@@ -97,7 +97,7 @@ def test_decay_varlen_packed_with_empty(oracle_mod):
 
 
 def test_decay_long_sequence_hi_lo_path(oracle_mod):
-    """131072 tokens: segments past 65536 hand S to the inter-block product as
+    """131072 tokens: segments past 32768 hand S to the inter-block product as
     bf16 hi + lo; heads with lambda = 1 and lambda close to 1 keep S growing."""
     B, N, H = 1, 131072, 4
     lam = [1.0, 1.0 - 1e-5, 0.9995, 0.6]

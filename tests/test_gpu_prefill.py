@@ -299,8 +299,81 @@ def test_block64_long_sequence_hi_lo(oracle_mod):
     check_state(to_np(st[0]), rst[0], what="block64 131072 state")
 
 
-def test_block64_rejected_with_decay():
+@pytest.mark.parametrize("block", [64, 256])
+def test_block_64_256_rejected_with_decay(block):
     q, k, v = la_inputs.qkv((1, 128, 2, D), seed=212, device="cuda")
     with pytest.raises(la.LAError) as e:
-        la.prefill(q, k, v, block=64, decay=torch.ones(2, device="cuda"))
+        la.prefill(q, k, v, block=block, decay=torch.ones(2, device="cuda"))
     assert e.value.status == la.LA_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------------------ row blocks of 256
+@pytest.mark.parametrize("N", [1, 127, 128, 129, 255, 256, 257, 383, 1000])
+@pytest.mark.parametrize("seg", [0, 128, 256, 512])
+def test_block256_ragged_and_segmented(oracle_mod, N, seg):
+    """block = 256: pairs of 128-row tiles share one state snapshot, the second
+    tile's queries meet the first tile's keys in the intra-block product;
+    against the oracle's blocked form at 256 (a segment length of 128 is
+    raised to 256 so that segments hold whole blocks)."""
+    B, H = 2, 3
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=300 + N, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(19)
+    state_in = torch.randn((B, H, D, D), generator=gen, device="cuda") * 0.3
+    la.set_segment_len(seg)
+    out, st = la.prefill(q, k, v, block=256, state_in=state_in, out_dtype=torch.float32)
+    assert la.get_device_status() == la.LA_OK
+    if seg:
+        assert la.last_segment_len() % 256 == 0
+    cu = la_inputs.cu_seqlens_from_lengths([N] * B)
+    qf, kf, vf = (x.reshape(B * N, H, D) for x in (q, k, v))
+    ref, rst = _oracle_prefill(oracle_mod, qf, kf, vf, cu, state_in=state_in, form="blocked", block=256)
+    check_out(to_np(out.reshape(B * N, H, D)), ref, bf16_out=False, what=f"block256 N={N} seg={seg}")
+    check_state(to_np(st), rst, what=f"block256 N={N} seg={seg}")
+
+
+def test_block256_varlen_bf16(oracle_mod):
+    lens = [0, 1, 256, 257, 1000, 0, 2500, 383]
+    H = 4
+    T = sum(lens)
+    q, k, v = la_inputs.qkv((T, H, D), seed=310, device="cuda")
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    la.set_segment_len(512)
+    out, st = la.prefill_varlen(q, k, v, torch.from_numpy(cu).cuda(), max(lens), block=256,
+                                out_dtype=torch.bfloat16)
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = _oracle_prefill(oracle_mod, q, k, v, cu, form="blocked", block=256)
+    check_out(to_np(out), ref, bf16_out=True, what="block256 varlen")
+    check_state(to_np(st), rst, what="block256 varlen states")
+
+
+def test_block256_32k_all_heads(oracle_mod):
+    """The 32K-token, 64-head workload at block 256, bf16 output, every head."""
+    B, N, H = 1, 32768, 64
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=20250101, device="cuda")
+    out, st = la.prefill(q, k, v, block=256, out_dtype=torch.bfloat16)
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = _oracle_prefill(oracle_mod, q[0], k[0], v[0], np.array([0, N], np.int32))
+    check_out(to_np(out[0]), ref, bf16_out=True, what="block256 32K")
+    check_state(to_np(st[0]), rst[0], what="block256 32K states")
+
+
+def test_block256_long_sequence_hi_lo(oracle_mod):
+    B, N, H = 1, 131072, 2
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=311, device="cuda")
+    out, st = la.prefill(q, k, v, block=256, out_dtype=torch.float32)
+    assert la.get_device_status() == la.LA_OK
+    ref, rst = _oracle_prefill(oracle_mod, q[0], k[0], v[0], np.array([0, N], np.int32))
+    check_out(to_np(out[0]), ref, bf16_out=False, what="block256 131072")
+    check_state(to_np(st[0]), rst[0], what="block256 131072 state")
+
+
+def test_blocks_agree():
+    """The three block lengths compute the same operation: outputs agree to the
+    output tolerance, final states to the state tolerance."""
+    B, N, H = 2, 3000, 4
+    q, k, v = la_inputs.qkv((B, N, H, D), seed=312, device="cuda")
+    res = {blk: la.prefill(q, k, v, block=blk, out_dtype=torch.float32) for blk in (64, 128, 256)}
+    assert la.get_device_status() == la.LA_OK
+    for blk in (64, 256):
+        check_out(to_np(res[blk][0]), to_np(res[128][0]), bf16_out=False, what=f"block {blk} vs 128")
+        check_state(to_np(res[blk][1]), to_np(res[128][1]), what=f"block {blk} vs 128 states")

@@ -9,7 +9,7 @@ inputs (the calls share the scratch), and compared element by element with
 the fp64 oracle under the tolerances of the other parity tests, for both
 output dtypes, with and without a carried-in state; the shapes include one
 just under the scratch limit and one where the segments are lengthened past
-65536 tokens (the state then reaches the inter-block product as bf16 hi + lo).
+32768 tokens (the state then reaches the inter-block product as bf16 hi + lo).
 A second comparison against la_prefill on the same inputs, run with the
 segment length the scratch-bound call chose, checks that the two entry points
 compute the same thing.  This file is collected last on purpose."""
@@ -55,7 +55,7 @@ CASES = [
     ((2, 1500, 4), None, None),
     ((1, 32768, 64), 8, None),
     ((4, 4096, 64), 8, 4096),        # 256 (sequence, head) pairs: one segment each, under the limit
-    ((1, 131072, 64), 4, 32768),     # segments of 32768 tokens; the last two end past 65536
+    ((1, 131072, 64), 4, 32768),     # segments of 32768 tokens; the last three end past 32768
 ]
 
 
