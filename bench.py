@@ -446,49 +446,56 @@ def run_cuda(args, world, rank, local):
     f_dense = prefill_survey_exec_flops(tok_heads, BLOCK)
     achieved_gbs = byts / (ms * 1e-3) / 1e9
 
+    legs = set(args.legs.split(",")) if args.legs else None
+    want = lambda name: legs is None or name in legs  # noqa: E731
+
     # ---------------- end to end through the public API with host buffers
-    e2e_steps = max(3, min(args.steps, 20))
-    qh = q.cpu().pin_memory(); kh = k.cpu().pin_memory(); vh = v.cpu().pin_memory()
-    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    sh = torch.empty(st.shape, dtype=st.dtype).pin_memory()
-    bufs = la.make_buffers(B, E2E_CHUNK, H, out.dtype, dev)
+    e2e_steps = max(3, min(args.steps, 20)) if want("e2e") else 0
+    e2e_ms = None
+    if e2e_steps:
+        qh = q.cpu().pin_memory(); kh = k.cpu().pin_memory(); vh = v.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        sh = torch.empty(st.shape, dtype=st.dtype).pin_memory()
+        bufs = la.make_buffers(B, E2E_CHUNK, H, out.dtype, dev)
 
-    def e2e_step():
-        # the public host-memory entry point: chunks of tokens copied in, scanned
-        # and copied out on three streams, the state carried between chunks
-        la.prefill_from_host(qh, kh, vh, chunk_tokens=E2E_CHUNK, out=oh, state_out=sh, buffers=bufs, device=dev)
+        def e2e_step():
+            # the public host-memory entry point (la_prefill_from_host): chunks of
+            # tokens copied in, scanned and copied out on three streams, the state
+            # carried between chunks
+            la.prefill_from_host(qh, kh, vh, chunk_tokens=E2E_CHUNK, out=oh, state_out=sh, buffers=bufs,
+                                 device=dev)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
-    del bufs
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+        del bufs, qh, kh, vh, oh, sh
 
     # ---------------- fused batched decode on its own workload
     dec = None
-    if rank == 0 or world > 1:
+    if want("decode") and (rank == 0 or world > 1):
         dec = bench_decode(la, dev, stream, args, hbm_peak, world)
 
     # ---------------- the same workload at row blocks of 64 and 256
     by_block = {f"block{blk}": bench_prefill_block(la, dev, stream, q, k, v, blk, args, hbm_peak, tc_peak, world)
-                for blk in (64, 256)}
+                for blk in (64, 256) if want(f"block{blk}")}
     # ---------------- the same workload with a per-head decay
-    dec_pref = bench_prefill_decay(la, dev, stream, q, k, v, args, hbm_peak, world)
+    dec_pref = bench_prefill_decay(la, dev, stream, q, k, v, args, hbm_peak, world) if want("decay") else None
 
     # ---------------- the packed varlen batch and the 1M-token prefill
-    varlen = bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank)
-    longc = bench_long_context(la, dev, stream, args, hbm_peak, tc_peak, world, rank)
+    varlen = bench_varlen(la, dev, stream, args, hbm_peak, tc_peak, world, rank) if want("varlen") else None
+    longc = bench_long_context(la, dev, stream, args, hbm_peak, tc_peak, world, rank) if want("long") else None
 
     # ---------------- local prefix of sequence parallelism on the same k, v
-    agg = bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world)
+    agg = bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world) if want("aggregate") else None
     # ---------------- gradients of the prefill on the same q, k, v
-    bwd = bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world)
+    bwd = bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world) if want("backward") else None
 
     status2 = la.get_device_status()
     if rank != 0:
@@ -519,8 +526,10 @@ def run_cuda(args, world, rank, local):
                      "kernel": "la_prefill_kernel", "bytes_per_launch": byts,
                      "duration": "CUDA events around each la_prefill call (scheduler + prefill kernel)",
                      "peak_source": f"{peak_src} hbm_gbs"},
-        "e2e": {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tok/s", "ms_per_step": e2e_ms,
-                "steps": e2e_steps, "api": f"prefill_from_host, {E2E_CHUNK}-token chunks",
+        "e2e": None if e2e_ms is None else {"value": tokens_all / (e2e_ms * 1e-3), "unit": "tok/s", "ms_per_step": e2e_ms,
+                "steps": e2e_steps,
+                "api": f"la_prefill_from_host (C ABI) through prefill_from_host, {E2E_CHUNK}-token chunks pipelined "
+                       "over copy-in / compute / copy-out streams",
                 "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                 "d2h_bytes_per_step": out.numel() * out.element_size() + st.numel() * st.element_size()},
         "gpu_launches": int(launches),
@@ -827,6 +836,9 @@ def main():
                     help="CPU time budget of the oracle baseline sample (rank 0, N=1)")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="approximate total CPU time of the --impl reference run")
+    ap.add_argument("--legs", default="",
+                    help="comma-separated subset of the legs after the main prefill step to run (e2e, decode, "
+                         "block64, block256, decay, varlen, long, aggregate, backward); default all")
     args = ap.parse_args()
     if args.impl == "reference":
         # the oracle runs on the host cores of rank 0 only; no process group needed

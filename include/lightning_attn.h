@@ -221,6 +221,45 @@ LA_API la_status la_mixed_step(const void *q, const void *k, const void *v,
                         cudaStream_t prefill_stream, cudaStream_t decode_stream);
 
 /* ---------------------------------------------------------------------------
+ * Prefill of inputs that live in pinned host memory.  When q, k, v are on the
+ * host the host link, not the kernel, sets the pace (at B=1, H=64, N=32768:
+ * 1.61 GB in and 0.54 GB out, tens of milliseconds against half a
+ * millisecond of compute), so the sequence is cut into chunks of
+ * chunk_tokens tokens pipelined over three streams: chunk c+1 is copied in
+ * on copy_in while chunk c is scanned on compute and chunk c-1 is copied out
+ * on copy_out.  Each chunk is an la_prefill from the state the previous
+ * chunk left (the state-carry identity of the recurrence: the result equals
+ * one prefill of the whole sequence, to rounding).
+ *
+ *   q, k, v     PINNED HOST bf16 [B, N, H, d] (cudaHostAlloc / registered).
+ *   out         PINNED HOST [B, N, H, d] in out_dtype.
+ *   state_in    device fp32 [B, H, d, d] or NULL (zero state).
+ *   state_out   fp32 [B, H, d, d], device or pinned host, or NULL.
+ *   buffers     device scratch of la_prefill_from_host_buffer_size(B,
+ *               chunk_tokens, H, d, out_dtype) bytes, 256-byte aligned,
+ *               caller-owned: two chunk slots of q, k, v and out, the
+ *               running state and a prefill workspace.
+ *   copy_in, compute, copy_out   three streams (may be the same stream, which
+ *               serialises the pipeline).  The copy streams first wait for the
+ *               work already queued on compute; on return, work queued on
+ *               compute after the call sees every result (outputs copied out,
+ *               state_out written).  Nothing is synchronised; the host buffers
+ *               must stay valid until compute reaches that point.
+ * Errors before any work is queued: argument and shape errors, a host buffer
+ * that is not pinned (LA_ERR_INVALID_ARGUMENT), a short buffer
+ * (LA_ERR_WORKSPACE).  The call keeps a few CUDA events per host thread
+ * (created on its first call, reused afterwards) and allocates no memory.
+ * ------------------------------------------------------------------------- */
+LA_API size_t la_prefill_from_host_buffer_size(int B, int chunk_tokens, int H, int d, la_dtype out_dtype);
+
+LA_API la_status la_prefill_from_host(const void *q, const void *k, const void *v,
+                                      int B, int N, int H, int d, int chunk_tokens,
+                                      const float *state_in, void *out, la_dtype out_dtype,
+                                      float *state_out, void *buffers, size_t buffer_bytes,
+                                      cudaStream_t copy_in, cudaStream_t compute,
+                                      cudaStream_t copy_out);
+
+/* ---------------------------------------------------------------------------
  * la_prefill without a workspace argument, for callers that cannot allocate
  * device memory when they call: e.g. a plugin inside a host framework that
  * owns the allocator and offers no allocation hook, or a serving process that

@@ -27,7 +27,8 @@ EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_worksp
             "la_prefill_varlen_slots", "la_decode_step_slots", "la_mixed_step",
             "la_kv_aggregate_workspace_size", "la_kv_aggregate", "la_state_prefix",
             "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_decay",
-            "la_prefill_varlen_decay", "la_decode_step_decay")
+            "la_prefill_varlen_decay", "la_decode_step_decay", "la_prefill_from_host_buffer_size",
+            "la_prefill_from_host")
 
 
 class LAError(RuntimeError):
@@ -76,6 +77,11 @@ def lib():
         L.la_prefill_varlen_decay.restype = c_int
         L.la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp]
         L.la_decode_step_decay.restype = c_int
+        L.la_prefill_from_host_buffer_size.argtypes = [c_int, c_int, c_int, c_int, c_int]
+        L.la_prefill_from_host_buffer_size.restype = sz
+        L.la_prefill_from_host.argtypes = [vp, vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, c_int, vp, vp, sz,
+                                           vp, vp, vp]
+        L.la_prefill_from_host.restype = c_int
         L.la_prefill_varlen_slots.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, c_int,
                                               vp, c_int, vp, c_int, vp, sz, vp]
         L.la_prefill_varlen_slots.restype = c_int

@@ -515,6 +515,138 @@ la_status la_mixed_step(const void *q, const void *k, const void *v, const int *
 }
 
 
+// ---------------------------------------------------------------------------
+// Prefill of inputs in pinned host memory: chunks of tokens copied in, scanned
+// from the carried state and copied out, pipelined over three streams.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct HostLayout {
+    size_t slot_in, slot_out, slot, state, ws, total;
+};
+
+HostLayout host_layout(int B, int C, int H, size_t esz) {
+    HostLayout l;
+    l.slot_in = round_up((size_t)B * C * H * la::D * 2, 256);
+    l.slot_out = round_up((size_t)B * C * H * la::D * esz, 256);
+    l.slot = 3 * l.slot_in + l.slot_out;
+    l.state = round_up((size_t)B * H * la::D * la::D * 4, 256);
+    // the workspace of the longest chunk, or of a shorter last chunk (which may
+    // be cut into more, shorter segments)
+    size_t ws = 0;
+    for (int n = 1; n <= C; ++n) {
+        const size_t w = la_prefill_workspace_size(B, n, H, la::D, 0);
+        ws = w > ws ? w : ws;
+    }
+    l.ws = round_up(ws, 256);
+    l.total = 2 * l.slot + l.state + l.ws;
+    return l;
+}
+
+bool pinned_host(const void *p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
+}  // namespace
+
+size_t la_prefill_from_host_buffer_size(int B, int chunk_tokens, int H, int d, la_dtype out_dtype) {
+    if (B <= 0 || chunk_tokens <= 0 || H <= 0 || d != la::D) return 0;
+    return host_layout(B, chunk_tokens, H, out_dtype == LA_FP32 ? 4 : 2).total;
+}
+
+la_status la_prefill_from_host(const void *q, const void *k, const void *v, int B, int N, int H, int d,
+                               int chunk_tokens, const float *state_in, void *out, la_dtype out_dtype,
+                               float *state_out, void *buffers, size_t buffer_bytes, cudaStream_t copy_in,
+                               cudaStream_t compute, cudaStream_t copy_out) {
+    la_status st = check_common(H, d, 0, out_dtype);
+    if (st != LA_OK) return st;
+    if (B < 0 || N < 0 || chunk_tokens <= 0) return LA_ERR_INVALID_ARGUMENT;
+    if (B == 0) return LA_OK;
+    if ((long long)B * N > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    const int C = chunk_tokens < N ? chunk_tokens : (N > 0 ? N : 1);
+    const size_t esz = out_dtype == LA_FP32 ? 4 : 2;
+    const HostLayout l = host_layout(B, C, H, esz);
+    if (!buffers || buffer_bytes < l.total) return LA_ERR_WORKSPACE;
+    if (!aligned(buffers, 256)) return LA_ERR_INVALID_ARGUMENT;
+    if (N > 0) {
+        if (!q || !k || !v || !out) return LA_ERR_INVALID_ARGUMENT;
+        const void *host[4] = {q, k, v, out};
+        for (const void *p : host)
+            if (!pinned_host(p)) return LA_ERR_INVALID_ARGUMENT;  // pinned host memory only
+    }
+    if ((state_in && !aligned(state_in, 16)) || (state_out && !aligned(state_out, 16))) return LA_ERR_INVALID_ARGUMENT;
+    const size_t n_state = (size_t)B * H * la::D * la::D * 4;
+    if (ranges_overlap(buffers, l.total, state_in, n_state) || ranges_overlap(buffers, l.total, state_out, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+
+    // events: per host thread and device, created once, reused by every call
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LA_ERR_CUDA;
+    static thread_local cudaEvent_t events[kMaxDevices][7] = {};
+    cudaEvent_t *ev = events[dev];
+    if (!ev[6])  // the last one is set only once all seven exist
+        for (int i = 0; i < 7; ++i)
+            if (!ev[i] && cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) != cudaSuccess) return LA_ERR_CUDA;
+    cudaEvent_t *ev_in = ev, *ev_cmp = ev + 2, *ev_out = ev + 4, ev_start = ev[6];
+
+    uint8_t *base = static_cast<uint8_t *>(buffers);
+    float *state = reinterpret_cast<float *>(base + 2 * l.slot);
+    void *ws = base + 2 * l.slot + l.state;
+    // the copy streams start after the compute stream's earlier work
+    if (cudaEventRecord(ev_start, compute) != cudaSuccess) return LA_ERR_CUDA;
+    if (cudaStreamWaitEvent(copy_in, ev_start, 0) != cudaSuccess) return LA_ERR_CUDA;
+    if (cudaStreamWaitEvent(copy_out, ev_start, 0) != cudaSuccess) return LA_ERR_CUDA;
+    // the running state starts as state_in (or zero)
+    if ((st = la_state_prefix(nullptr, 0, state_in, state, B * H, d, compute)) != LA_OK) return st;
+
+    const size_t row_in = (size_t)H * la::D * 2, row_out = (size_t)H * la::D * esz;
+    const int nchunks = N > 0 ? (N + C - 1) / C : 0;
+    for (int c = 0; c < nchunks; ++c) {
+        const int j = c & 1;
+        const int t0 = c * C, n = (t0 + C < N ? C : N - t0);
+        uint8_t *slot = base + j * l.slot;
+        uint8_t *dq = slot, *dk = slot + l.slot_in, *dv = slot + 2 * l.slot_in, *dout = slot + 3 * l.slot_in;
+        // copy in (slot j is free once the chunk two before it was scanned and copied out)
+        if (c >= 2 && (cudaStreamWaitEvent(copy_in, ev_cmp[j], 0) != cudaSuccess ||
+                       cudaStreamWaitEvent(copy_in, ev_out[j], 0) != cudaSuccess))
+            return LA_ERR_CUDA;
+        for (int b = 0; b < B; ++b) {
+            const size_t src = ((size_t)b * N + t0) * row_in, dst = (size_t)b * n * row_in, bytes = (size_t)n * row_in;
+            if (cudaMemcpyAsync(dq + dst, static_cast<const uint8_t *>(q) + src, bytes, cudaMemcpyHostToDevice, copy_in) != cudaSuccess ||
+                cudaMemcpyAsync(dk + dst, static_cast<const uint8_t *>(k) + src, bytes, cudaMemcpyHostToDevice, copy_in) != cudaSuccess ||
+                cudaMemcpyAsync(dv + dst, static_cast<const uint8_t *>(v) + src, bytes, cudaMemcpyHostToDevice, copy_in) != cudaSuccess)
+                return LA_ERR_CUDA;
+        }
+        if (cudaEventRecord(ev_in[j], copy_in) != cudaSuccess) return LA_ERR_CUDA;
+        // scan the chunk from the carried state, in place (the state-carry
+        // identity: a prefill of chunk c from the state after chunk c-1 is the
+        // prefill of the longer sequence)
+        if (cudaStreamWaitEvent(compute, ev_in[j], 0) != cudaSuccess) return LA_ERR_CUDA;
+        if (c >= 2 && cudaStreamWaitEvent(compute, ev_out[j], 0) != cudaSuccess) return LA_ERR_CUDA;
+        st = la_prefill(dq, dk, dv, B, n, H, d, 0, state, dout, out_dtype, state, ws, l.ws, compute);
+        if (st != LA_OK) return st;
+        if (cudaEventRecord(ev_cmp[j], compute) != cudaSuccess) return LA_ERR_CUDA;
+        // copy out
+        if (cudaStreamWaitEvent(copy_out, ev_cmp[j], 0) != cudaSuccess) return LA_ERR_CUDA;
+        for (int b = 0; b < B; ++b) {
+            const size_t dst = ((size_t)b * N + t0) * row_out, src = (size_t)b * n * row_out, bytes = (size_t)n * row_out;
+            if (cudaMemcpyAsync(static_cast<uint8_t *>(out) + dst, dout + src, bytes, cudaMemcpyDeviceToHost, copy_out) != cudaSuccess)
+                return LA_ERR_CUDA;
+        }
+        if (cudaEventRecord(ev_out[j], copy_out) != cudaSuccess) return LA_ERR_CUDA;
+    }
+    if (state_out && cudaMemcpyAsync(state_out, state, n_state, cudaMemcpyDefault, compute) != cudaSuccess)
+        return LA_ERR_CUDA;
+    // work queued on the compute stream after this call sees every result
+    if (nchunks > 0 && cudaStreamWaitEvent(compute, ev_out[(nchunks - 1) & 1], 0) != cudaSuccess) return LA_ERR_CUDA;
+    return LA_OK;
+}
+
 la_status la_get_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return LA_ERR_CUDA;
     int v = 0;

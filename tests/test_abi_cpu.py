@@ -264,6 +264,26 @@ def test_host_memory_entry_point_validates_before_any_copy():
             la.prefill_from_host(bad, bad, bad)
 
 
+def test_host_pipeline_argument_errors(L):
+    """la_prefill_from_host checks shapes, the scratch size and alignment, and
+    that the host buffers are pinned, before queueing anything."""
+    far = 1 << 40
+    need = L.la_prefill_from_host_buffer_size(1, 256, 2, 128, 0)
+    assert need > 0 and L.la_prefill_from_host_buffer_size(1, 256, 2, 64, 0) == 0
+    assert L.la_prefill_from_host_buffer_size(1, 256, 2, 128, 1) > need        # fp32 output slots
+
+    def call(B=1, N=512, H=2, d=128, chunk=256, buf=far, nbytes=None, host=FAKE):
+        return L.la_prefill_from_host(V(host), V(host), V(host), B, N, H, d, chunk, None, V(host), 0, None,
+                                      V(buf), need if nbytes is None else nbytes, None, None, None)
+    assert call(d=64) == la.LA_ERR_UNSUPPORTED
+    assert call(chunk=0) == la.LA_ERR_INVALID_ARGUMENT
+    assert call(N=-1) == la.LA_ERR_INVALID_ARGUMENT
+    assert call(B=0) == la.LA_OK
+    assert call(nbytes=need - 1) == la.LA_ERR_WORKSPACE
+    assert call(buf=far + 16) == la.LA_ERR_INVALID_ARGUMENT                  # scratch alignment
+    assert call() == la.LA_ERR_INVALID_ARGUMENT                              # host buffers not pinned
+
+
 def test_header_is_plain_c_and_links_from_c(tmp_path):
     """The boundary as a C user sees it: a C99 translation unit that includes
     include/lightning_attn.h, takes the address of every entry point, links
