@@ -236,6 +236,13 @@ class NvmlClockSampler:
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    # every other reason bit, reported so that a clock below the maximum is
+    # never left unexplained by the record
+    OTHER_REASONS = (("gpu_idle", "nvmlClocksEventReasonGpuIdle"),
+                     ("applications_clocks_setting", "nvmlClocksEventReasonApplicationsClocksSetting"),
+                     ("sync_boost", "nvmlClocksEventReasonSyncBoost"),
+                     ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+                     ("display_clock_setting", "nvmlClocksEventReasonDisplayClockSetting"))
 
     def __init__(self, dev: torch.device, period: float = 0.002):
         self.samples = []
@@ -250,6 +257,11 @@ class NvmlClockSampler:
             self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
             self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
             self.masks = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            self.other_masks = [(name, getattr(nv, attr)) for name, attr in self.OTHER_REASONS if hasattr(nv, attr)]
+            try:
+                self.power_limit_w = nv.nvmlDeviceGetEnforcedPowerLimit(self.h) / 1000.0
+            except Exception:
+                self.power_limit_w = None
             self.period = period
             self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
@@ -263,7 +275,11 @@ class NvmlClockSampler:
             try:
                 mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                self.samples.append((time.time(), mhz, rs))
+                try:
+                    mw = nv.nvmlDeviceGetPowerUsage(self.h)
+                except Exception:
+                    mw = -1
+                self.samples.append((time.time(), mhz, rs, mw))
             except Exception:
                 pass
             time.sleep(self.period)
@@ -272,12 +288,19 @@ class NvmlClockSampler:
         self._stop.set()
 
     def summary(self, t0: float, t1: float):
-        rows = [(m, r) for (t, m, r) in self.samples if t0 <= t <= t1]
+        rows = [(m, r, w) for (t, m, r, w) in self.samples if t0 <= t <= t1]
         if not rows:
             return None
-        reasons = sorted({name for (_, r) in rows for (name, mask) in self.masks if r & mask})
-        return {"sm_mhz": float(np.median([m for m, _ in rows])), "sm_max_mhz": float(self.max_mhz),
-                "reasons": reasons, "samples": len(rows), "source": "NVML, 2 ms period"}
+        reasons = sorted({name for (_, r, _) in rows for (name, mask) in self.masks if r & mask})
+        other = sorted({name for (_, r, _) in rows for (name, mask) in self.other_masks if r & mask})
+        watts = [w / 1000.0 for (_, _, w) in rows if w >= 0]
+        out = {"sm_mhz": float(np.median([m for m, _, _ in rows])), "sm_max_mhz": float(self.max_mhz),
+               "reasons": reasons, "other_reasons": other, "samples": len(rows), "source": "NVML, 2 ms period"}
+        if watts:
+            out["power_w_median"] = float(np.median(watts))
+            out["power_w_max"] = float(np.max(watts))
+            out["power_limit_w"] = self.power_limit_w
+        return out
 
 
 def dist_setup():
@@ -604,7 +627,7 @@ def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
     return {"workload": "prefill backward B=1 H=64 N=32768 d=128, bf16 dq/dk/dv + fp32 dS_in",
             "ms_per_call": ms, "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (three scans) + la_kv_aggregate_kernel (one sum)",
+                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (dQ scan + paired dK/dV scan) + la_kv_aggregate_kernel (one sum)",
                          "traffic": None, "bytes_per_launch": byts,
                          "duration": "CUDA events around each la_prefill_backward call (about ten kernels)"}}
 

@@ -147,8 +147,8 @@ la_status ensure_smem_attr(SmemAttr &a, Kernel *kernel, int bytes) {
     return LA_OK;
 }
 
-SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_prefill_decay, g_attr_prefill_b64, g_attr_prefill_b256,
-    g_attr_agg;
+SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_prefill_pair, g_attr_prefill_decay, g_attr_prefill_b64,
+    g_attr_prefill_b256, g_attr_agg;
 
 bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
     if (!a || !b || na == 0 || nb == 0) return false;
@@ -164,10 +164,11 @@ la_status check_common(int H, int d, int block, la_dtype out_dtype) {
     return LA_OK;
 }
 
-// The prefill kernel instantiation for a row-block length (0 = 128).
+// The prefill kernel instantiation for a row-block length (0 = 128); with
+// mq2 (ANTI only), the paired instantiation that also runs (q2, v, k).
 template <bool ANTI, bool DECAY>
 la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                         const la::PrefillParams &pp, cudaStream_t stream);
+                         const la::PrefillParams &pp, cudaStream_t stream, const CUtensorMap *mq2 = nullptr);
 
 // Shared body of la_prefill / la_prefill_varlen.
 la_status prefill_impl(const void *q, const void *k, const void *v, const int *cu, int fixed_len,
@@ -175,7 +176,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
                        const float *state_in, void *out, la_dtype out_dtype, float *state_out,
                        void *workspace, size_t ws_bytes, cudaStream_t stream,
                        const int *slots = nullptr, int n_slots = 0, bool anti = false,
-                       const float *decay = nullptr) {
+                       const float *decay = nullptr, const void *q2 = nullptr, void *out2 = nullptr) {
     la_status st = check_common(H, d, block, out_dtype);
     if (st != LA_OK) return st;
     if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -191,6 +192,10 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
         return LA_ERR_INVALID_ARGUMENT;
     if (decay && (anti || !aligned(decay, 4))) return LA_ERR_INVALID_ARGUMENT;
     if ((block == 64 || block == 256) && (anti || decay)) return LA_ERR_UNSUPPORTED;
+    // paired ANTI problems (q, k, v) and (q2, v, k): one bf16 state term only
+    if ((q2 != nullptr) != (out2 != nullptr)) return LA_ERR_INVALID_ARGUMENT;
+    if (q2 && (!anti || (block != 0 && block != la::BLK) || slots || state_out || max_seqlen > LA_LO_SPLIT_FROM))
+        return LA_ERR_UNSUPPORTED;
     const size_t n_state = (size_t)(slots ? n_slots : nseq) * H * la::D * la::D * 4;
     if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
@@ -201,6 +206,14 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     }
     if (ranges_overlap(out, n_out, state_out, n_state) || ranges_overlap(out, n_out, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
+    if (q2) {
+        if (!aligned(q2, 16) || !aligned(out2, 16)) return LA_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(out2, n_out, out, n_out) || ranges_overlap(out2, n_out, state_in, n_state) ||
+            ranges_overlap(out2, n_out, q2, n_in) || ranges_overlap(out, n_out, q2, n_in))
+            return LA_ERR_INVALID_ARGUMENT;
+        for (const void *p : ins)
+            if (ranges_overlap(out2, n_out, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+    }
 
     const int L = choose_seg_len(nseq, T, H, block);
     if (L <= 0 || L % la::BLK) return LA_ERR_INVALID_ARGUMENT;
@@ -240,9 +253,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     ++g_launches;
     if (T == 0) return LA_OK;
 
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mq2;
     if (!encode_qkv_map(&mq, q, (int)T, H) || !encode_qkv_map(&mk, k, (int)T, H) ||
-        !encode_qkv_map(&mv, v, (int)T, H))
+        !encode_qkv_map(&mv, v, (int)T, H) || (q2 && !encode_qkv_map(&mq2, q2, (int)T, H)))
         return LA_ERR_CUDA;
 
     la::PrefillParams pp;
@@ -250,8 +263,9 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.state_out = state_out;
     pp.slots = slots;
     pp.out = out;
+    pp.out2 = out2;
     pp.out_fp32 = out_dtype == LA_FP32;
-    pp.out_al32 = aligned(out, 32);
+    pp.out_al32 = aligned(out, 32) && (!out2 || aligned(out2, 32));
     pp.H = H;
     pp.hdr = sp.hdr;
     pp.segs = sp.segs;
@@ -266,7 +280,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
 
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    st = anti ? launch_prefill<true, false>(block, grid, mq, mk, mv, pp, stream)
+    st = anti ? launch_prefill<true, false>(block, grid, mq, mk, mv, pp, stream, q2 ? &mq2 : nullptr)
          : decay ? launch_prefill<false, true>(block, grid, mq, mk, mv, pp, stream)
                  : launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream);
     if (st != LA_OK) return st;
@@ -274,18 +288,23 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     return LA_OK;
 }
 
-template <bool ANTI, bool DECAY, int BK>
+template <bool ANTI, bool DECAY, int BK, bool PAIR = false>
 la_status launch_prefill_bk(SmemAttr &attr, int grid, const CUtensorMap &mq, const CUtensorMap &mk,
-                            const CUtensorMap &mv, const la::PrefillParams &pp, cudaStream_t stream) {
-    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<ANTI, DECAY, BK>, la::PREFILL_SMEM);
+                            const CUtensorMap &mv, const la::PrefillParams &pp, cudaStream_t stream,
+                            const CUtensorMap *mq2 = nullptr) {
+    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<ANTI, DECAY, BK, PAIR>, la::PREFILL_SMEM);
     if (st != LA_OK) return st;
-    la::la_prefill_kernel<ANTI, DECAY, BK><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(mq, mk, mv, pp);
+    // (unpaired instantiations never read the fourth map)
+    la::la_prefill_kernel<ANTI, DECAY, BK, PAIR><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(
+        mq, mk, mv, mq2 ? *mq2 : mq, pp);
     return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
 template <bool ANTI, bool DECAY>
 la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
-                         const la::PrefillParams &pp, cudaStream_t stream) {
+                         const la::PrefillParams &pp, cudaStream_t stream, const CUtensorMap *mq2) {
+    if (ANTI && mq2)
+        return launch_prefill_bk<true, false, 128, true>(g_attr_prefill_pair, grid, mq, mk, mv, pp, stream, mq2);
     if (ANTI) return launch_prefill_bk<true, false, 128>(g_attr_prefill_anti, grid, mq, mk, mv, pp, stream);
     if (DECAY) return launch_prefill_bk<false, true, 128>(g_attr_prefill_decay, grid, mq, mk, mv, pp, stream);
     if (block == 64) return launch_prefill_bk<false, false, 64>(g_attr_prefill_b64, grid, mq, mk, mv, pp, stream);
@@ -356,7 +375,7 @@ la_status launch_transpose(const float *in, float *out, long long nstates, cudaS
 }
 
 // Workspace of la_prefill_backward: one prefill workspace (reused by the
-// three scans, which run in stream order), one la_kv_aggregate workspace and
+// scans, which run in stream order), one la_kv_aggregate workspace and
 // three [B, H, D, D] fp32 states.
 struct BwdLayout {
     size_t prefill, agg, st0, st1, st2, total;
@@ -813,17 +832,27 @@ la_status la_prefill_backward(const void *q, const void *k, const void *v, const
         if ((st = la_state_prefix(C, 1, dstate_out, Bs, (int)nstates, d, stream)) != LA_OK) return st;
         s0v = Bs;
     }
-    if ((st = launch_transpose(s0v, A, nstates, stream)) != LA_OK) return st;
-    // dK: an ANTI scan of (q, k, v) = (V, dO, Q) from W_k
-    //     dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
-    st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, A, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
-                      stream, nullptr, 0, true);
-    if (st != LA_OK) return st;
     // dV: an ANTI scan of (q, k, v) = (K, Q, dO) from W_v
     //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t = sum_{t >= s} (q_t . k_s) g_t + k_s G
-    st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
-                      stream, nullptr, 0, true);
-    if (st != LA_OK) return st;
+    // dK: an ANTI scan of (q, k, v) = (V, dO, Q) from W_k = W_v^T
+    //     dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
+    // Up to LA_LO_SPLIT_FROM tokens both run as one paired scan (dK as the
+    // second problem, its state the transpose of dV's); longer sequences hand
+    // the state to the inter-block product as hi + lo, which the paired scan
+    // does not, and run the two scans one after the other.
+    if (N <= LA_LO_SPLIT_FROM) {
+        st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
+                          stream, nullptr, 0, true, nullptr, v, dk);
+        if (st != LA_OK) return st;
+    } else {
+        if ((st = launch_transpose(s0v, A, nstates, stream)) != LA_OK) return st;
+        st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, A, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
+                          stream, nullptr, 0, true);
+        if (st != LA_OK) return st;
+        st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
+                          stream, nullptr, 0, true);
+        if (st != LA_OK) return st;
+    }
     if (dstate_in) return la_state_prefix(nullptr, 0, s0v, dstate_in, (int)nstates, d, stream);
     return LA_OK;
 }
@@ -980,6 +1009,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.state_out = state_out;
     pp.slots = nullptr;
     pp.out = out;
+    pp.out2 = nullptr;
     pp.out_fp32 = out_dtype == LA_FP32;
     pp.out_al32 = aligned(out, 32);
     pp.H = H;

@@ -54,6 +54,18 @@
 // hi^T V + lo^T V.  The state warps rescale S by lambda^{nb} in TMEM when they
 // take each snapshot.  DECAY and ANTI are not combined.
 //
+// A third flag, PAIR (with ANTI, 128-row blocks and S as one bf16 term), runs
+// two ANTI problems that share their keys, values and state in one sweep:
+// problem 1 is (q, k, v) and problem 2 is (q2, v, k), whose state
+// sum v^T k is the transpose of problem 1's.  Each row block b becomes two
+// sub-blocks, u = 2b (problem 1) and u = 2b + 1 (problem 2), which take turns
+// in the score buffer, in the Q ring (q tile, then q2 tile) and in the two O
+// buffers (sub-block u in buffer u & 1; problem 1 writes `out`, problem 2
+// `out2`).  a5 of problem 2 reads the same state snapshot through K-major
+// descriptors, which present it transposed; a6 runs once per block.  With
+// (q, k, v, q2) = (K, Q, dO, V) the two outputs are the gradients dV and dK,
+// and Q and dO are read once for both.
+//
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
 //               loads Q
@@ -138,6 +150,7 @@ struct PrefillParams {
     float *state_out;       // [nseq, H, D, D] or null (or a pool of states, see slots)
     const int *slots;       // null, or [nseq]: sequence i reads and writes state slots[i]
     void *out;              // [T, H, D]
+    void *out2;             // PAIR: [T, H, D], the second problem's output (same dtype)
     int out_fp32;
     int out_al32;           // out is 32-byte aligned: rows are written with 32-byte stores
     int H;
@@ -414,13 +427,16 @@ __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane
     return item[IT_VALID] != 0;
 }
 
-template <bool ANTI, bool DECAY, int BK>
+template <bool ANTI, bool DECAY, int BK, bool PAIR = false>
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ PrefillParams p) {
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq2,
+                  const __grid_constant__ PrefillParams p) {
     static_assert(BK == 64 || BK == 128 || BK == 256, "row blocks of 64, 128 or 256 tokens");
     static_assert(BK == 128 || (!ANTI && !DECAY), "64- and 256-row blocks: the plain forward only");
+    static_assert(!PAIR || (ANTI && !DECAY && BK == 128), "PAIR: two ANTI problems at 128-row blocks");
     constexpr bool B64 = BK == 64;  // two 64-row blocks per 128-row tile
+    constexpr int SUBS = PAIR ? 2 : 1;  // sub-blocks per row block (PAIR: problem 1, problem 2)
     // BK == 256: one row block per pair of 128-row tiles (see the MMA warp)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -463,6 +479,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         tma_prefetch_desc(&tmq);
         tma_prefetch_desc(&tmk);
         tma_prefetch_desc(&tmv);
+        if (PAIR) tma_prefetch_desc(&tmq2);
     }
     if (warp == 1) {
         tmem_alloc(&cb->tmem_base, TM_COLS);
@@ -506,7 +523,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const int jj = seg.w & (SEG_LAST - 1);
                     const long long seg_end = (long long)jj * p.seg_len + (seg.z - seg.y);
                     item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) |
-                                     ((ANTI ? p.anti_lo != 0 : seg_end > LA_LO_SPLIT_FROM) ? ITF_LO : 0);
+                                     ((ANTI ? (!PAIR && p.anti_lo != 0) : seg_end > LA_LO_SPLIT_FROM) ? ITF_LO : 0);
                 }
                 mbar_arrive(&cb->item_full[islot]);
                 ++it;
@@ -556,13 +573,15 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 if (!item[IT_VALID]) break;
                 const int h = item[IT_H], tok0 = item[IT_TOK0];
                 const int nblk = (item[IT_TOK1] - tok0 + BLK - 1) / BLK;
-                for (int b = 0; b < nblk; ++b) {
+                for (int u = 0; u < SUBS * nblk; ++u) {  // PAIR: q and q2 tiles of each block in turn
+                    const int b = u / SUBS;
                     if (cb->abort) { ok = false; break; }
                     if (PF_Q > 0 && b + PF_Q < nblk) tma_prefetch_4d(&tmq, 0, h, tok0 + (b + PF_Q) * BLK, 0, pol_last);
                     const int qs = q_n % Q_STAGES;
                     if (!wait_or_abort(&cb->q_empty[qs], ((q_n / Q_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
                     mbar_expect_tx(&cb->q_full[qs], TILE_BYTES);
-                    tma_load_4d(smem + SM_Q + qs * TILE_BYTES, &tmq, &cb->q_full[qs], 0, h, tok0 + b * BLK, 0, pol_first);
+                    tma_load_4d(smem + SM_Q + qs * TILE_BYTES, (PAIR && (u & 1)) ? &tmq2 : &tmq, &cb->q_full[qs], 0, h,
+                                tok0 + b * BLK, 0, pol_first);
                     q_last_fill[qs] = q_n / Q_STAGES;
                     ++q_n;
                 }
@@ -651,6 +670,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const bool want_final = last && p.state_out != nullptr;
             const uint32_t kv0 = kv_n, q0 = q_n, blk0 = blk_n;
             int i2 = 0, i4 = 0, i5 = 0, sub = 0;  // next block of a2 / a4 / a5; a5 sub-step pending
+            const int nsub = SUBS * nblk;         // PAIR: i2, i4, i5 count sub-blocks
             uint32_t spins = 0;
             uint64_t deadline = 0;
             if constexpr (BK == 256) {
@@ -810,7 +830,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
                 stp_n += nsteps;
             } else
-            while (i4 < nblk) {
+            while (i4 < nsub) {
                 bool prog = false;
                 // O chain, a4(i4): P ready, a5 of the block issued
                 // (DECAY: P ready also means the block's K rows are scaled into
@@ -819,8 +839,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const uint32_t bn = blk0 + i4;
                     if (ready(&cb->p_full, bn & 1)) {
                         tc_fence_after();
-                        const int s = (kv0 + i4) % KV_STAGES;
-                        const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
+                        const bool second = PAIR && (i4 & 1);  // problem 2: its values are the K tile
+                        const int s = (kv0 + i4 / SUBS) % KV_STAGES;
+                        const uint32_t vt = sbase + (second ? SM_K : SM_V) + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < BLK / 16; ++kk)  // P: first 64 score columns; DECAY: P V
                             mma_ts_w(tmem + TM_O + ob(bn) * 128, tmem + TM_SC + kk * 8, desc_mnmajor(vt, kk), ID_PV,
@@ -841,7 +862,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                             tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // a5 and a6 have read the Q slot
                         }
                         tc_commit_w(&cb->o_full[ob(bn)]);
-                        tc_commit_w(&cb->kv_empty[s]);  // a2, a6 and a4 of this block are issued
+                        if (!PAIR || second) tc_commit_w(&cb->kv_empty[s]);  // a2, a6 and a4 of this block are issued
                         ++i4;
                         prog = true;
                     }
@@ -851,19 +872,24 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 // ready, the block's O buffer free (block i5 - 2 read out; for the
                 // first block of a segment with a successor, A_j read out of it)
                 // DECAY: a5 goes to O buffer 1 and a6 waits for the scaled keys
+                // PAIR: the second sub-block reads the snapshot the first one waited
+                // for (released after both), into the other O buffer
                 if (i5 < i2) {
                     const uint32_t bn = blk0 + i5;
+                    const bool second = PAIR && (i5 & 1);
                     const bool a_read = last || i5 > 0 || ready(&cb->a_free, afree_n & 1);
-                    if (a_read && ready(&cb->snap_full, snap_n & 1) && ready(&cb->o_empty[ob(bn)], obpar(bn) ^ 1)) {
+                    if (a_read && (second || ready(&cb->snap_full, snap_n & 1)) &&
+                        ready(&cb->o_empty[ob(bn)], obpar(bn) ^ 1)) {
                         tc_fence_after();
-                        const int s = (kv0 + i5) % KV_STAGES;
+                        const int bi = i5 / SUBS;  // row block
+                        const int s = (kv0 + bi) % KV_STAGES;
                         const uint32_t qn = q0 + i5;
                         const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
                         const uint32_t sh = sbase + SM_SHI, sl = sbase + SM_SLO;
                         const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
                         const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
                         const uint32_t tq = DECAY ? tmem + TM_O + 128 : tmem + TM_O + ob(bn) * 128;
-                        const bool upd = (i5 < nblk - 1) || want_final;
+                        const bool upd = (bi < nblk - 1) || want_final;
                         // sub-step: one snapshot arrival = one column half (hi + lo
                         // mode) of one row half (64-row blocks) of the tile
                         const int nch = lo ? 2 : 1;
@@ -871,7 +897,11 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const int ch = sub % nch;            // hi + lo: columns 64 ch .. 64 ch + 63
                         // 64-row blocks: only the lanes (rows) of this block are written
                         const uint32_t m_lo = (B64 && rh == 1) ? ~0u : 0u, m_hi = (B64 && rh == 0) ? ~0u : 0u;
-                        if (!lo) {  // O = Q S, S = the whole [128 x 128] snapshot
+                        if (second) {  // O = Q2 S^T: K-major reads of the snapshot give S transposed
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk)
+                                mma_ss_w(tq, desc_kmajor(qt, kk), desc_kmajor(sh, kk), ID_QK, kk > 0 ? 1u : 0u);
+                        } else if (!lo) {  // O = Q S, S = the whole [128 x 128] snapshot
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 if (B64)
@@ -899,8 +929,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                     mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
                             }
                         }
-                        tc_commit_w(&cb->snap_empty);
-                        ++snap_n;
+                        if (!PAIR || second) {
+                            tc_commit_w(&cb->snap_empty);
+                            ++snap_n;
+                        }
                         const bool rh_done = ch == nch - 1;
                         const bool tile_done = rh_done && (!B64 || rh == 1);
                         if (!last && i5 == 0 && tile_done) ++afree_n;
@@ -916,7 +948,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                 tc_commit_w(&cb->a5_done);  // the Q slot may now take the block's K lo
                             } else {
                                 tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // a2 and a5 have read the Q tile
-                                if (upd) {  // a6: S += K^T V (S_{<b} has been read out); 64-row blocks: rows 64-127
+                                // PAIR: a6 after the first sub-block's a5 (S has been read
+                                // out of TMEM; the snapshot in shared memory stays for the
+                                // second)
+                                if (upd && !second) {  // a6: S += K^T V (S_{<b} has been read out); 64-row blocks: rows 64-127
 #pragma unroll
                                     for (int kk = B64 ? BLK / 32 : 0; kk < BLK / 16; ++kk)
                                         mma_ss_w(tmem + TM_S, desc_mnmajor(kt, kk), desc_mnmajor(vt, kk), ID_KV, 1u);
@@ -931,12 +966,14 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
                 // intra chain, a2(i2): its score buffer free (a4 of block i2 - 1
                 // issued), tiles landed
-                if (i2 < nblk && i2 <= i4) {
-                    const int s = (kv0 + i2) % KV_STAGES;
-                    const uint32_t kn = (kv0 + i2) / KV_STAGES, qn = q0 + i2;
+                if (i2 < nsub && i2 <= i4) {
+                    const int bi = i2 / SUBS;
+                    const bool second = PAIR && (i2 & 1);  // problem 2: its keys are the V tile
+                    const int s = (kv0 + bi) % KV_STAGES;
+                    const uint32_t kn = (kv0 + bi) / KV_STAGES, qn = q0 + i2;
                     if (ready(&cb->kv_full[s], kn & 1) && ready(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1)) {
-                        const int valid = min(BLK, tok1 - (tok0 + i2 * BLK));
-                        if (valid < BLK) {
+                        const int valid = min(BLK, tok1 - (tok0 + bi * BLK));
+                        if (valid < BLK && !second) {  // (PAIR: the first sub-block's a2 reads the tiles first)
                             // rows past the end of the sequence must add nothing to S or O:
                             // zero them in K and V (they may hold the next sequence's tokens)
                             uint8_t *kp = smem + SM_K + s * TILE_BYTES;
@@ -952,7 +989,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         }
                         tc_fence_after();
                         const uint32_t qt = sbase + SM_Q + (qn % Q_STAGES) * TILE_BYTES;
-                        const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
+                        const uint32_t kt = sbase + (second ? SM_V : SM_K) + s * TILE_BYTES;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)  // a2: Sc = Q K^T
                             mma_ss_w(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
@@ -983,8 +1020,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 }
             }
             kv_n = kv0 + nblk;
-            q_n = q0 + nblk;
-            blk_n = blk0 + nblk;
+            q_n = q0 + nsub;
+            blk_n = blk0 + nsub;
         }
         // Tear-down: all MMAs issued by this thread must finish before TMEM is freed.
         __syncwarp();
@@ -1032,7 +1069,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             // score steps: one per tile, or, with 256-row blocks, three per pair of
             // tiles (the third, the second tile's queries against the first tile's
             // keys, is not masked)
-            const int nsteps = BK == 256 ? 3 * (nblk / 2) + (nblk & 1) : nblk;
+            // (PAIR: two per block, one per problem, the same mask)
+            const int nsteps = BK == 256 ? 3 * (nblk / 2) + (nblk & 1) : SUBS * nblk;
             for (int b = 0; b < nsteps; ++b) {
                 // P = bf16(Sc ⊙ M), inclusive mask (exclusive under ANTI), packed
                 // two per 32-bit column over the first 64 score columns
@@ -1113,8 +1151,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             }
             // DECAY: the inter-block term of row r carries lambda^{r+1}
             const float fq = DECAY ? decay_pow(log2f(__ldg(p.decay + h)), r + 1) : 1.f;
-            for (int b = 0; b < nblk && ok; ++b) {
-                const uint32_t bn = blk_n + b;
+            for (int u = 0; u < SUBS * nblk && ok; ++u) {  // PAIR: out, then out2, per block
+                const int b = u / SUBS;
+                const uint32_t bn = blk_n + u;
+                void *const outp = (PAIR && (u & 1)) ? p.out2 : p.out;
                 const int row0 = tok0 + b * BLK;
                 const int valid = min(BLK, tok1 - row0);
                 const uint32_t obuf = DECAY ? 0u : (bn & 1), opar = DECAY ? (bn & 1) : ((bn >> 1) & 1);
@@ -1146,7 +1186,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                 uint32_t w[16];
 #pragma unroll
                                 for (int i = 0; i < 16; ++i) w[i] = bf16x2_round(xi[2 * i], xi[2 * i + 1]);
-                                uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow) + 16 * c;
+                                uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(outp) + orow) + 16 * c;
                                 if (p.out_al32) {
                                     st_global_cs_v8(o, &w[0]);
                                     st_global_cs_v8(o + 8, &w[8]);
@@ -1156,7 +1196,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                         __stcs(reinterpret_cast<uint4 *>(o + 4 * q), make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
                                 }
                             } else {
-                                uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(p.out) + orow) + 32 * c;
+                                uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(outp) + orow) + 32 * c;
                                 if (p.out_al32) {
 #pragma unroll
                                     for (int q = 0; q < 4; ++q) st_global_cs_v8(o + 8 * q, &xi[8 * q]);
@@ -1184,7 +1224,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&cb->o_empty[bn & 1]);
                     if (r < valid) {
-                        uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(p.out) + orow);
+                        uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<__nv_bfloat16 *>(outp) + orow);
                         if (p.out_al32) {
 #pragma unroll
                             for (int q = 0; q < 8; ++q) st_global_cs_v8(o + 8 * q, &w[8 * q]);
@@ -1205,7 +1245,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                             if (lane == 0) mbar_arrive(&cb->o_empty[bn & 1]);
                         }
                         if (r < valid) {
-                            uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(p.out) + orow + hf * 64);
+                            uint32_t *o = reinterpret_cast<uint32_t *>(reinterpret_cast<float *>(outp) + orow + hf * 64);
                             if (p.out_al32) {
 #pragma unroll
                                 for (int q = 0; q < 8; ++q) st_global_cs_v8(o + 8 * q, &x[8 * q]);
@@ -1218,7 +1258,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                 }
             }
-            blk_n += nblk;
+            blk_n += SUBS * nblk;
         }
     } else {
         // ===== warps 10-13: segment hand-off (phase L), state snapshots, final state =====
@@ -1440,7 +1480,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     }
                 }
             }
-            blk_n += nblk;
+            blk_n += SUBS * nblk;  // (O buffers count sub-blocks)
             if (!ok) break;
         }
     }
