@@ -627,9 +627,9 @@ def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
     return {"workload": "prefill backward B=1 H=64 N=32768 d=128, bf16 dq/dk/dv + fp32 dS_in",
             "ms_per_call": ms, "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (dQ scan + paired dK/dV scan) + la_kv_aggregate_kernel (one sum)",
+                         "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (dQ sweep + reversed paired dK/dV sweep)",
                          "traffic": None, "bytes_per_launch": byts,
-                         "duration": "CUDA events around each la_prefill_backward call (about ten kernels)"}}
+                         "duration": "CUDA events around each la_prefill_backward call (two schedule kernels + two sweeps)"}}
 
 
 DATASHEET_HBM_GBS = 7700.0  # HGX B200 HBM3e datasheet figure (8000 on DGX), context only

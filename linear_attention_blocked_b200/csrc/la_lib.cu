@@ -165,7 +165,7 @@ la_status check_common(int H, int d, int block, la_dtype out_dtype) {
 }
 
 // The prefill kernel instantiation for a row-block length (0 = 128); with
-// mq2 (ANTI only), the paired instantiation that also runs (q2, v, k).
+// mq2, the paired reversed sweep that also runs (q2, v, k).
 template <bool ANTI, bool DECAY>
 la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                          const la::PrefillParams &pp, cudaStream_t stream, const CUtensorMap *mq2 = nullptr);
@@ -176,7 +176,8 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
                        const float *state_in, void *out, la_dtype out_dtype, float *state_out,
                        void *workspace, size_t ws_bytes, cudaStream_t stream,
                        const int *slots = nullptr, int n_slots = 0, bool anti = false,
-                       const float *decay = nullptr, const void *q2 = nullptr, void *out2 = nullptr) {
+                       const float *decay = nullptr, const void *q2 = nullptr, void *out2 = nullptr,
+                       bool rev = false) {
     la_status st = check_common(H, d, block, out_dtype);
     if (st != LA_OK) return st;
     if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
@@ -192,9 +193,10 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
         return LA_ERR_INVALID_ARGUMENT;
     if (decay && (anti || !aligned(decay, 4))) return LA_ERR_INVALID_ARGUMENT;
     if ((block == 64 || block == 256) && (anti || decay)) return LA_ERR_UNSUPPORTED;
-    // paired ANTI problems (q, k, v) and (q2, v, k): one bf16 state term only
-    if ((q2 != nullptr) != (out2 != nullptr)) return LA_ERR_INVALID_ARGUMENT;
-    if (q2 && (!anti || (block != 0 && block != la::BLK) || slots || state_out || max_seqlen > LA_LO_SPLIT_FROM))
+    // paired problems (q, k, v) and (q2, v, k) in a reversed sweep: one bf16
+    // state term only, so sequences of up to LA_LO_SPLIT_FROM tokens
+    if ((q2 != nullptr) != (out2 != nullptr) || (q2 != nullptr) != rev) return LA_ERR_INVALID_ARGUMENT;
+    if (q2 && (anti || decay || (block != 0 && block != la::BLK) || slots || max_seqlen > LA_LO_SPLIT_FROM))
         return LA_ERR_UNSUPPORTED;
     const size_t n_state = (size_t)(slots ? n_slots : nseq) * H * la::D * la::D * 4;
     if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
@@ -247,6 +249,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     sp.slots = slots;
     sp.n_slots = n_slots;
     sp.decay = decay;
+    sp.reverse = rev ? 1 : 0;
     sp.status = status;
     la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;
@@ -280,22 +283,22 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
 
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    st = anti ? launch_prefill<true, false>(block, grid, mq, mk, mv, pp, stream, q2 ? &mq2 : nullptr)
+    st = anti  ? launch_prefill<true, false>(block, grid, mq, mk, mv, pp, stream)
          : decay ? launch_prefill<false, true>(block, grid, mq, mk, mv, pp, stream)
-                 : launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream);
+                 : launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream, q2 ? &mq2 : nullptr);
     if (st != LA_OK) return st;
     ++g_launches;
     return LA_OK;
 }
 
-template <bool ANTI, bool DECAY, int BK, bool PAIR = false>
+template <bool ANTI, bool DECAY, int BK, bool PAIR = false, bool REV = false>
 la_status launch_prefill_bk(SmemAttr &attr, int grid, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, const la::PrefillParams &pp, cudaStream_t stream,
                             const CUtensorMap *mq2 = nullptr) {
-    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<ANTI, DECAY, BK, PAIR>, la::PREFILL_SMEM);
+    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<ANTI, DECAY, BK, PAIR, REV>, la::PREFILL_SMEM);
     if (st != LA_OK) return st;
     // (unpaired instantiations never read the fourth map)
-    la::la_prefill_kernel<ANTI, DECAY, BK, PAIR><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(
+    la::la_prefill_kernel<ANTI, DECAY, BK, PAIR, REV><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(
         mq, mk, mv, mq2 ? *mq2 : mq, pp);
     return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
@@ -303,8 +306,9 @@ la_status launch_prefill_bk(SmemAttr &attr, int grid, const CUtensorMap &mq, con
 template <bool ANTI, bool DECAY>
 la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                          const la::PrefillParams &pp, cudaStream_t stream, const CUtensorMap *mq2) {
-    if (ANTI && mq2)
-        return launch_prefill_bk<true, false, 128, true>(g_attr_prefill_pair, grid, mq, mk, mv, pp, stream, mq2);
+    if (!ANTI && !DECAY && mq2)  // the paired reversed sweep
+        return launch_prefill_bk<false, false, 128, true, true>(g_attr_prefill_pair, grid, mq, mk, mv, pp, stream,
+                                                               mq2);
     if (ANTI) return launch_prefill_bk<true, false, 128>(g_attr_prefill_anti, grid, mq, mk, mv, pp, stream);
     if (DECAY) return launch_prefill_bk<false, true, 128>(g_attr_prefill_decay, grid, mq, mk, mv, pp, stream);
     if (block == 64) return launch_prefill_bk<false, false, 64>(g_attr_prefill_b64, grid, mq, mk, mv, pp, stream);
@@ -824,35 +828,33 @@ la_status la_prefill_backward(const void *q, const void *k, const void *v, const
     st = prefill_impl(dout, v, k, nullptr, N, B, T, N, H, d, 0, state_in ? A : nullptr, dq, grad_dtype, nullptr,
                       ws_pre, pre_bytes, stream);
     if (st != LA_OK) return st;
-    // the two starting states: W_v = sum_t q_t^T g_t + G (= dS_in) and
-    // W_k = sum_t g_t^T q_t + G^T = W_v^T -- one sum over (q, dout) serves both
+    // dV and dK, sums over the later tokens:
+    //     dv_s = sum_{t >= s} (q_t . k_s) g_t + k_s G,   dk_s = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
+    // Up to LA_LO_SPLIT_FROM tokens: one reversed sweep of the paired problems
+    // (q, k, v) = (K, Q, dO) and (q2, v, k) = (V, dO, Q) from G, dK's state
+    // being dV's transposed; the sweep's final state G + sum_t q_t^T g_t is dS_in.
+    if (N <= LA_LO_SPLIT_FROM)
+        return prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, dstate_out, dv, grad_dtype, dstate_in, ws_pre,
+                            pre_bytes, stream, nullptr, 0, false, nullptr, v, dk, true);
+    // Longer sequences hand the state to the inter-block product as hi + lo,
+    // which the paired sweep does not: two ANTI scans, forward sweeps that
+    // start from the full sums W_v = sum_t q_t^T g_t + G (= dS_in) and
+    // W_k = W_v^T and remove each block's tokens after using them --
+    //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t,  dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t
+    // -- with one sum over (q, dout) for both.
     if ((st = la_kv_aggregate(q, dout, B, N, H, d, C, ws_agg, agg_bytes, stream)) != LA_OK) return st;
     const float *s0v = C;
     if (dstate_out) {
         if ((st = la_state_prefix(C, 1, dstate_out, Bs, (int)nstates, d, stream)) != LA_OK) return st;
         s0v = Bs;
     }
-    // dV: an ANTI scan of (q, k, v) = (K, Q, dO) from W_v
-    //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t = sum_{t >= s} (q_t . k_s) g_t + k_s G
-    // dK: an ANTI scan of (q, k, v) = (V, dO, Q) from W_k = W_v^T
-    //     dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
-    // Up to LA_LO_SPLIT_FROM tokens both run as one paired scan (dK as the
-    // second problem, its state the transpose of dV's); longer sequences hand
-    // the state to the inter-block product as hi + lo, which the paired scan
-    // does not, and run the two scans one after the other.
-    if (N <= LA_LO_SPLIT_FROM) {
-        st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
-                          stream, nullptr, 0, true, nullptr, v, dk);
-        if (st != LA_OK) return st;
-    } else {
-        if ((st = launch_transpose(s0v, A, nstates, stream)) != LA_OK) return st;
-        st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, A, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
-                          stream, nullptr, 0, true);
-        if (st != LA_OK) return st;
-        st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
-                          stream, nullptr, 0, true);
-        if (st != LA_OK) return st;
-    }
+    if ((st = launch_transpose(s0v, A, nstates, stream)) != LA_OK) return st;
+    st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, A, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
+                      stream, nullptr, 0, true);
+    if (st != LA_OK) return st;
+    st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
+                      stream, nullptr, 0, true);
+    if (st != LA_OK) return st;
     if (dstate_in) return la_state_prefix(nullptr, 0, s0v, dstate_in, (int)nstates, d, stream);
     return LA_OK;
 }
@@ -994,6 +996,7 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     sp.slots = nullptr;
     sp.n_slots = 0;
     sp.decay = nullptr;
+    sp.reverse = 0;
     sp.status = status;
     la::la_schedule_kernel<<<1, la::SCHED_THREADS, 0, stream>>>(sp);
     if (cudaGetLastError() != cudaSuccess) return LA_ERR_CUDA;

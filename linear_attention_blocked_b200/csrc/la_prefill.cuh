@@ -54,17 +54,25 @@
 // hi^T V + lo^T V.  The state warps rescale S by lambda^{nb} in TMEM when they
 // take each snapshot.  DECAY and ANTI are not combined.
 //
-// A third flag, PAIR (with ANTI, 128-row blocks and S as one bf16 term), runs
-// two ANTI problems that share their keys, values and state in one sweep:
-// problem 1 is (q, k, v) and problem 2 is (q2, v, k), whose state
-// sum v^T k is the transpose of problem 1's.  Each row block b becomes two
-// sub-blocks, u = 2b (problem 1) and u = 2b + 1 (problem 2), which take turns
-// in the score buffer, in the Q ring (q tile, then q2 tile) and in the two O
-// buffers (sub-block u in buffer u & 1; problem 1 writes `out`, problem 2
-// `out2`).  a5 of problem 2 reads the same state snapshot through K-major
-// descriptors, which present it transposed; a6 runs once per block.  With
-// (q, k, v, q2) = (K, Q, dO, V) the two outputs are the gradients dV and dK,
-// and Q and dO are read once for both.
+// REV makes the sweep run backwards: the scheduler lists each sequence's
+// segments from its end, every item visits its row blocks from the last, and
+// the mask keeps key t for row s iff t >= s, so from a state S_0 passed as
+// state_in
+//       o_s = q_s (S_0 + sum_{t >= s} k_t^T v_t)
+// with the final state S_0 + sum_t k_t^T v_t -- sums over later tokens from
+// a sweep that adds, where ANTI subtracts them from a full sum.
+//
+// PAIR (with REV or ANTI, 128-row blocks and S as one bf16 term) runs two
+// problems that share their keys, values and state in one sweep: problem 1
+// is (q, k, v) and problem 2 is (q2, v, k), whose state sum v^T k is the
+// transpose of problem 1's.  Each row block b becomes two sub-blocks, u = 2b
+// (problem 1) and u = 2b + 1 (problem 2), which take turns in the score
+// buffer, in the Q ring (q tile, then q2 tile) and in the two O buffers
+// (sub-block u in buffer u & 1; problem 1 writes `out`, problem 2 `out2`).
+// a5 of problem 2 reads the same state snapshot through K-major descriptors,
+// which present it transposed; a6 runs once per block.  With (q, k, v, q2) =
+// (K, Q, dO, V) in a reversed sweep the two outputs are the gradients dV and
+// dK, Q and dO are read once for both, and the final state is dS_in.
 //
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
@@ -414,6 +422,13 @@ __device__ __forceinline__ void scale_row_hi_lo(uint8_t *tile, uint8_t *lo_tile,
     }
 }
 
+// First row of the b-th row block a sweep visits in an item of nblk blocks
+// starting at tok0: in token order, or, for a reversed sweep, from the last.
+template <bool REV>
+__device__ __forceinline__ int block_row(int tok0, int nblk, int b) {
+    return tok0 + (REV ? nblk - 1 - b : b) * BLK;
+}
+
 // Every role reads the same item from the two-slot queue the producer fills.
 __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane, const PrefillParams &p,
                                           CtrlBlock *cb) {
@@ -427,14 +442,15 @@ __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane
     return item[IT_VALID] != 0;
 }
 
-template <bool ANTI, bool DECAY, int BK, bool PAIR = false>
+template <bool ANTI, bool DECAY, int BK, bool PAIR = false, bool REV = false>
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq2,
                   const __grid_constant__ PrefillParams p) {
     static_assert(BK == 64 || BK == 128 || BK == 256, "row blocks of 64, 128 or 256 tokens");
     static_assert(BK == 128 || (!ANTI && !DECAY), "64- and 256-row blocks: the plain forward only");
-    static_assert(!PAIR || (ANTI && !DECAY && BK == 128), "PAIR: two ANTI problems at 128-row blocks");
+    static_assert(!PAIR || ((ANTI || REV) && !DECAY && BK == 128), "PAIR: two ANTI or reversed problems, 128-row blocks");
+    static_assert(!REV || (!ANTI && !DECAY && BK == 128), "REV: the plain operation at 128-row blocks");
     constexpr bool B64 = BK == 64;  // two 64-row blocks per 128-row tile
     constexpr int SUBS = PAIR ? 2 : 1;  // sub-blocks per row block (PAIR: problem 1, problem 2)
     // BK == 256: one row block per pair of 128-row tiles (see the MMA warp)
@@ -523,7 +539,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const int jj = seg.w & (SEG_LAST - 1);
                     const long long seg_end = (long long)jj * p.seg_len + (seg.z - seg.y);
                     item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) |
-                                     ((ANTI ? (!PAIR && p.anti_lo != 0) : seg_end > LA_LO_SPLIT_FROM) ? ITF_LO : 0);
+                                     ((!PAIR && (ANTI ? p.anti_lo != 0 : seg_end > LA_LO_SPLIT_FROM)) ? ITF_LO : 0);
                 }
                 mbar_arrive(&cb->item_full[islot]);
                 ++it;
@@ -539,7 +555,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                         const int s = kv_n % KV_STAGES;
                         if (!wait_or_abort(&cb->kv_empty[s], ((kv_n / KV_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
                         mbar_expect_tx(&cb->kv_full[s], 2 * TILE_BYTES);
-                        const int row = tok0 + b * BLK;
+                        const int row = block_row<REV>(tok0, nblk, b);
                         tma_load_4d(smem + SM_K + s * TILE_BYTES, &tmk, &cb->kv_full[s], 0, h, row, 0, pol);
                         tma_load_4d(smem + SM_V + s * TILE_BYTES, &tmv, &cb->kv_full[s], 0, h, row, 0, pol);
                         kv_last_fill[s] = kv_n / KV_STAGES;
@@ -581,7 +597,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     if (!wait_or_abort(&cb->q_empty[qs], ((q_n / Q_STAGES) & 1) ^ 1, p, cb)) { ok = false; break; }
                     mbar_expect_tx(&cb->q_full[qs], TILE_BYTES);
                     tma_load_4d(smem + SM_Q + qs * TILE_BYTES, (PAIR && (u & 1)) ? &tmq2 : &tmq, &cb->q_full[qs], 0, h,
-                                tok0 + b * BLK, 0, pol_first);
+                                block_row<REV>(tok0, nblk, b), 0, pol_first);
                     q_last_fill[qs] = q_n / Q_STAGES;
                     ++q_n;
                 }
@@ -647,6 +663,23 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     if (DECAY) tc_commit_w(&cb->alo_free);  // every MMA so far has read the lo tile
                     if (!warp_wait(&cb->kv_full[s], (kv_n / KV_STAGES) & 1, p, cb)) { ok = false; break; }
                     if (DECAY && !warp_wait(&cb->alo_ready, a_n & 1, p, cb)) { ok = false; break; }
+                    if (REV) {
+                        // a reversed sweep starts at a sequence's last segment, which may
+                        // end inside its first tile and still has a successor: rows past
+                        // the sequence end (the next sequence's tokens) must add nothing
+                        // to A_j, so they are zeroed in the K tile (in token order only
+                        // full segments have successors)
+                        const int valid = min(BLK, tok1 - block_row<REV>(tok0, nblk, b));
+                        if (valid < BLK) {
+                            uint8_t *kp = smem + SM_K + s * TILE_BYTES;
+                            const int nbytes = (BLK - valid) * 128;
+                            for (int hh = 0; hh < 2; ++hh)
+                                for (int o = lane * 16; o < nbytes; o += 32 * 16)
+                                    *reinterpret_cast<uint4 *>(kp + hh * HALF_BYTES + valid * 128 + o) = make_uint4(0, 0, 0, 0);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                        }
+                    }
                     tc_fence_after();
                     const uint32_t kt = sbase + SM_K + s * TILE_BYTES;
                     const uint32_t vt = sbase + SM_V + s * TILE_BYTES;
@@ -972,7 +1005,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const int s = (kv0 + bi) % KV_STAGES;
                     const uint32_t kn = (kv0 + bi) / KV_STAGES, qn = q0 + i2;
                     if (ready(&cb->kv_full[s], kn & 1) && ready(&cb->q_full[qn % Q_STAGES], (qn / Q_STAGES) & 1)) {
-                        const int valid = min(BLK, tok1 - (tok0 + bi * BLK));
+                        const int valid = min(BLK, tok1 - block_row<REV>(tok0, nblk, bi));
                         if (valid < BLK && !second) {  // (PAIR: the first sub-block's a2 reads the tiles first)
                             // rows past the end of the sequence must add nothing to S or O:
                             // zero them in K and V (they may hold the next sequence's tokens)
@@ -1037,7 +1070,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int q4 = warp & 3;               // TMEM lane quarter this warp may access
         const int r = q4 * 32 + lane;          // tile row = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
-        constexpr int EXCL = ANTI ? 1 : 0;     // key s kept iff s + EXCL <= t
+        constexpr int EXCL = ANTI ? 1 : 0;     // key s kept iff s + EXCL <= t (REV: iff s >= t)
         uint32_t it = 0, blk_n = 0, kv_n = 0, q_n = 0, a_n = 0;
         bool ok = true;
         int item[8];
@@ -1082,9 +1115,10 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t x[64];
-                    if (!full && ((hf == 1 && q4 < 2) || (B64 && hf == 0 && q4 >= 2))) {
+                    if (!full && (REV ? (hf == 0 && q4 >= 2) : ((hf == 1 && q4 < 2) || (B64 && hf == 0 && q4 >= 2)))) {
                         // rows 0-63 see none of the keys 64-127; with 64-row blocks,
-                        // rows 64-127 (the second block) see none of the keys 0-63
+                        // rows 64-127 (the second block) see none of the keys 0-63;
+                        // reversed, rows 64-127 see none of the keys 0-63
 #pragma unroll
                         for (int w = 0; w < 32; ++w) x[w] = 0u;
                     } else {
@@ -1105,8 +1139,9 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                         for (int w = 0; w < 32; ++w) {
                             const int c = hf * 64 + 2 * w;
-                            x[w] = bf16x2_round(full || c + EXCL <= r ? x[2 * w] : 0u,
-                                                full || c + 1 + EXCL <= r ? x[2 * w + 1] : 0u);
+                            const bool k0 = REV ? c >= r : (full || c + EXCL <= r);
+                            const bool k1 = REV ? c + 1 >= r : (full || c + 1 + EXCL <= r);
+                            x[w] = bf16x2_round(k0 ? x[2 * w] : 0u, k1 ? x[2 * w + 1] : 0u);
                         }
                     }
                     tmem_st32(tsc + hf * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
@@ -1155,7 +1190,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 const int b = u / SUBS;
                 const uint32_t bn = blk_n + u;
                 void *const outp = (PAIR && (u & 1)) ? p.out2 : p.out;
-                const int row0 = tok0 + b * BLK;
+                const int row0 = block_row<REV>(tok0, nblk, b);
                 const int valid = min(BLK, tok1 - row0);
                 const uint32_t obuf = DECAY ? 0u : (bn & 1), opar = DECAY ? (bn & 1) : ((bn >> 1) & 1);
                 if (!warp_wait(&cb->o_full[obuf], opar, p, cb)) { ok = false; break; }
@@ -1511,6 +1546,7 @@ struct ScheduleParams {
     const int *slots;       // null, or [nseq] state slots in a pool of n_slots
     int n_slots;
     const float *decay;     // null, or [H] per-head decays, each must lie in (0, 1]
+    int reverse;            // list each sequence's segments from its end (reversed sweep)
     int *status;
 };
 
@@ -1580,7 +1616,8 @@ __global__ void __launch_bounds__(SCHED_THREADS, 1) la_schedule_kernel(const Sch
         __syncthreads();
         const int excl = carry_sh + x - nseg + ((tid >> 5) ? warp_sums[(tid >> 5) - 1] : 0);
         for (int jj = 0; jj < nseg; ++jj) {
-            const int t0 = a + jj * s.seg_len;
+            // jj: position in the sweep; reversed, the sweep starts at the last segment
+            const int t0 = a + (s.reverse ? nseg - 1 - jj : jj) * s.seg_len;
             const int t1 = min(t0 + s.seg_len, a + len);
             s.segs[excl + jj] = make_int4(i, t0, t1, jj | (jj == nseg - 1 ? SEG_LAST : 0));
         }
