@@ -628,7 +628,9 @@ def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
             "ms_per_call": ms, "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": gbs / hbm_peak, "kernel": "la_prefill_kernel (dQ sweep + reversed paired dK/dV sweep)",
-                         "traffic": None, "bytes_per_launch": byts,
+                         # DRAM bytes of both sweeps of one call
+                         "traffic": recorded_traffic("la_prefill_kernel", "backward_B1_H64_N32768"),
+                         "bytes_per_launch": byts,
                          "duration": "CUDA events around each la_prefill_backward call (two schedule kernels + two sweeps)"}}
 
 
@@ -759,7 +761,7 @@ def bench_prefill_decay(la, dev, stream, q, k, v, args, hbm_peak, world):
             "ms_per_call": ms, "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
                          "kernel": "la_prefill_kernel (decay)", "bytes_per_launch": byts,
-                         "traffic": None,
+                         "traffic": recorded_traffic("la_prefill_kernel", "prefill_decay_B1_H64_N32768"),
                          "duration": "CUDA events around each la_prefill_decay call (scheduler + prefill)"}}
 
 

@@ -344,14 +344,11 @@ LA_API la_status la_state_prefix(const float *parts, int count, const float *sta
  *   dv_s  = sum_{t >= s} (q_t . k_s) g_t + k_s G
  *   dS_in = sum_t q_t^T g_t + G
  *
- * computed as blocked sweeps: dq is a forward sweep of (dout, v, k) from
- * S_in^T; dv and dk, sums over the later tokens, are one reversed sweep
+ * computed as two blocked sweeps: dq is a forward sweep of (dout, v, k)
+ * from S_in^T; dv and dk, sums over the later tokens, are one reversed sweep
  * (segments and row blocks from the end of each sequence, the mask keeping
  * t >= s) of the paired problems (k, q, dout) and (v, dout, q) from G,
- * whose final state is dS_in.  Sequences longer than 32768 tokens take
- * instead one la_kv_aggregate for W_v = sum_t q_t^T g_t + G (= dS_in) and
- * two forward sweeps from W_v and W_k = W_v^T that remove the earlier
- * tokens as they go (an exclusive mask and a subtracted state update).
+ * whose final state is dS_in.
  *
  * q, k, v, dout: bf16 [B, N, H, d] contiguous (read only).  state_in,
  * dstate_out: fp32 [B, H, d, d] row-major or NULL (= 0).  dq, dk, dv: [B, N,
@@ -360,8 +357,8 @@ LA_API la_status la_state_prefix(const float *parts, int count, const float *sta
  * [B, H, d, d] or NULL (not computed).  workspace: at least
  * la_prefill_backward_workspace_size(B, N, H, d) bytes, 256-byte aligned,
  * caller-owned scratch.  fp32 accumulation on the tensor cores.  Enqueues
- * four kernels (five with a state_in; about a dozen past 32768 tokens) on `stream` and
- * returns; argument errors are
+ * four kernels (five with a state_in) on `stream` and returns; argument
+ * errors are
  * returned before any launch; device-side problems are reported by
  * la_get_device_status.
  * ------------------------------------------------------------------------- */

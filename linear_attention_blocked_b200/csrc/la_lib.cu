@@ -147,7 +147,7 @@ la_status ensure_smem_attr(SmemAttr &a, Kernel *kernel, int bytes) {
     return LA_OK;
 }
 
-SmemAttr g_attr_prefill, g_attr_prefill_anti, g_attr_prefill_pair, g_attr_prefill_decay, g_attr_prefill_b64,
+SmemAttr g_attr_prefill, g_attr_prefill_pair, g_attr_prefill_decay, g_attr_prefill_b64,
     g_attr_prefill_b256, g_attr_agg;
 
 bool ranges_overlap(const void *a, size_t na, const void *b, size_t nb) {
@@ -166,7 +166,7 @@ la_status check_common(int H, int d, int block, la_dtype out_dtype) {
 
 // The prefill kernel instantiation for a row-block length (0 = 128); with
 // mq2, the paired reversed sweep that also runs (q2, v, k).
-template <bool ANTI, bool DECAY>
+template <bool DECAY>
 la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                          const la::PrefillParams &pp, cudaStream_t stream, const CUtensorMap *mq2 = nullptr);
 
@@ -175,7 +175,7 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
                        int nseq, long long T, int max_seqlen, int H, int d, int block,
                        const float *state_in, void *out, la_dtype out_dtype, float *state_out,
                        void *workspace, size_t ws_bytes, cudaStream_t stream,
-                       const int *slots = nullptr, int n_slots = 0, bool anti = false,
+                       const int *slots = nullptr, int n_slots = 0,
                        const float *decay = nullptr, const void *q2 = nullptr, void *out2 = nullptr,
                        bool rev = false) {
     la_status st = check_common(H, d, block, out_dtype);
@@ -191,13 +191,11 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     const size_t n_in = (size_t)T * H * la::D * 2, n_out = (size_t)T * H * la::D * esz;
     if (slots && (n_slots <= 0 || !aligned(slots, 4) || state_in != state_out || !state_out))
         return LA_ERR_INVALID_ARGUMENT;
-    if (decay && (anti || !aligned(decay, 4))) return LA_ERR_INVALID_ARGUMENT;
-    if ((block == 64 || block == 256) && (anti || decay)) return LA_ERR_UNSUPPORTED;
-    // paired problems (q, k, v) and (q2, v, k) in a reversed sweep: one bf16
-    // state term only, so sequences of up to LA_LO_SPLIT_FROM tokens
+    if (decay && !aligned(decay, 4)) return LA_ERR_INVALID_ARGUMENT;
+    if ((block == 64 || block == 256) && decay) return LA_ERR_UNSUPPORTED;
+    // paired problems (q, k, v) and (q2, v, k) in a reversed sweep
     if ((q2 != nullptr) != (out2 != nullptr) || (q2 != nullptr) != rev) return LA_ERR_INVALID_ARGUMENT;
-    if (q2 && (anti || decay || (block != 0 && block != la::BLK) || slots || max_seqlen > LA_LO_SPLIT_FROM))
-        return LA_ERR_UNSUPPORTED;
+    if (q2 && (decay || (block != 0 && block != la::BLK) || slots)) return LA_ERR_UNSUPPORTED;
     const size_t n_state = (size_t)(slots ? n_slots : nseq) * H * la::D * la::D * 4;
     if (state_out && state_out != state_in && ranges_overlap(state_out, n_state, state_in, n_state))
         return LA_ERR_INVALID_ARGUMENT;
@@ -276,44 +274,40 @@ la_status prefill_impl(const void *q, const void *k, const void *v, const int *c
     pp.incl = reinterpret_cast<float *>(ws + w.incl);
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
-    pp.anti_lo = anti && max_seqlen > LA_LO_SPLIT_FROM;
     pp.decay = decay;
     pp.seg_len = L;
     pp.status = status;
 
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    st = anti  ? launch_prefill<true, false>(block, grid, mq, mk, mv, pp, stream)
-         : decay ? launch_prefill<false, true>(block, grid, mq, mk, mv, pp, stream)
-                 : launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream, q2 ? &mq2 : nullptr);
+    st = decay ? launch_prefill<true>(block, grid, mq, mk, mv, pp, stream)
+               : launch_prefill<false>(block, grid, mq, mk, mv, pp, stream, q2 ? &mq2 : nullptr);
     if (st != LA_OK) return st;
     ++g_launches;
     return LA_OK;
 }
 
-template <bool ANTI, bool DECAY, int BK, bool PAIR = false, bool REV = false>
+template <bool DECAY, int BK, bool PAIR = false, bool REV = false>
 la_status launch_prefill_bk(SmemAttr &attr, int grid, const CUtensorMap &mq, const CUtensorMap &mk,
                             const CUtensorMap &mv, const la::PrefillParams &pp, cudaStream_t stream,
                             const CUtensorMap *mq2 = nullptr) {
-    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<ANTI, DECAY, BK, PAIR, REV>, la::PREFILL_SMEM);
+    la_status st = ensure_smem_attr(attr, la::la_prefill_kernel<DECAY, BK, PAIR, REV>, la::PREFILL_SMEM);
     if (st != LA_OK) return st;
     // (unpaired instantiations never read the fourth map)
-    la::la_prefill_kernel<ANTI, DECAY, BK, PAIR, REV><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(
+    la::la_prefill_kernel<DECAY, BK, PAIR, REV><<<grid, la::PREFILL_THREADS, la::PREFILL_SMEM, stream>>>(
         mq, mk, mv, mq2 ? *mq2 : mq, pp);
     return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
-template <bool ANTI, bool DECAY>
+template <bool DECAY>
 la_status launch_prefill(int block, int grid, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                          const la::PrefillParams &pp, cudaStream_t stream, const CUtensorMap *mq2) {
-    if (!ANTI && !DECAY && mq2)  // the paired reversed sweep
-        return launch_prefill_bk<false, false, 128, true, true>(g_attr_prefill_pair, grid, mq, mk, mv, pp, stream,
-                                                               mq2);
-    if (ANTI) return launch_prefill_bk<true, false, 128>(g_attr_prefill_anti, grid, mq, mk, mv, pp, stream);
-    if (DECAY) return launch_prefill_bk<false, true, 128>(g_attr_prefill_decay, grid, mq, mk, mv, pp, stream);
-    if (block == 64) return launch_prefill_bk<false, false, 64>(g_attr_prefill_b64, grid, mq, mk, mv, pp, stream);
-    if (block == 256) return launch_prefill_bk<false, false, 256>(g_attr_prefill_b256, grid, mq, mk, mv, pp, stream);
-    return launch_prefill_bk<false, false, 128>(g_attr_prefill, grid, mq, mk, mv, pp, stream);
+    if (!DECAY && mq2)  // the paired reversed sweep
+        return launch_prefill_bk<false, 128, true, true>(g_attr_prefill_pair, grid, mq, mk, mv, pp, stream, mq2);
+    if (DECAY) return launch_prefill_bk<true, 128>(g_attr_prefill_decay, grid, mq, mk, mv, pp, stream);
+    if (block == 64) return launch_prefill_bk<false, 64>(g_attr_prefill_b64, grid, mq, mk, mv, pp, stream);
+    if (block == 256) return launch_prefill_bk<false, 256>(g_attr_prefill_b256, grid, mq, mk, mv, pp, stream);
+    return launch_prefill_bk<false, 128>(g_attr_prefill, grid, mq, mk, mv, pp, stream);
 }
 
 // Shared body of la_decode_step / la_decode_step_slots.
@@ -379,10 +373,10 @@ la_status launch_transpose(const float *in, float *out, long long nstates, cudaS
 }
 
 // Workspace of la_prefill_backward: one prefill workspace (reused by the
-// scans, which run in stream order), one la_kv_aggregate workspace and
-// three [B, H, D, D] fp32 states.
+// two sweeps, which run in stream order) and one [B, H, D, D] fp32 state
+// (S_in transposed).
 struct BwdLayout {
-    size_t prefill, agg, st0, st1, st2, total;
+    size_t prefill, st0, total;
 };
 
 BwdLayout bwd_layout(int B, int N, int H) {
@@ -390,14 +384,10 @@ BwdLayout bwd_layout(int B, int N, int H) {
     const long long T = (long long)B * N;
     const int L = choose_seg_len(B, T, H);
     const size_t pre = ws_layout(gmax_fixed(B, N, L), H).total;
-    const size_t agg = agg_ws_bytes(agg_plan((long long)B * H, N));
     const size_t st = (size_t)B * H * la::D * la::D * sizeof(float);
     w.prefill = 0;
-    w.agg = round_up(pre, 256);
-    w.st0 = w.agg + round_up(agg, 256);
-    w.st1 = w.st0 + round_up(st, 256);
-    w.st2 = w.st1 + round_up(st, 256);
-    w.total = w.st2 + st;
+    w.st0 = round_up(pre, 256);
+    w.total = w.st0 + st;
     return w;
 }
 
@@ -471,7 +461,7 @@ la_status la_prefill_decay(const void *q, const void *k, const void *v, int B, i
     if (B < 0 || N < 0 || !decay) return LA_ERR_INVALID_ARGUMENT;
     const long long T = (long long)B * N;
     return prefill_impl(q, k, v, nullptr, N, B, T, N, H, d, block, state_in, out, out_dtype, state_out,
-                        workspace, ws_bytes, stream, nullptr, 0, false, decay);
+                        workspace, ws_bytes, stream, nullptr, 0, decay);
 }
 
 la_status la_prefill_varlen_decay(const void *q, const void *k, const void *v, const int *cu_seqlens, int nseq,
@@ -481,7 +471,7 @@ la_status la_prefill_varlen_decay(const void *q, const void *k, const void *v, c
     if (!cu_seqlens || nseq < 0 || total_tokens < 0 || !decay) return LA_ERR_INVALID_ARGUMENT;
     if (!aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARGUMENT;
     return prefill_impl(q, k, v, cu_seqlens, 0, nseq, total_tokens, max_seqlen, H, d, block, state_in,
-                        out, out_dtype, state_out, workspace, ws_bytes, stream, nullptr, 0, false, decay);
+                        out, out_dtype, state_out, workspace, ws_bytes, stream, nullptr, 0, decay);
 }
 
 la_status la_decode_step_decay(const void *q, const void *k, const void *v, const float *decay, float *state,
@@ -814,15 +804,11 @@ la_status la_prefill_backward(const void *q, const void *k, const void *v, const
             return LA_ERR_INVALID_ARGUMENT;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     void *ws_pre = ws + w.prefill;
-    const size_t pre_bytes = w.agg - w.prefill;
-    void *ws_agg = ws + w.agg;
-    const size_t agg_bytes = w.st0 - w.agg;
+    const size_t pre_bytes = w.st0 - w.prefill;
     float *A = reinterpret_cast<float *>(ws + w.st0);
-    float *Bs = reinterpret_cast<float *>(ws + w.st1);
-    float *C = reinterpret_cast<float *>(ws + w.st2);
     const long long nstates = (long long)B * H;
 
-    // dQ: a forward scan of (q, k, v) = (dO, V, K) from S_in^T
+    // dQ: a forward sweep of (q, k, v) = (dO, V, K) from S_in^T
     //     dq_t = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T
     if (state_in && (st = launch_transpose(state_in, A, nstates, stream)) != LA_OK) return st;
     st = prefill_impl(dout, v, k, nullptr, N, B, T, N, H, d, 0, state_in ? A : nullptr, dq, grad_dtype, nullptr,
@@ -830,33 +816,11 @@ la_status la_prefill_backward(const void *q, const void *k, const void *v, const
     if (st != LA_OK) return st;
     // dV and dK, sums over the later tokens:
     //     dv_s = sum_{t >= s} (q_t . k_s) g_t + k_s G,   dk_s = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
-    // Up to LA_LO_SPLIT_FROM tokens: one reversed sweep of the paired problems
-    // (q, k, v) = (K, Q, dO) and (q2, v, k) = (V, dO, Q) from G, dK's state
-    // being dV's transposed; the sweep's final state G + sum_t q_t^T g_t is dS_in.
-    if (N <= LA_LO_SPLIT_FROM)
-        return prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, dstate_out, dv, grad_dtype, dstate_in, ws_pre,
-                            pre_bytes, stream, nullptr, 0, false, nullptr, v, dk, true);
-    // Longer sequences hand the state to the inter-block product as hi + lo,
-    // which the paired sweep does not: two ANTI scans, forward sweeps that
-    // start from the full sums W_v = sum_t q_t^T g_t + G (= dS_in) and
-    // W_k = W_v^T and remove each block's tokens after using them --
-    //     dv_s = k_s W_v - sum_{t < s} (k_s . q_t) g_t,  dk_s = v_s W_k - sum_{t < s} (v_s . g_t) q_t
-    // -- with one sum over (q, dout) for both.
-    if ((st = la_kv_aggregate(q, dout, B, N, H, d, C, ws_agg, agg_bytes, stream)) != LA_OK) return st;
-    const float *s0v = C;
-    if (dstate_out) {
-        if ((st = la_state_prefix(C, 1, dstate_out, Bs, (int)nstates, d, stream)) != LA_OK) return st;
-        s0v = Bs;
-    }
-    if ((st = launch_transpose(s0v, A, nstates, stream)) != LA_OK) return st;
-    st = prefill_impl(v, dout, q, nullptr, N, B, T, N, H, d, 0, A, dk, grad_dtype, nullptr, ws_pre, pre_bytes,
-                      stream, nullptr, 0, true);
-    if (st != LA_OK) return st;
-    st = prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, s0v, dv, grad_dtype, nullptr, ws_pre, pre_bytes,
-                      stream, nullptr, 0, true);
-    if (st != LA_OK) return st;
-    if (dstate_in) return la_state_prefix(nullptr, 0, s0v, dstate_in, (int)nstates, d, stream);
-    return LA_OK;
+    // one reversed sweep of the paired problems (q, k, v) = (K, Q, dO) and
+    // (q2, v, k) = (V, dO, Q) from G, dK's state being dV's transposed; the
+    // sweep's final state G + sum_t q_t^T g_t is dS_in.
+    return prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, dstate_out, dv, grad_dtype, dstate_in, ws_pre,
+                        pre_bytes, stream, nullptr, 0, nullptr, v, dk, true);
 }
 
 la_status la_state_prefix(const float *parts, int count, const float *state_in, float *out, int nstates, int d,
@@ -1022,13 +986,12 @@ extern "C" la_status la_prefill_noalloc(const void *q, const void *k, const void
     pp.incl = reinterpret_cast<float *>(ws + w.incl);
     pp.wait_limit_ns = g_wait_limit_ns.load();
     pp.inject = g_inject.load();
-    pp.anti_lo = 0;
     pp.decay = nullptr;
     pp.seg_len = L;
     pp.status = status;
     const long long items = gmax * (long long)H;
     const int grid = (int)(items < device_sm_count() ? items : device_sm_count());
-    st = launch_prefill<false, false>(block, grid, mq, mk, mv, pp, stream);
+    st = launch_prefill<false>(block, grid, mq, mk, mv, pp, stream);
     if (st != LA_OK) return st;
     ++g_launches;
     return LA_OK;

@@ -21,20 +21,7 @@
 //       out = O (bf16 or fp32)             a7
 //   and, for the last segment, the final state S goes to state_out.
 //
-// The kernel is a template on ANTI.  ANTI = false is the operation above.
-// ANTI = true computes, from a state S_0 passed as state_in,
-//       o_t = q_t (S_0 - sum_{s < t} k_s^T v_s)
-//           = q_t S_0 - sum_{s < t} (q_t . k_s) v_s
-// -- an exclusive mask (s < t) and the V operand negated in a4, a6 and
-// phase A (bit 14 of the MMA instruction descriptor) -- which is how the
-// gradients dK and dV, sums over later tokens, are formed in one forward
-// sweep: with S_0 the sum over all tokens, S_0 minus the earlier tokens
-// leaves the later ones.  S starts at the sum over the whole sequence, as
-// large as the forward's state at its end, so ANTI hands S to a5 as hi + lo
-// exactly when the forward would need it somewhere in the sequence: when the
-// host sets p.anti_lo (sequences longer than LA_LO_SPLIT_FROM tokens).
-//
-// A second template flag, DECAY, adds a per-head decay lambda_h in (0, 1]
+// The kernel is a template.  DECAY adds a per-head decay lambda_h in (0, 1]
 // (the "decay value computation" of "MiniMax-01技术报告解读" §3.3 item 1, read
 // as the decayed recurrence S_t = lambda S_{t-1} + k_t^T v_t, o_t = q_t S_t).
 // With r the row in a block of nb rows:
@@ -52,7 +39,7 @@
 // the scores have read it, lo into the block's Q slot once a5 has read it (in
 // phase A: into the snapshot buffer, idle there), and a6 is the two products
 // hi^T V + lo^T V.  The state warps rescale S by lambda^{nb} in TMEM when they
-// take each snapshot.  DECAY and ANTI are not combined.
+// take each snapshot.
 //
 // REV makes the sweep run backwards: the scheduler lists each sequence's
 // segments from its end, every item visits its row blocks from the last, and
@@ -60,19 +47,20 @@
 // state_in
 //       o_s = q_s (S_0 + sum_{t >= s} k_t^T v_t)
 // with the final state S_0 + sum_t k_t^T v_t -- sums over later tokens from
-// a sweep that adds, where ANTI subtracts them from a full sum.
+// a sweep that adds.
 //
-// PAIR (with REV or ANTI, 128-row blocks and S as one bf16 term) runs two
-// problems that share their keys, values and state in one sweep: problem 1
-// is (q, k, v) and problem 2 is (q2, v, k), whose state sum v^T k is the
-// transpose of problem 1's.  Each row block b becomes two sub-blocks, u = 2b
-// (problem 1) and u = 2b + 1 (problem 2), which take turns in the score
-// buffer, in the Q ring (q tile, then q2 tile) and in the two O buffers
-// (sub-block u in buffer u & 1; problem 1 writes `out`, problem 2 `out2`).
-// a5 of problem 2 reads the same state snapshot through K-major descriptors,
-// which present it transposed; a6 runs once per block.  With (q, k, v, q2) =
-// (K, Q, dO, V) in a reversed sweep the two outputs are the gradients dV and
-// dK, Q and dO are read once for both, and the final state is dS_in.
+// PAIR (with REV) runs two problems that share their keys, values and state
+// in one sweep: problem 1 is (q, k, v) and problem 2 is (q2, v, k), whose
+// state sum v^T k is the transpose of problem 1's.  Each row block b becomes
+// two sub-blocks, u = 2b (problem 1) and u = 2b + 1 (problem 2), which take
+// turns in the score buffer, in the Q ring (q tile, then q2 tile) and in the
+// two O buffers (sub-block u in buffer u & 1; problem 1 writes `out`, problem
+// 2 `out2`).  a5 of problem 2 reads the same state snapshot through K-major
+// descriptors, which present it transposed (with S as hi + lo, the snapshot
+// holds one column half at a time, and both problems read each half before
+// it is released); a6 runs once per block.  With (q, k, v, q2) = (K, Q, dO,
+// V) the two outputs are the gradients dV and dK, Q and dO are read once for
+// both, and the final state is dS_in.
 //
 // Warp roles (448 threads):
 //   warp 0      TMA producers: lane 0 takes tickets and loads K and V, lane 1
@@ -169,7 +157,6 @@ struct PrefillParams {
     int seg_len;            // tokens per segment (the last one of a sequence may be shorter)
     unsigned long long wait_limit_ns;
     int inject;
-    int anti_lo;            // ANTI: hand S to a5 as hi + lo (the sequences are long)
     const float *decay;     // DECAY: lambda_h per head, [H] (validated by the scheduler)
     int *status;            // sticky device status word
 };
@@ -442,15 +429,15 @@ __device__ __forceinline__ bool next_item(uint32_t &it, int (&item)[8], int lane
     return item[IT_VALID] != 0;
 }
 
-template <bool ANTI, bool DECAY, int BK, bool PAIR = false, bool REV = false>
+template <bool DECAY, int BK, bool PAIR = false, bool REV = false>
 __global__ void __launch_bounds__(PREFILL_THREADS, 1)
 la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmq2,
                   const __grid_constant__ PrefillParams p) {
     static_assert(BK == 64 || BK == 128 || BK == 256, "row blocks of 64, 128 or 256 tokens");
-    static_assert(BK == 128 || (!ANTI && !DECAY), "64- and 256-row blocks: the plain forward only");
-    static_assert(!PAIR || ((ANTI || REV) && !DECAY && BK == 128), "PAIR: two ANTI or reversed problems, 128-row blocks");
-    static_assert(!REV || (!ANTI && !DECAY && BK == 128), "REV: the plain operation at 128-row blocks");
+    static_assert(BK == 128 || !DECAY, "64- and 256-row blocks: the plain forward only");
+    static_assert(!PAIR || REV, "PAIR: two problems in a reversed sweep");
+    static_assert(!REV || (!DECAY && BK == 128), "REV: the plain operation at 128-row blocks");
     constexpr bool B64 = BK == 64;  // two 64-row blocks per 128-row tile
     constexpr int SUBS = PAIR ? 2 : 1;  // sub-blocks per row block (PAIR: problem 1, problem 2)
     // BK == 256: one row block per pair of 128-row tiles (see the MMA warp)
@@ -539,7 +526,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                     const int jj = seg.w & (SEG_LAST - 1);
                     const long long seg_end = (long long)jj * p.seg_len + (seg.z - seg.y);
                     item[IT_FLAGS] = ((seg.w & SEG_LAST) ? ITF_LAST : 0) |
-                                     ((!PAIR && (ANTI ? p.anti_lo != 0 : seg_end > LA_LO_SPLIT_FROM)) ? ITF_LO : 0);
+                                     (seg_end > LA_LO_SPLIT_FROM ? ITF_LO : 0);
                 }
                 mbar_arrive(&cb->item_full[islot]);
                 ++it;
@@ -627,9 +614,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         constexpr uint32_t ID_QK = idesc_bf16_f32(BLK, BLK, 0, 0);    // Q (K-major) x K (K-major)
         constexpr uint32_t ID_QS = idesc_bf16_f32(BLK, D / 2, 0, 1);  // Q (K-major) x S half (MN-major)
         constexpr uint32_t ID_QF = idesc_bf16_f32(BLK, D, 0, 1);      // Q (K-major) x S (MN-major)
-        constexpr uint32_t NEG_V = ANTI ? IDESC_NEGATE_B : 0u;        // ANTI: the V operand negated
-        constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1) | NEG_V;  // K^T (MN) x V (MN)
-        constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1) | NEG_V;  // P (TMEM) x V (MN)
+        constexpr uint32_t ID_KV = idesc_bf16_f32(D, D, 1, 1);  // K^T (MN) x V (MN)
+        constexpr uint32_t ID_PV = idesc_bf16_f32(BLK, D, 0, 1);  // P (TMEM) x V (MN)
         // The whole warp runs this loop in step: every lane holds the same
         // counters, barrier probes are combined with __all_sync, and each MMA or
         // commit is issued by the lane that elect.sync picks.
@@ -907,12 +893,20 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                 // DECAY: a5 goes to O buffer 1 and a6 waits for the scaled keys
                 // PAIR: the second sub-block reads the snapshot the first one waited
                 // for (released after both), into the other O buffer
+                // PAIR with S as hi + lo: the snapshot holds one column half at a
+                // time, which both problems read before it is released, so a5 of
+                // the two sub-blocks runs as one step per half (both O buffers
+                // free, the second q tile landed; i5 advances by two)
+                const bool pair_lo = PAIR && lo;
                 if (i5 < i2) {
                     const uint32_t bn = blk0 + i5;
-                    const bool second = PAIR && (i5 & 1);
+                    const bool second = PAIR && (i5 & 1);  // (never with pair_lo)
                     const bool a_read = last || i5 > 0 || ready(&cb->a_free, afree_n & 1);
+                    const uint32_t qn2 = q0 + i5 + 1;     // pair_lo: the second sub-block's q tile
                     if (a_read && (second || ready(&cb->snap_full, snap_n & 1)) &&
-                        ready(&cb->o_empty[ob(bn)], obpar(bn) ^ 1)) {
+                        ready(&cb->o_empty[ob(bn)], obpar(bn) ^ 1) &&
+                        (!pair_lo || (ready(&cb->o_empty[ob(bn + 1)], obpar(bn + 1) ^ 1) &&
+                                      ready(&cb->q_full[qn2 % Q_STAGES], (qn2 / Q_STAGES) & 1)))) {
                         tc_fence_after();
                         const int bi = i5 / SUBS;  // row block
                         const int s = (kv0 + bi) % KV_STAGES;
@@ -961,8 +955,21 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                 else
                                     mma_ss_w(to, desc_kmajor(qt, kk), desc_mnmajor(sl, kk), ID_QS, 1u);
                             }
+                            if (pair_lo) {
+                                // problem 2: O2 += Q2[:, half ch] (S_hi + S_lo)^T[half ch, :] --
+                                // the half read K-major is rows 64 ch .. 64 ch + 63 of S^T
+                                const uint32_t tq2 = tmem + TM_O + ob(bn + 1) * 128;
+                                const uint32_t qt2 = sbase + SM_Q + (qn2 % Q_STAGES) * TILE_BYTES;
+#pragma unroll
+                                for (int kk = 0; kk < D / 32; ++kk)
+                                    mma_ss_w(tq2, desc_kmajor(qt2, 4 * ch + kk), desc_kmajor(sh, kk), ID_QK,
+                                             (ch > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+                                for (int kk = 0; kk < D / 32; ++kk)
+                                    mma_ss_w(tq2, desc_kmajor(qt2, 4 * ch + kk), desc_kmajor(sl, kk), ID_QK, 1u);
+                            }
                         }
-                        if (!PAIR || second) {
+                        if (!PAIR || second || pair_lo) {  // every reader of this snapshot (half) is issued
                             tc_commit_w(&cb->snap_empty);
                             ++snap_n;
                         }
@@ -991,7 +998,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                                     tc_commit_w(&cb->s_done);
                                 }
                             }
-                            ++i5;
+                            i5 += pair_lo ? 2 : 1;  // (pair_lo: the second q tile is released after its a2)
                         }
                         sub = tile_done ? 0 : sub + 1;
                         prog = true;
@@ -1028,6 +1035,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
                             mma_ss_w(tmem + TM_SC, desc_kmajor(qt, kk), desc_kmajor(kt, kk), ID_QK,
                                      kk > 0 ? 1u : 0u);
                         tc_commit_w(&cb->sc_full);
+                        if (PAIR && lo && second) tc_commit_w(&cb->q_empty[qn % Q_STAGES]);  // its a5 came first
                         ++i2;
                         prog = true;
                     }
@@ -1070,7 +1078,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
         const int q4 = warp & 3;               // TMEM lane quarter this warp may access
         const int r = q4 * 32 + lane;          // tile row = TMEM lane
         const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
-        constexpr int EXCL = ANTI ? 1 : 0;     // key s kept iff s + EXCL <= t (REV: iff s >= t)
+        // key s kept for row t iff s <= t (REV: iff s >= t)
         uint32_t it = 0, blk_n = 0, kv_n = 0, q_n = 0, a_n = 0;
         bool ok = true;
         int item[8];
@@ -1082,14 +1090,15 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             const float lam = DECAY ? exp2f(l2) : 1.f;
             if (DECAY && !last) {
                 // phase A: scale each K tile's rows to the segment end, row r of
-                // block b by lambda^{len-1-128b-r}, hi in place, lo into the
-                // snapshot buffer (free: every MMA that read it has completed)
+                // the block starting at token t0 by lambda^{tok1-1-t0-r}, hi in
+                // place, lo into the snapshot buffer (free: every MMA that read it
+                // has completed)
                 for (int b = 0; b < nblk; ++b) {
                     const int s = kv_n % KV_STAGES;
                     if (!warp_wait(&cb->alo_free, a_n & 1, p, cb)) { ok = false; break; }
                     if (!warp_wait(&cb->kv_full[s], (kv_n / KV_STAGES) & 1, p, cb)) { ok = false; break; }
                     scale_row_hi_lo(smem + SM_K + s * TILE_BYTES, smem + SM_SHI, r,
-                                    decay_pow(l2, (tok1 - tok0) - 1 - b * BLK - r));
+                                    decay_pow(l2, tok1 - 1 - block_row<REV>(tok0, nblk, b) - r));
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&cb->alo_ready);
@@ -1105,7 +1114,7 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
             // (PAIR: two per block, one per problem, the same mask)
             const int nsteps = BK == 256 ? 3 * (nblk / 2) + (nblk & 1) : SUBS * nblk;
             for (int b = 0; b < nsteps; ++b) {
-                // P = bf16(Sc ⊙ M), inclusive mask (exclusive under ANTI), packed
+                // P = bf16(Sc ⊙ M), inclusive mask, packed
                 // two per 32-bit column over the first 64 score columns
                 // (DECAY: P = bf16(Sc lambda^{r-c}) for c <= r)
                 const uint32_t bn = blk_n + b, tsc = trow + TM_SC;
@@ -1139,8 +1148,8 @@ la_prefill_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant
 #pragma unroll
                         for (int w = 0; w < 32; ++w) {
                             const int c = hf * 64 + 2 * w;
-                            const bool k0 = REV ? c >= r : (full || c + EXCL <= r);
-                            const bool k1 = REV ? c + 1 >= r : (full || c + 1 + EXCL <= r);
+                            const bool k0 = REV ? c >= r : (full || c <= r);
+                            const bool k1 = REV ? c + 1 >= r : (full || c + 1 <= r);
                             x[w] = bf16x2_round(k0 ? x[2 * w] : 0u, k1 ? x[2 * w + 1] : 0u);
                         }
                     }

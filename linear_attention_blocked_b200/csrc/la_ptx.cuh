@@ -392,9 +392,6 @@ __host__ __device__ constexpr uint64_t smem_desc_sw128(uint32_t saddr, uint32_t 
 //   bits 4-5 D format (1 = f32), bits 7-9 A format (1 = bf16), bits 10-12 B
 //   format (1 = bf16), bit 15 A major (0 = K, 1 = MN), bit 16 B major,
 //   bits 17-22 N >> 3, bits 24-28 M >> 4.
-// bit 14 of the same descriptor: negate the B operand (D (+)= A * (-B))
-constexpr uint32_t IDESC_NEGATE_B = 1u << 14;
-
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, uint32_t a_mn_major,
                                                       uint32_t b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | (a_mn_major << 15) | (b_mn_major << 16) |

@@ -235,7 +235,7 @@ def test_backward_argument_errors(L):
     q, k, v, g = (V(base + i * n) for i in range(4))
     dq, dk, dv = (V(base + (4 + i) * n) for i in range(3))
     ws_size = L.la_prefill_backward_workspace_size(B, N, H, 128)
-    assert ws_size >= L.la_prefill_workspace_size(B, N, H, 128, 0) + 3 * B * H * 128 * 128 * 4
+    assert ws_size >= L.la_prefill_workspace_size(B, N, H, 128, 0) + B * H * 128 * 128 * 4  # + S_in transposed
     ws = V(base + 64 * n)
     args = lambda **kw: dict(dict(q=q, k=k, v=v, g=g, B=B, N=N, H=H, d=128, sin=None, dsout=None, dq=dq, dk=dk,
                                   dv=dv, gd=0, dsin=None, ws=ws, wsb=ws_size, s=None), **kw)

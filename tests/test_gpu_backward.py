@@ -2,9 +2,10 @@
 the fp64 oracle's gradients, element by element, on seeded inputs: ragged
 tails, several cross-SM segments, carried-in states and state gradients, bf16
 and fp32 gradients, sampled heads at 4096 tokens, and at the single-sequence
-prefill workload (B=1, H=64, N=32768) and at 131072 tokens the first and
-last rows of sampled heads, with the rest of the sequence summarised by the
-oracle's forward."""
+prefill workload (B=1, H=64, N=32768) and at 131072 tokens windows of rows
+of sampled heads (the first, the last, and one across the point where the
+reversed sweep switches its state to bf16 hi + lo), with the rest of the
+sequence summarised by the oracle's forward."""
 import numpy as np
 import pytest
 import torch
@@ -75,45 +76,38 @@ def test_backward_bf16_sampled_heads(oracle_mod):
     _check_all(got, ref, B, N, len(heads), True, "bf16 sampled heads")
 
 
-@pytest.mark.parametrize("N,H,heads,R", [(32768, 64, [0, 37], 4096), (131072, 2, [0, 1], 2048)])
-def test_backward_long_sequence_sampled_rows(oracle_mod, N, H, heads, R):
+@pytest.mark.parametrize("N,H,heads,R,mid", [(32768, 64, [0, 37], 4096, None), (131072, 2, [0, 1], 2048, 98304)])
+def test_backward_long_sequence_sampled_rows(oracle_mod, N, H, heads, R, mid):
     """B=1 and N=32768, H=64 (the single-sequence prefill workload) or
-    N=131072, H=2 (past the length where the scans split their state into
-    bf16 hi + lo): bf16 gradients of the sampled heads on the first and the
-    last R rows against the oracle.  The rows' gradients depend on the rest
-    of the sequence only through d x d sums, which the oracle's forward
-    supplies:
-      first rows: dk_s, dv_s also see the later tokens t >= R, whose share is
-        v_s G^T and k_s G with G = sum_{t >= R} q_t^T g_t -- the oracle's
-        state from zero over those tokens with (k, v) = (q, g) -- passed to
-        the oracle's backward of the first rows as dS_out;
-      last rows: dq_t also sees the earlier tokens through S_in = their k^T v
-        sum, the oracle's final state over them.
-    dS_in = sum_t q_t^T g_t: against the oracle on the sampled heads; past
-    32768 tokens it is la_kv_aggregate(q, dout) bit for bit (the ANTI scans
-    start from that sum), up to 32768 the reversed sweep's own final state."""
+    N=131072, H=2 (long enough for the reversed sweep to switch its state to
+    bf16 hi + lo, at token 98304 with 4096-token segments): bf16 gradients of
+    the sampled heads on windows of R rows -- the first, the last and, at
+    131072 tokens, one straddling that switch -- against the oracle.  A
+    window [a, b) sees the rest of the sequence only through d x d sums,
+    which the oracle's forward supplies: S_in = sum_{t < a} k_t^T v_t (its
+    final state over the earlier tokens) for dq, and dS_out = sum_{t >= b}
+    q_t^T g_t (its final state with (k, v) = (q, g) over the later tokens)
+    for dk and dv.  dS_in = sum_t q_t^T g_t, the reversed sweep's final
+    state: against the oracle on the sampled heads and against
+    la_kv_aggregate(q, dout) on all."""
     B = 1
     q, k, v, g = _inputs(B, N, H, seed=960 + H)
     dq, dk, dv, dsin = la.prefill_backward(q, k, v, g)
     assert la.get_device_status() == la.LA_OK
-    agg = la.kv_aggregate(q, g)
-    if N > 32768:
-        assert torch.equal(dsin, agg)
-    else:
-        check_state(to_np(dsin), to_np(agg), what=f"N={N} dS_in vs la_kv_aggregate")
+    check_state(to_np(dsin), to_np(la.kv_aggregate(q, g)), what=f"N={N} dS_in vs la_kv_aggregate")
     bits = lambda t, a, b: la_inputs.bits(t[0, a:b])  # noqa: E731
     cu = lambda n: np.array([0, n], np.int32)  # noqa: E731
     _, W = oracle_mod.recurrent(bits(q, 0, N), bits(q, 0, N), bits(g, 0, N), cu(N), heads=heads)
     check_state(to_np(dsin[0, heads]), W[0], what=f"N={N} dS_in vs oracle")
-    # first rows
-    _, G = oracle_mod.recurrent(bits(q, R, N), bits(q, R, N), bits(g, R, N), cu(N - R), heads=heads)
-    ref = oracle_mod.backward(bits(q, 0, R), bits(k, 0, R), bits(v, 0, R), bits(g, 0, R), cu(R), heads=heads,
-                              dstate_out=G)
-    for name, x, y in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
-        check_out(to_np(x[0, :R, heads]), y, bf16_out=True, what=f"N={N} first rows {name}")
-    # last rows
-    _, S = oracle_mod.recurrent(bits(q, 0, N - R), bits(k, 0, N - R), bits(v, 0, N - R), cu(N - R), heads=heads)
-    ref = oracle_mod.backward(bits(q, N - R, N), bits(k, N - R, N), bits(v, N - R, N), bits(g, N - R, N), cu(R),
-                              heads=heads, state_in=S)
-    for name, x, y in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
-        check_out(to_np(x[0, N - R:, heads]), y, bf16_out=True, what=f"N={N} last rows {name}")
+    windows = [(0, R), (N - R, N)] + ([(mid - R // 2, mid + R // 2)] if mid else [])
+    for a, b in windows:
+        S = None
+        if a > 0:
+            _, S = oracle_mod.recurrent(bits(q, 0, a), bits(k, 0, a), bits(v, 0, a), cu(a), heads=heads)
+        G = None
+        if b < N:
+            _, G = oracle_mod.recurrent(bits(q, b, N), bits(q, b, N), bits(g, b, N), cu(N - b), heads=heads)
+        ref = oracle_mod.backward(bits(q, a, b), bits(k, a, b), bits(v, a, b), bits(g, a, b), cu(b - a),
+                                  heads=heads, state_in=S, dstate_out=G)
+        for name, x, y in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
+            check_out(to_np(x[0, a:b, heads]), y, bf16_out=True, what=f"N={N} rows {a}-{b} {name}")
