@@ -371,6 +371,27 @@ LA_API la_status la_prefill_backward(const void *q, const void *k, const void *v
                                      float *dstate_in, void *workspace, size_t ws_bytes,
                                      cudaStream_t stream);
 
+/* la_prefill_backward_varlen: the gradients of la_prefill_varlen -- the
+ * same derivatives for every sequence of a packed batch (the pages train on
+ * packed sequences: "MiniMax-01技术报告解读" §3.2 item 1).  q, k, v, dout,
+ * dq, dk, dv: [total_tokens, H, d]; cu_seqlens: device int32 [nseq + 1],
+ * validated on the device as for la_prefill_varlen (an invalid table sets
+ * LA_ERR_INVALID_ARGUMENT in the device word and computes nothing);
+ * state_in, dstate_out, dstate_in: fp32 [nseq, H, d, d] or NULL.  The
+ * gradients of an empty sequence are empty and its dS_in is its dS_out.
+ * Workspace: la_prefill_backward_varlen_workspace_size bytes, 256-byte
+ * aligned.  Otherwise as la_prefill_backward. */
+LA_API size_t la_prefill_backward_varlen_workspace_size(int nseq, int total_tokens, int max_seqlen,
+                                                        int H, int d);
+
+LA_API la_status la_prefill_backward_varlen(const void *q, const void *k, const void *v,
+                                            const void *dout, const int *cu_seqlens, int nseq,
+                                            int total_tokens, int max_seqlen, int H, int d,
+                                            const float *state_in, const float *dstate_out,
+                                            void *dq, void *dk, void *dv, la_dtype grad_dtype,
+                                            float *dstate_in, void *workspace, size_t ws_bytes,
+                                            cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Status.
  * la_get_device_status synchronises `stream`, then returns and clears the

@@ -19,11 +19,13 @@ ABI (include/lightning_attn.h).  Entry points:
   lasp_prefill_varlen(q, k, v, cu, bounds)   the same for a packed batch cut at any token
   lasp_prefill_backward(q, k, v, dout, ...)  gradients of lasp_prefill across ranks
   prefill_backward(q, k, v, dout, ...)       la_prefill_backward: dq, dk, dv, dS_in
+  prefill_backward_varlen(q, k, v, dout, cu, ...)  la_prefill_backward_varlen: the same per packed sequence
   prefill_from_host(q, k, v, ...)            la_prefill of pinned host tensors, chunks pipelined
                                              over copy-in / scan / copy-out streams
   get_device_status()                        la_get_device_status
 """
-from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, prefill_backward, EXPORTED, LA_BF16, LA_ERR_CUDA,  # noqa: F401
+from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, backward_varlen_workspace_size,  # noqa: F401
+                       prefill_backward, prefill_backward_varlen, EXPORTED, LA_BF16, LA_ERR_CUDA,
                        LA_ERR_INVALID_ARGUMENT, LA_ERR_TIMEOUT, LA_ERR_UNSUPPORTED,
                        LA_ERR_WORKSPACE, LA_FP32, LA_INJECT_NONE, LA_INJECT_SKIP_PUBLISH, LA_OK,
                        LAError, debug_inject, decode_step, decode_step_slots, get_device_status,

@@ -28,7 +28,7 @@ EXPORTED = ("la_prefill_workspace_size", "la_prefill", "la_prefill_varlen_worksp
             "la_kv_aggregate_workspace_size", "la_kv_aggregate", "la_state_prefix",
             "la_prefill_backward_workspace_size", "la_prefill_backward", "la_prefill_decay",
             "la_prefill_varlen_decay", "la_decode_step_decay", "la_prefill_from_host_buffer_size",
-            "la_prefill_from_host")
+            "la_prefill_from_host", "la_prefill_backward_varlen_workspace_size", "la_prefill_backward_varlen")
 
 
 class LAError(RuntimeError):
@@ -101,6 +101,11 @@ def lib():
         L.la_prefill_backward.argtypes = [vp, vp, vp, vp, c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, c_int, vp,
                                           vp, sz, vp]
         L.la_prefill_backward.restype = c_int
+        L.la_prefill_backward_varlen_workspace_size.argtypes = [c_int] * 5
+        L.la_prefill_backward_varlen_workspace_size.restype = sz
+        L.la_prefill_backward_varlen.argtypes = [vp, vp, vp, vp, vp, c_int, c_int, c_int, c_int, c_int, vp, vp, vp,
+                                                 vp, vp, c_int, vp, vp, sz, vp]
+        L.la_prefill_backward_varlen.restype = c_int
         L.la_get_device_status.argtypes = [vp]
         L.la_get_device_status.restype = c_int
         L.la_status_string.argtypes = [c_int]
@@ -466,6 +471,49 @@ def prefill_backward(q, k, v, dout, state_in=None, dstate_out=None, grad_dtype=t
                                    _out_code(grads[0].dtype), _ptr(dsin), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _check(st, "la_prefill_backward")
+    return grads[0], grads[1], grads[2], dsin
+
+
+def backward_varlen_workspace_size(nseq: int, total_tokens: int, max_seqlen: int, H: int, d: int = D) -> int:
+    return int(lib().la_prefill_backward_varlen_workspace_size(nseq, total_tokens, max_seqlen, H, d))
+
+
+def prefill_backward_varlen(q, k, v, dout, cu_seqlens, max_seqlen: int, state_in=None, dstate_out=None,
+                            grad_dtype=torch.bfloat16, want_dstate_in: bool = True, dq=None, dk=None, dv=None,
+                            workspace=None, stream=None):
+    """la_prefill_backward_varlen on packed [T, H, d] bf16 tensors with device
+    int32 cu_seqlens: gradients of la_prefill_varlen for dL/dout and
+    dL/dstate_out.  Returns (dq, dk, dv, dstate_in or None)."""
+    if q.dim() != 3:
+        raise ValueError("q must be [T, H, d]")
+    T, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("dout", dout)):
+        _need(t, name, torch.bfloat16, (T, H, d))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    nseq = cu_seqlens.numel() - 1
+    if nseq < 0:
+        raise ValueError("cu_seqlens must hold nseq + 1 entries")
+    for name, t in (("state_in", state_in), ("dstate_out", dstate_out)):
+        if t is not None:
+            _need(t, name, torch.float32, (nseq, H, d, d))
+    grads = []
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        if t is None:
+            t = torch.empty((T, H, d), dtype=grad_dtype, device=q.device)
+        _need(t, name, t.dtype, (T, H, d))
+        grads.append(t)
+    if len({t.dtype for t in grads}) != 1:
+        raise TypeError("dq, dk and dv must share one dtype")
+    dsin = torch.empty((nseq, H, d, d), dtype=torch.float32, device=q.device) if want_dstate_in else None
+    ws_bytes = backward_varlen_workspace_size(nseq, T, max_seqlen, H, d)
+    if workspace is None:
+        workspace = _alloc_workspace(ws_bytes, q.device)
+    st = lib().la_prefill_backward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(cu_seqlens), nseq, T,
+                                          int(max_seqlen), H, d, _ptr(state_in), _ptr(dstate_out), _ptr(grads[0]),
+                                          _ptr(grads[1]), _ptr(grads[2]), _out_code(grads[0].dtype), _ptr(dsin),
+                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                          _stream_handle(stream))
+    _check(st, "la_prefill_backward_varlen")
     return grads[0], grads[1], grads[2], dsin
 
 

@@ -372,23 +372,84 @@ la_status launch_transpose(const float *in, float *out, long long nstates, cudaS
     return LA_OK;
 }
 
-// Workspace of la_prefill_backward: one prefill workspace (reused by the
-// two sweeps, which run in stream order) and one [B, H, D, D] fp32 state
-// (S_in transposed).
+// Workspace of la_prefill_backward(_varlen): one prefill workspace (reused
+// by the two sweeps, which run in stream order) and one [nseq, H, D, D] fp32
+// state (S_in transposed).  cu: packed sequences (segment count bounded as
+// for la_prefill_varlen), else nseq sequences of fixed_len tokens.
 struct BwdLayout {
     size_t prefill, st0, total;
 };
 
-BwdLayout bwd_layout(int B, int N, int H) {
+BwdLayout bwd_layout(bool packed, int nseq, int fixed_len, long long T, int H) {
     BwdLayout w;
-    const long long T = (long long)B * N;
-    const int L = choose_seg_len(B, T, H);
-    const size_t pre = ws_layout(gmax_fixed(B, N, L), H).total;
-    const size_t st = (size_t)B * H * la::D * la::D * sizeof(float);
+    const int L = choose_seg_len(nseq, T, H);
+    const long long gmax = packed ? gmax_for(nseq, T, L) : gmax_fixed(nseq, fixed_len, L);
+    const size_t pre = ws_layout(gmax, H).total;
+    const size_t st = (size_t)nseq * H * la::D * la::D * sizeof(float);
     w.prefill = 0;
     w.st0 = round_up(pre, 256);
     w.total = w.st0 + st;
     return w;
+}
+
+// Shared body of la_prefill_backward and la_prefill_backward_varlen.
+la_status backward_impl(const void *q, const void *k, const void *v, const void *dout, const int *cu,
+                        int fixed_len, int nseq, long long T, int max_seqlen, int H, int d,
+                        const float *state_in, const float *dstate_out, void *dq, void *dk, void *dv,
+                        la_dtype grad_dtype, float *dstate_in, void *workspace, size_t ws_bytes,
+                        cudaStream_t stream) {
+    la_status st = check_common(H, d, 0, grad_dtype);
+    if (st != LA_OK) return st;
+    if (nseq < 0 || T < 0 || max_seqlen < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (nseq == 0) return T == 0 ? LA_OK : LA_ERR_INVALID_ARGUMENT;
+    if (T > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return LA_ERR_INVALID_ARGUMENT;
+    const void *ptrs[10] = {q, k, v, dout, dq, dk, dv, state_in, dstate_out, dstate_in};
+    for (const void *p : ptrs)
+        if (p && !aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
+    const size_t esz = grad_dtype == LA_FP32 ? 4 : 2;
+    const size_t n_in = (size_t)T * H * la::D * 2, n_g = (size_t)T * H * la::D * esz;
+    const size_t n_state = (size_t)nseq * H * la::D * la::D * 4;
+    const void *ins[4] = {q, k, v, dout};
+    void *gs[3] = {dq, dk, dv};
+    for (int i = 0; i < 3; ++i) {
+        void *g = gs[i];
+        for (const void *p : ins)
+            if (ranges_overlap(g, n_g, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
+        for (int j = i + 1; j < 3; ++j)
+            if (ranges_overlap(g, n_g, gs[j], n_g)) return LA_ERR_INVALID_ARGUMENT;
+        if (ranges_overlap(g, n_g, dstate_in, n_state) || ranges_overlap(g, n_g, state_in, n_state) ||
+            ranges_overlap(g, n_g, dstate_out, n_state))
+            return LA_ERR_INVALID_ARGUMENT;
+    }
+    if (ranges_overlap(dstate_in, n_state, state_in, n_state) || ranges_overlap(dstate_in, n_state, dstate_out, n_state))
+        return LA_ERR_INVALID_ARGUMENT;
+    const BwdLayout w = bwd_layout(cu != nullptr, nseq, fixed_len, T, H);
+    if (!workspace || ws_bytes < w.total) return LA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return LA_ERR_INVALID_ARGUMENT;
+    for (const void *p : ptrs)
+        if (p && ranges_overlap(workspace, w.total, p, p == q || p == k || p == v || p == dout ? n_in
+                                                       : (p == dq || p == dk || p == dv ? n_g : n_state)))
+            return LA_ERR_INVALID_ARGUMENT;
+    if (cu && ranges_overlap(workspace, w.total, cu, (size_t)(nseq + 1) * sizeof(int))) return LA_ERR_INVALID_ARGUMENT;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *ws_pre = ws + w.prefill;
+    const size_t pre_bytes = w.st0 - w.prefill;
+    float *A = reinterpret_cast<float *>(ws + w.st0);
+
+    // dQ: a forward sweep of (q, k, v) = (dO, V, K) from S_in^T
+    //     dq_t = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T
+    if (state_in && (st = launch_transpose(state_in, A, (long long)nseq * H, stream)) != LA_OK) return st;
+    st = prefill_impl(dout, v, k, cu, fixed_len, nseq, T, max_seqlen, H, d, 0, state_in ? A : nullptr, dq,
+                      grad_dtype, nullptr, ws_pre, pre_bytes, stream);
+    if (st != LA_OK) return st;
+    // dV and dK, sums over the later tokens:
+    //     dv_s = sum_{t >= s} (q_t . k_s) g_t + k_s G,   dk_s = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
+    // one reversed sweep of the paired problems (q, k, v) = (K, Q, dO) and
+    // (q2, v, k) = (V, dO, Q) from G, dK's state being dV's transposed; the
+    // sweep's final state G + sum_t q_t^T g_t is dS_in.
+    return prefill_impl(k, q, dout, cu, fixed_len, nseq, T, max_seqlen, H, d, 0, dstate_out, dv, grad_dtype,
+                        dstate_in, ws_pre, pre_bytes, stream, nullptr, 0, nullptr, v, dk, true);
 }
 
 }  // namespace
@@ -761,66 +822,35 @@ la_status la_kv_aggregate(const void *k, const void *v, int B, int N, int H, int
 size_t la_prefill_backward_workspace_size(int B, int N, int H, int d) {
     (void)d;
     if (B <= 0 || N < 0 || H <= 0) return la::HDR_BYTES;
-    return bwd_layout(B, N, H).total;
+    return bwd_layout(false, B, N, (long long)B * N, H).total;
 }
 
 la_status la_prefill_backward(const void *q, const void *k, const void *v, const void *dout, int B, int N, int H,
                               int d, const float *state_in, const float *dstate_out, void *dq, void *dk, void *dv,
                               la_dtype grad_dtype, float *dstate_in, void *workspace, size_t ws_bytes,
                               cudaStream_t stream) {
-    la_status st = check_common(H, d, 0, grad_dtype);
-    if (st != LA_OK) return st;
     if (B < 0 || N < 0) return LA_ERR_INVALID_ARGUMENT;
-    if (B == 0) return LA_OK;
-    const long long T = (long long)B * N;
-    if (T > 0x7fffffffLL) return LA_ERR_INVALID_ARGUMENT;
-    if (T > 0 && (!q || !k || !v || !dout || !dq || !dk || !dv)) return LA_ERR_INVALID_ARGUMENT;
-    const void *ptrs[10] = {q, k, v, dout, dq, dk, dv, state_in, dstate_out, dstate_in};
-    for (const void *p : ptrs)
-        if (p && !aligned(p, 16)) return LA_ERR_INVALID_ARGUMENT;
-    const size_t esz = grad_dtype == LA_FP32 ? 4 : 2;
-    const size_t n_in = (size_t)T * H * la::D * 2, n_g = (size_t)T * H * la::D * esz;
-    const size_t n_state = (size_t)B * H * la::D * la::D * 4;
-    const void *ins[4] = {q, k, v, dout};
-    void *gs[3] = {dq, dk, dv};
-    for (int i = 0; i < 3; ++i) {
-        void *g = gs[i];
-        for (const void *p : ins)
-            if (ranges_overlap(g, n_g, p, n_in)) return LA_ERR_INVALID_ARGUMENT;
-        for (int j = i + 1; j < 3; ++j)
-            if (ranges_overlap(g, n_g, gs[j], n_g)) return LA_ERR_INVALID_ARGUMENT;
-        if (ranges_overlap(g, n_g, dstate_in, n_state) || ranges_overlap(g, n_g, state_in, n_state) ||
-            ranges_overlap(g, n_g, dstate_out, n_state))
-            return LA_ERR_INVALID_ARGUMENT;
-    }
-    if (ranges_overlap(dstate_in, n_state, state_in, n_state) || ranges_overlap(dstate_in, n_state, dstate_out, n_state))
-        return LA_ERR_INVALID_ARGUMENT;
-    const BwdLayout w = bwd_layout(B, N, H);
-    if (!workspace || ws_bytes < w.total) return LA_ERR_WORKSPACE;
-    if (!aligned(workspace, 256)) return LA_ERR_INVALID_ARGUMENT;
-    for (const void *p : ptrs)
-        if (p && ranges_overlap(workspace, w.total, p, p == q || p == k || p == v || p == dout ? n_in
-                                                       : (p == dq || p == dk || p == dv ? n_g : n_state)))
-            return LA_ERR_INVALID_ARGUMENT;
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    void *ws_pre = ws + w.prefill;
-    const size_t pre_bytes = w.st0 - w.prefill;
-    float *A = reinterpret_cast<float *>(ws + w.st0);
-    const long long nstates = (long long)B * H;
+    if (B == 0) return check_common(H, d, 0, grad_dtype);
+    return backward_impl(q, k, v, dout, nullptr, N, B, (long long)B * N, N, H, d, state_in, dstate_out, dq, dk,
+                         dv, grad_dtype, dstate_in, workspace, ws_bytes, stream);
+}
 
-    // dQ: a forward sweep of (q, k, v) = (dO, V, K) from S_in^T
-    //     dq_t = sum_{s <= t} (g_t . v_s) k_s + g_t S_in^T
-    if (state_in && (st = launch_transpose(state_in, A, nstates, stream)) != LA_OK) return st;
-    st = prefill_impl(dout, v, k, nullptr, N, B, T, N, H, d, 0, state_in ? A : nullptr, dq, grad_dtype, nullptr,
-                      ws_pre, pre_bytes, stream);
-    if (st != LA_OK) return st;
-    // dV and dK, sums over the later tokens:
-    //     dv_s = sum_{t >= s} (q_t . k_s) g_t + k_s G,   dk_s = sum_{t >= s} (g_t . v_s) q_t + v_s G^T
-    // one reversed sweep of the paired problems (q, k, v) = (K, Q, dO) and
-    // (q2, v, k) = (V, dO, Q) from G, dK's state being dV's transposed; the
-    // sweep's final state G + sum_t q_t^T g_t is dS_in.
-    return prefill_impl(k, q, dout, nullptr, N, B, T, N, H, d, 0, dstate_out, dv, grad_dtype, dstate_in, ws_pre,
-                        pre_bytes, stream, nullptr, 0, nullptr, v, dk, true);
+size_t la_prefill_backward_varlen_workspace_size(int nseq, int total_tokens, int max_seqlen, int H, int d) {
+    (void)d;
+    (void)max_seqlen;
+    if (nseq <= 0 || total_tokens < 0 || H <= 0) return la::HDR_BYTES;
+    return bwd_layout(true, nseq, 0, total_tokens, H).total;
+}
+
+la_status la_prefill_backward_varlen(const void *q, const void *k, const void *v, const void *dout,
+                                     const int *cu_seqlens, int nseq, int total_tokens, int max_seqlen, int H,
+                                     int d, const float *state_in, const float *dstate_out, void *dq, void *dk,
+                                     void *dv, la_dtype grad_dtype, float *dstate_in, void *workspace,
+                                     size_t ws_bytes, cudaStream_t stream) {
+    if (!cu_seqlens || nseq < 0 || total_tokens < 0) return LA_ERR_INVALID_ARGUMENT;
+    if (!aligned(cu_seqlens, 4)) return LA_ERR_INVALID_ARGUMENT;
+    return backward_impl(q, k, v, dout, cu_seqlens, 0, nseq, total_tokens, max_seqlen, H, d, state_in, dstate_out,
+                         dq, dk, dv, grad_dtype, dstate_in, workspace, ws_bytes, stream);
 }
 
 la_status la_state_prefix(const float *parts, int count, const float *state_in, float *out, int nstates, int d,

@@ -254,6 +254,35 @@ def test_backward_argument_errors(L):
     assert call(args(B=0)) == la.LA_OK                           # nothing to do
 
 
+def test_backward_varlen_argument_errors(L):
+    """la_prefill_backward_varlen rejects bad arguments before launching."""
+    V = ctypes.c_void_p
+    bad = la.LA_ERR_INVALID_ARGUMENT
+    base = 1 << 32
+    nseq, T, H = 3, 500, 2
+    n = T * H * 128 * 2                          # bytes of one bf16 tensor
+    q, k, v, g = (V(base + i * n) for i in range(4))
+    dq, dk, dv = (V(base + (4 + i) * n) for i in range(3))
+    cu = V(base + 40 * n)
+    ws_size = L.la_prefill_backward_varlen_workspace_size(nseq, T, 300, H, 128)
+    assert ws_size >= L.la_prefill_varlen_workspace_size(nseq, T, 300, H, 128, 0) + nseq * H * 128 * 128 * 4
+    ws = V(base + 64 * n)
+    args = lambda **kw: dict(dict(q=q, k=k, v=v, g=g, cu=cu, nseq=nseq, T=T, maxlen=300, H=H, d=128, sin=None,
+                                  dsout=None, dq=dq, dk=dk, dv=dv, gd=0, dsin=None, ws=ws, wsb=ws_size, s=None), **kw)
+    call = lambda a: L.la_prefill_backward_varlen(*a.values())
+    assert call(args(cu=None)) == bad                            # no cu_seqlens
+    assert call(args(cu=V(base + 40 * n + 2))) == bad            # cu_seqlens misaligned
+    assert call(args(d=64)) == la.LA_ERR_UNSUPPORTED
+    assert call(args(gd=7)) == bad
+    assert call(args(T=-1)) == bad
+    assert call(args(nseq=0)) == bad                             # tokens without sequences
+    assert call(args(dq=g)) == bad                               # a gradient over an input
+    assert call(args(ws=None)) == la.LA_ERR_WORKSPACE
+    assert call(args(wsb=ws_size - 1)) == la.LA_ERR_WORKSPACE
+    assert call(args(ws=cu)) == bad                              # workspace over cu_seqlens
+    assert call(args(nseq=0, T=0)) == la.LA_OK                   # nothing to do
+
+
 def test_host_memory_entry_point_validates_before_any_copy():
     """prefill_from_host refuses unpinned, non-bf16 or non-contiguous host
     inputs before touching a device."""

@@ -5,7 +5,12 @@ and fp32 gradients, sampled heads at 4096 tokens, and at the single-sequence
 prefill workload (B=1, H=64, N=32768) and at 131072 tokens windows of rows
 of sampled heads (the first, the last, and one across the point where the
 reversed sweep switches its state to bf16 hi + lo), with the rest of the
-sequence summarised by the oracle's forward."""
+sequence summarised by the oracle's forward; and the packed-batch form
+(la_prefill_backward_varlen) on packed sequences with empty and ragged
+members, against the oracle and bit for bit against the fixed-length form
+at equal lengths."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -111,3 +116,76 @@ def test_backward_long_sequence_sampled_rows(oracle_mod, N, H, heads, R, mid):
                                   heads=heads, state_in=S, dstate_out=G)
         for name, x, y in zip(("dq", "dk", "dv"), (dq, dk, dv), ref[:3]):
             check_out(to_np(x[0, a:b, heads]), y, bf16_out=True, what=f"N={N} rows {a}-{b} {name}")
+
+
+def _oracle_packed(oracle_mod, q, k, v, g, cu, sin=None, gs=None):
+    return oracle_mod.backward(la_inputs.bits(q), la_inputs.bits(k), la_inputs.bits(v), la_inputs.bits(g), cu,
+                               state_in=None if sin is None else to_np(sin),
+                               dstate_out=None if gs is None else to_np(gs))
+
+
+@pytest.mark.parametrize("lens,H,seg", [([300, 0, 1, 2500, 129, 0, 777], 3, 256), ([128, 256, 1000], 2, 0),
+                                        ([5000, 37, 3100], 2, 1024)])
+@pytest.mark.parametrize("with_states", [False, True])
+def test_backward_varlen_matches_oracle(oracle_mod, lens, H, seg, with_states):
+    """la_prefill_backward_varlen on packed batches with empty, one-token and
+    ragged sequences, several segments per sequence (the reversed sweep
+    starts at each sequence's last, partial segment), with and without
+    carried-in states and state gradients: fp32 gradients and dS_in of every
+    sequence against the oracle's gradients of the packed forward."""
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    T, nseq = int(cu[-1]), len(lens)
+    q, k, v = la_inputs.qkv((T, H, D), seed=980 + T, device="cuda")
+    g, _, _ = la_inputs.qkv((T, H, D), seed=981 + T, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(982)
+    sin = torch.randn((nseq, H, D, D), generator=gen, device="cuda") * 0.2 if with_states else None
+    gs = torch.randn((nseq, H, D, D), generator=gen, device="cuda") * 0.05 if with_states else None
+    if seg:
+        la.set_segment_len(seg)
+    got = la.prefill_backward_varlen(q, k, v, g, torch.from_numpy(cu).cuda(), max(lens), state_in=sin,
+                                     dstate_out=gs, grad_dtype=torch.float32)
+    assert la.get_device_status() == la.LA_OK
+    ref = _oracle_packed(oracle_mod, q, k, v, g, cu, sin, gs)
+    what = f"lens={lens} seg={seg} states={with_states}"
+    for name, x, y in zip(("dq", "dk", "dv"), got[:3], ref[:3]):
+        check_out(to_np(x), y, bf16_out=False, what=f"{what} {name}")
+    check_state(to_np(got[3]), ref[3], what=f"{what} dS_in")
+    for i, n in enumerate(lens):  # an empty sequence passes its state gradient through
+        if n == 0:
+            assert torch.equal(got[3][i], gs[i] if gs is not None else torch.zeros_like(got[3][i]))
+
+
+def test_backward_varlen_equal_lengths_match_fixed():
+    """Equal lengths: the packed entry point builds the same segments as the
+    fixed-length one, so its gradients are the same bits."""
+    B, N, H = 3, 700, 2
+    q, k, v, g = _inputs(B, N, H, seed=990)
+    la.set_segment_len(256)
+    fixed = la.prefill_backward(q, k, v, g)
+    cu = torch.from_numpy(la_inputs.cu_seqlens_from_lengths([N] * B)).cuda()
+    flat = lambda t: t.reshape(B * N, H, D)  # noqa: E731
+    packed = la.prefill_backward_varlen(flat(q), flat(k), flat(v), flat(g), cu, N)
+    assert la.get_device_status() == la.LA_OK
+    for x, y in zip(fixed[:3], packed[:3]):
+        assert torch.equal(flat(x), y)
+    assert torch.equal(fixed[3], packed[3])
+
+
+def test_backward_varlen_rejects_a_bad_table():
+    """A cu_seqlens table that does not end at the token count is refused on
+    the device: the status word says so and no gradient is written."""
+    lens = [100, 200]
+    T, H = 300, 2
+    q, k, v = la_inputs.qkv((T, H, D), seed=995, device="cuda")
+    bad = torch.tensor([0, 100, 250], dtype=torch.int32, device="cuda")
+    grads = [torch.full((T, H, D), 7.0, dtype=torch.float32, device="cuda") for _ in range(3)]
+    dsin = torch.full((2, H, D, D), 7.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(la.backward_varlen_workspace_size(2, T, max(lens), H), dtype=torch.uint8, device="cuda")
+    L = la.lib()
+    P = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    st = L.la_prefill_backward_varlen(P(q), P(k), P(v), P(q), P(bad), 2, T, 200, H, D, None, None, P(grads[0]),
+                                      P(grads[1]), P(grads[2]), la.LA_FP32, P(dsin), P(ws), ws.numel(),
+                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == la.LA_OK                           # the table is checked on the device
+    assert la.get_device_status() == la.LA_ERR_INVALID_ARGUMENT
+    assert all(torch.all(x == 7.0) for x in grads) and torch.all(dsin == 7.0)
