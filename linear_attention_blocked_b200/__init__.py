@@ -18,6 +18,7 @@ ABI (include/lightning_attn.h).  Entry points:
   lasp_prefill(q, k, v, group=...)           sequence parallelism across ranks (seqpar.py)
   lasp_prefill_varlen(q, k, v, cu, bounds)   the same for a packed batch cut at any token
   lasp_prefill_backward(q, k, v, dout, ...)  gradients of lasp_prefill across ranks
+  lasp_prefill_backward_varlen(...)          gradients of lasp_prefill_varlen across ranks
   prefill_backward(q, k, v, dout, ...)       la_prefill_backward: dq, dk, dv, dS_in
   prefill_backward_varlen(q, k, v, dout, cu, ...)  la_prefill_backward_varlen: the same per packed sequence
   prefill_from_host(q, k, v, ...)            la_prefill of pinned host tensors, chunks pipelined
@@ -33,7 +34,8 @@ from ._binding import (D, DEFAULT_BLOCK, backward_workspace_size, backward_varle
                        prefill, prefill_varlen, prefill_varlen_slots,
                        set_segment_len, set_wait_limit_ns, state_prefix, status_string,
                        varlen_workspace_size, workspace_size)
-from .seqpar import (lasp_prefill, lasp_prefill_backward, lasp_prefill_varlen, plan_varlen_rank,  # noqa: F401,E402
+from .seqpar import (lasp_prefill, lasp_prefill_backward, lasp_prefill_backward_varlen,  # noqa: F401,E402
+                     lasp_prefill_varlen, plan_varlen_rank,
                      split_tokens)
 from .serving import BatchPlan, plan_batch  # noqa: F401,E402
 from .streaming import make_buffers, prefill_from_host  # noqa: F401,E402

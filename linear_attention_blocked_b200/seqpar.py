@@ -28,7 +28,11 @@ Gradients across ranks (lasp_prefill_backward): a rank's tokens see the
 earlier ranks only through the state they hand on and the later ranks only
 through that state's gradient, so each rank gathers two d x d sums per
 (sequence, head) from every rank and runs la_prefill_backward on its own
-tokens from the two.
+tokens from the two.  For packed batches (lasp_prefill_backward_varlen)
+only the sequence carried into a rank's range and the one still open at its
+end cross rank boundaries, so each rank contributes the forward sum of its
+open tail and the state-gradient sum of its carried-in head, and runs
+la_prefill_backward_varlen on its own tokens.
 
 The device steps run in the CUDA library (la_kv_aggregate, la_state_prefix,
 la_prefill, la_prefill_varlen, la_prefill_backward); the collective is
@@ -70,6 +74,12 @@ class DeviceOps:
     def prefill_varlen(q, k, v, cu_seqlens, max_seqlen, state_in, out_dtype):
         cu = torch.from_numpy(np.ascontiguousarray(cu_seqlens, dtype=np.int32)).to(q.device)
         return _binding.prefill_varlen(q, k, v, cu, max_seqlen, state_in=state_in, out_dtype=out_dtype)
+
+    @staticmethod
+    def prefill_backward_varlen(q, k, v, dout, cu_seqlens, max_seqlen, state_in, dstate_out, grad_dtype):
+        cu = torch.from_numpy(np.ascontiguousarray(cu_seqlens, dtype=np.int32)).to(q.device)
+        return _binding.prefill_backward_varlen(q, k, v, dout, cu, max_seqlen, state_in=state_in,
+                                                dstate_out=dstate_out, grad_dtype=grad_dtype)
 
 
 def lasp_prefill(q, k, v, group=None, state_in=None, out_dtype=torch.bfloat16, want_state: bool = True,
@@ -171,6 +181,15 @@ class VarlenRankPlan:
     @property
     def n_local(self) -> int:
         return self.seq1 - self.seq0
+
+    @property
+    def starts_here(self) -> np.ndarray:
+        """bool [seq1 - seq0]: that sequence's first token is on this rank (so
+        its state gradient dS_in is formed here)."""
+        first = np.ones(self.n_local, bool)
+        if self.n_local:
+            first[0] = self.carried_from == self.rank
+        return first
 
 
 def plan_varlen_rank(cu_seqlens, bounds, rank: int) -> VarlenRankPlan:
@@ -277,3 +296,86 @@ def lasp_prefill_varlen(q, k, v, cu_seqlens, bounds, group=None, state_in=None, 
     dist.all_gather_into_tensor(gathered, local.contiguous(), group=group)
     out, st = varlen_local_scan(plan, q, k, v, gathered.view(world, H, d, d), state_in, out_dtype, ops)
     return out, st, plan
+
+
+def varlen_backward_local_sums(plan: VarlenRankPlan, q, k, v, dout, ops=DeviceOps):
+    """Step 1 of lasp_prefill_backward_varlen on one rank: A_r = sum of
+    k_t^T v_t over the sequence still open at the end of its range (the
+    forward prefix later ranks need) and B_r = sum of q_t^T g_t over the
+    sequence carried into its range (the state gradient earlier ranks need);
+    zero where there is no such sequence.  Both [H, d, d]."""
+    _, H, d = q.shape
+    if plan.open_tail is not None:
+        a, b = plan.open_tail
+        A = ops.kv_aggregate(k[a:b].reshape(1, b - a, H, d), v[a:b].reshape(1, b - a, H, d))[0]
+    else:
+        A = ops.kv_aggregate(k[0:0].reshape(1, 0, H, d), v[0:0].reshape(1, 0, H, d))[0]
+    n0 = int(plan.local_cu[1]) if plan.n_local and plan.carried_from < plan.rank else 0
+    B = ops.kv_aggregate(q[0:n0].reshape(1, n0, H, d), dout[0:n0].reshape(1, n0, H, d))[0]
+    return A, B
+
+
+def varlen_backward_local_grads(plan: VarlenRankPlan, cu_seqlens, bounds, q, k, v, dout, a_parts, b_parts,
+                                state_in=None, dstate_out=None, grad_dtype=torch.bfloat16, ops=DeviceOps):
+    """Step 3 on one rank, given every rank's two sums (a_parts, b_parts:
+    [W, H, d, d], rank order).  The sequence carried into the range starts
+    from its carried-in state plus the A of the ranks it spanned before; the
+    sequence still open at the end of the range ends with its state gradient
+    plus the B of the ranks it spans after; every other sequence is local.
+    Returns (dq, dk, dv for the rank's tokens, dS_in [seq1 - seq0, H, d, d]):
+    row i is the whole dS_in of global sequence plan.seq0 + i where
+    plan.starts_here[i]."""
+    _, H, d = q.shape
+    if plan.n_local == 0:
+        e = q.new_empty((q.shape[0], H, d), dtype=grad_dtype)
+        return e, e.clone(), e.clone(), a_parts.new_empty((0, H, d, d))
+    r, cf = plan.rank, plan.carried_from
+    sin = a_parts.new_empty((plan.n_local, H, d, d))
+    s0 = None if state_in is None else state_in[plan.seq0]
+    ops.state_prefix(a_parts[cf:r] if cf < r else None, r - cf, s0, sin[0])
+    if plan.n_local > 1:
+        rest = None if state_in is None else state_in[plan.seq0 + 1:plan.seq1]
+        ops.state_prefix(None, 0, rest, sin[1:])
+    gout = a_parts.new_empty((plan.n_local, H, d, d))
+    last = plan.seq1 - 1
+    head = None if dstate_out is None else dstate_out[plan.seq0:last]
+    if plan.n_local > 1:
+        ops.state_prefix(None, 0, head, gout[:-1])
+    g_last = None if dstate_out is None else dstate_out[last]
+    if plan.open_tail is not None:
+        # the ranks after this one up to the one holding the sequence's last token
+        bd = np.asarray(bounds, dtype=np.int64)
+        end = int(np.searchsorted(bd[1:], int(np.asarray(cu_seqlens)[last + 1]), side="left"))
+        ops.state_prefix(b_parts[r + 1:end + 1], end - r, g_last, gout[-1])
+    else:
+        ops.state_prefix(None, 0, g_last, gout[-1])
+    return ops.prefill_backward_varlen(q, k, v, dout, plan.local_cu, plan.max_seqlen, sin, gout, grad_dtype)
+
+
+def lasp_prefill_backward_varlen(q, k, v, dout, cu_seqlens, bounds, group=None, state_in=None, dstate_out=None,
+                                 grad_dtype=torch.bfloat16, ops=DeviceOps):
+    """Gradients of lasp_prefill_varlen on this rank's range [bounds[r],
+    bounds[r+1]) of a packed batch, for dL/dout (this rank's rows) and
+    dL/dS_out of every sequence's final state (dstate_out, fp32 [nseq, H, d,
+    d], the same on every rank, or None).  Returns (dq, dk, dv [tokens, H,
+    d], dS_in [seq1 - seq0, H, d, d], plan): row i of dS_in is the whole
+    dS_in of global sequence plan.seq0 + i where plan.starts_here[i].  Two
+    AllGathers of one d x d matrix per head."""
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if len(bounds) != world + 1:
+        raise ValueError("bounds must hold world + 1 entries")
+    plan = plan_varlen_rank(cu_seqlens, bounds, rank)
+    if q.dim() != 3 or q.shape[0] != plan.tok1 - plan.tok0:
+        raise ValueError("q must be [this rank's tokens, H, d]")
+    _, H, d = q.shape
+    a, b = varlen_backward_local_sums(plan, q, k, v, dout, ops)
+    parts = []
+    for local in (a, b):
+        gathered = local.new_empty((world * H, d, d))  # rank-major
+        dist.all_gather_into_tensor(gathered, local.contiguous(), group=group)
+        parts.append(gathered.view(world, H, d, d))
+    dq, dk, dv, dsin = varlen_backward_local_grads(plan, cu_seqlens, bounds, q, k, v, dout, parts[0], parts[1],
+                                                   state_in, dstate_out, grad_dtype, ops)
+    return dq, dk, dv, dsin, plan
+

@@ -151,6 +151,45 @@ def test_emulated_ranks_on_a_packed_batch(oracle_mod, lens, world):
     check_state(to_np(final), rst, what="final states")
 
 
+@pytest.mark.parametrize("lens,world", [([300, 0, 1290, 77, 0, 2100, 1, 129], 3), ([40, 3000, 60], 4)])
+def test_emulated_ranks_gradients_on_a_packed_batch(oracle_mod, lens, world):
+    """The gradients of a packed batch cut evenly into ranges at arbitrary
+    tokens, through the two steps lasp_prefill_backward_varlen runs on each
+    rank (a stack of the local sums standing in for the AllGathers), against
+    the oracle's gradients of the whole batch; each sequence's dS_in is taken
+    from the rank where it starts."""
+    from linear_attention_blocked_b200 import seqpar
+    H = 2
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    T = int(cu[-1])
+    q, k, v = la_inputs.qkv((T, H, D), seed=430 + world, device="cuda")
+    g, _, _ = la_inputs.qkv((T, H, D), seed=431 + world, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(432)
+    sin = torch.randn((len(lens), H, D, D), generator=gen, device="cuda") * 0.1
+    gs = torch.randn((len(lens), H, D, D), generator=gen, device="cuda") * 0.05
+    bounds = seqpar.split_tokens(T, world)
+    plans = [seqpar.plan_varlen_rank(cu, bounds, r) for r in range(world)]
+    rng = lambda t, p: t[p.tok0:p.tok1].contiguous()  # noqa: E731
+    sums = [seqpar.varlen_backward_local_sums(p, rng(q, p), rng(k, p), rng(v, p), rng(g, p)) for p in plans]
+    a_parts = torch.stack([a for a, _ in sums])
+    b_parts = torch.stack([b for _, b in sums])
+    grads = [[], [], []]
+    dsin = torch.full((len(lens), H, D, D), float("nan"), device="cuda")
+    for p in plans:
+        dq, dk, dv, ds = seqpar.varlen_backward_local_grads(p, cu, bounds, rng(q, p), rng(k, p), rng(v, p),
+                                                            rng(g, p), a_parts, b_parts, sin, gs, torch.float32)
+        for lst, x in zip(grads, (dq, dk, dv)):
+            lst.append(x)
+        for i in np.nonzero(p.starts_here)[0]:
+            dsin[p.seq0 + i] = ds[i]
+    assert la.get_device_status() == la.LA_OK
+    ref = oracle_mod.backward(*(la_inputs.bits(t) for t in (q, k, v, g)), cu, state_in=to_np(sin),
+                              dstate_out=to_np(gs))
+    for name, lst, y in zip(("dq", "dk", "dv"), grads, ref[:3]):
+        check_out(to_np(torch.cat(lst, 0)), y, bf16_out=False, what=f"packed {name}")
+    check_state(to_np(dsin), ref[3], what="packed dS_in")
+
+
 def test_emulated_ranks_gradients(oracle_mod):
     """Gradients across three ranks (parts of 700, 1500 and 829 tokens), run
     one after the other on this GPU through the same two steps
