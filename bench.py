@@ -519,6 +519,8 @@ def run_cuda(args, world, rank, local):
     agg = bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world) if want("aggregate") else None
     # ---------------- gradients of the prefill on the same q, k, v
     bwd = bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world) if want("backward") else None
+    # ---------------- gradients of the packed varlen batch
+    bwd_v = bench_backward_varlen(la, dev, stream, args, hbm_peak, world, rank) if want("backward_varlen") else None
 
     status2 = la.get_device_status()
     if rank != 0:
@@ -564,6 +566,7 @@ def run_cuda(args, world, rank, local):
         "long_context": longc,
         "kv_aggregate": agg,
         "backward": bwd,
+        "backward_varlen": bwd_v,
         "cpu_baseline": cpu,
         "device_status": [int(status), int(status2)],
     }
@@ -597,6 +600,50 @@ def bench_kv_aggregate(la, dev, stream, k, v, args, hbm_peak, world):
                          "traffic": recorded_traffic("la_kv_aggregate_kernel", "aggregate_B1_H64_N32768"),
                          "bytes_per_launch": byts,
                          "duration": "CUDA events around each la_kv_aggregate call (aggregate + reduce)"}}
+
+
+def bench_backward_varlen(la, dev, stream, args, hbm_peak, world, rank):
+    """la_prefill_backward_varlen on the packed varlen workload (8 sequences
+    of lengths drawn in [1024, 65536], H=64; random dout), bf16 gradients."""
+    lens = la_inputs.varlen_lengths(8, 1024, 65536, seed=3)
+    cu = la_inputs.cu_seqlens_from_lengths(lens)
+    T = int(cu[-1])
+    q, k, v = la_inputs.qkv((T, H, D), seed=303 + rank, device=dev)
+    g, _, _ = la_inputs.qkv((T, H, D), seed=313 + rank, device=dev)
+    cu_d = torch.from_numpy(cu).to(dev)
+    grads = [torch.empty_like(q) for _ in range(3)]
+    ws = torch.empty(la.backward_varlen_workspace_size(len(lens), T, int(lens.max()), H, D), dtype=torch.uint8,
+                     device=dev)
+
+    def call():
+        la.prefill_backward_varlen(q, k, v, g, cu_d, int(lens.max()), dq=grads[0], dk=grads[1], dv=grads[2],
+                                   workspace=ws)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    steps = max(5, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    byts = backward_bytes(T * H)
+    gbs = byts / (ms * 1e-3) / 1e9
+    del q, k, v, g, grads, ws
+    return {"workload": f"packed varlen backward, 8 seqs U[1024, 65536] (seed 3), {T} tokens, H=64, d=128, "
+                        "bf16 dq/dk/dv + fp32 dS_in",
+            "tok_s": T / (ms * 1e-3), "ms_per_call": ms, "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                         "kernel": "la_prefill_kernel (dQ sweep + reversed paired dK/dV sweep)",
+                         # DRAM bytes of both sweeps of one call
+                         "traffic": recorded_traffic("la_prefill_kernel", "backward_varlen_S8_H64"),
+                         "bytes_per_launch": byts,
+                         "duration": "CUDA events around each la_prefill_backward_varlen call (two schedule kernels "
+                                     "+ two sweeps)"}}
 
 
 def bench_backward(la, dev, stream, q, k, v, args, hbm_peak, world):
@@ -863,7 +910,7 @@ def main():
                     help="approximate total CPU time of the --impl reference run")
     ap.add_argument("--legs", default="",
                     help="comma-separated subset of the legs after the main prefill step to run (e2e, decode, "
-                         "block64, block256, decay, varlen, long, aggregate, backward); default all")
+                         "block64, block256, decay, varlen, long, aggregate, backward, backward_varlen); default all")
     args = ap.parse_args()
     if args.impl == "reference":
         # the oracle runs on the host cores of rank 0 only; no process group needed
