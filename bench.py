@@ -65,7 +65,7 @@ def prefill_alg_flops(tok_heads: int, block: int) -> int:
     return tok_heads * (2 * (block + 1) * D + 4 * D * D)
 
 
-def prefill_survey_exec_flops(tok_heads: int, block: int) -> int:
+def prefill_dense_flops(tok_heads: int, block: int) -> int:
     """The dense count 4*Bk*d + 4*d^2 per token-head (full score and P V tiles,
     one Q S and one K^T V), independent of how the kernel splits the work."""
     return tok_heads * (4 * block * D + 4 * D * D)
@@ -466,7 +466,7 @@ def run_cuda(args, world, rank, local):
     L = la.last_segment_len()
     f_alg = prefill_alg_flops(tok_heads, BLOCK)
     f_mma = prefill_mma_flops([N] * B, H, L, want_state=True, block=BLOCK)
-    f_dense = prefill_survey_exec_flops(tok_heads, BLOCK)
+    f_dense = prefill_dense_flops(tok_heads, BLOCK)
     achieved_gbs = byts / (ms * 1e-3) / 1e9
 
     legs = set(args.legs.split(",")) if args.legs else None
@@ -764,7 +764,7 @@ def bench_prefill_block(la, dev, stream, q, k, v, block, args, hbm_peak, tc_peak
     gbs = byts / (ms * 1e-3) / 1e9
     f_mma = prefill_mma_flops([N] * B, H, L, want_state=True, block=block)
     f_alg = prefill_alg_flops(B * N * H, block)
-    f_dense = prefill_survey_exec_flops(B * N * H, block)
+    f_dense = prefill_dense_flops(B * N * H, block)
     del out, st, ws
     return {"workload": f"causal prefill B=1 H=64 N=32768 d=128 at row blocks of {block}",
             "ms_per_call": ms, "steps": steps, "segment_len": L,

@@ -41,9 +41,9 @@ def test_backward_aggregate_and_decode_bytes():
 def test_blocked_flop_definitions():
     th, bk = 1000, 128
     assert bench.prefill_alg_flops(th, bk) == th * (2 * 129 * D + 4 * D * D)
-    assert bench.prefill_survey_exec_flops(th, bk) == th * (4 * 128 * D + 4 * D * D)
+    assert bench.prefill_dense_flops(th, bk) == th * (4 * 128 * D + 4 * D * D)
     # the dense count exceeds the blocked definition by the masked half of each score tile
-    assert bench.prefill_survey_exec_flops(th, bk) - bench.prefill_alg_flops(th, bk) == th * 2 * (bk - 1) * D
+    assert bench.prefill_dense_flops(th, bk) - bench.prefill_alg_flops(th, bk) == th * 2 * (bk - 1) * D
 
 
 @pytest.mark.parametrize("lengths,heads,seg,want,block,units", [  # units per head
