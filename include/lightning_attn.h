@@ -51,7 +51,7 @@ extern "C" {
 typedef enum {
     LA_OK = 0,
     LA_ERR_INVALID_ARGUMENT = 1, /* bad pointer, shape, alignment or dtype        */
-    LA_ERR_UNSUPPORTED = 2,      /* valid but not built (d != 128, block != 128)  */
+    LA_ERR_UNSUPPORTED = 2,      /* valid but not built (d != 128, block not 0/64/128/256, decay at block 64 or 256) */
     LA_ERR_CUDA = 3,             /* a CUDA runtime call or launch failed          */
     LA_ERR_TIMEOUT = 4,          /* a bounded device-side wait ran out            */
     LA_ERR_WORKSPACE = 5         /* workspace missing or smaller than required    */
@@ -228,8 +228,10 @@ LA_API la_status la_mixed_step(const void *q, const void *k, const void *v,
  * chunk_tokens tokens pipelined over three streams: chunk c+1 is copied in
  * on copy_in while chunk c is scanned on compute and chunk c-1 is copied out
  * on copy_out.  Each chunk is an la_prefill from the state the previous
- * chunk left (the state-carry identity of the recurrence: the result equals
- * one prefill of the whole sequence, to rounding).
+ * chunk left.  This is the state-carry identity of the recurrent form
+ * ("MiniMax-01技术报告解读", §2.2 线性注意力: the running KV state summarises
+ * every earlier token), so the result equals one prefill of the whole
+ * sequence, to rounding.
  *
  *   q, k, v     PINNED HOST bf16 [B, N, H, d] (cudaHostAlloc / registered).
  *   out         PINNED HOST [B, N, H, d] in out_dtype.
